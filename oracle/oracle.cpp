@@ -1,0 +1,404 @@
+// Oracle for the blockwise-scaled FP8 linear layer — TEST INFRASTRUCTURE ONLY.
+//
+// A plain, slow, CPU implementation of what the library computes, written
+// from the pages' statement of the method and from the definitions of the
+// formats involved.  It shares no code, header, table or constant with the
+// CUDA library and must never be linked into it: only the tests, the smoke
+// check and the benchmark's CPU-baseline leg load it.
+//
+// Sources (page title, section):
+//  [P1] "NVIDIA NeMo RL erreicht 48% Geschwindigkeitssteigerung mit End-to-End
+//       FP8-Präzisionstraining", section "Der technische Durchbruch": the
+//       recipe quantizes to E4M3 with one scale per 128x128 weight block and
+//       one per 1x128 activation block; linear layers do FP8 math.
+//       Section "Leistungsgewinne in der Praxis": scales are recalibrated
+//       after every training step.  Section "Warum dies für die KI-Ökonomie
+//       wichtig ist": optional power-of-2 scale factors.
+//  [P2] "FP8 Trainingsinfrastructuur", section "Het landschap van numerieke
+//       precisie": E4M3 has 4 exponent bits, 3 mantissa bits and values up to
+//       +-448.
+//
+// Readings taken where the pages are silent (each is listed in the design doc):
+//  * block scale s = fp32(amax / 448) (current scaling), s = 1 for an
+//    all-zero block;
+//  * power-of-2 mode: s = 2^e with e the smallest integer such that
+//    amax <= 448 * 2^e, clamped to [-127, 127]; s = 1 for an all-zero block;
+//  * codes: q = E4M3_RNE_satfinite( fp32( fp32(x) / s ) ) — IEEE fp32
+//    division, then round-to-nearest-even onto the E4M3 grid, magnitudes
+//    beyond 448 saturate to 448, the sign of zero is kept;
+//  * GEMM reference: fp64 sum of products of the dequantized operands.
+//
+// Parity status: every function here is pinned by tests/test_oracle_*.py
+// (exhaustive code table, closed-form points, library cross-checks,
+// hand-worked blocks, invariants, brute force).  No function is unpinned.
+//
+// Build: g++ -O2 -std=c++17 -fPIC -shared -ffp-contract=off -fopenmp (no
+// -ffast-math: IEEE division and subnormals must be kept).  OpenMP only
+// splits independent blocks / output elements across threads; no value's
+// arithmetic changes with the thread count.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cstdlib>
+
+namespace {
+
+// ---------------------------------------------------------------- bf16 ----
+// A bf16 value is the upper 16 bits of an IEEE binary32 value.
+float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// fp32 -> bf16 with round-to-nearest-even (NaN kept as a quiet NaN).
+uint16_t float_to_bf16_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof u);
+  if (std::isnan(f)) return static_cast<uint16_t>((u >> 16) | 0x40);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return static_cast<uint16_t>(u >> 16);
+}
+
+// ---------------------------------------------------------------- E4M3 ----
+// E4M3 [P2]: sign bit, 4 exponent bits, 3 mantissa bits, largest value 448.
+// 448 = 1.75 * 2^8 is exponent field 15 with mantissa 110, so the exponent
+// bias is 7; exponent field 15 with mantissa 111 is NaN (no infinities).
+//   field e in 1..15: (1 + m/8) * 2^(e-7)
+//   field e == 0    : (m/8) * 2^(1-7) = m * 2^-9   (subnormals)
+double e4m3_decode(uint8_t code) {
+  int sign = (code >> 7) & 1;
+  int e = (code >> 3) & 0xF;
+  int m = code & 0x7;
+  if (e == 15 && m == 7) return std::nan("");
+  double mag;
+  if (e == 0)
+    mag = std::ldexp(static_cast<double>(m), -9);
+  else
+    mag = std::ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+// Round a finite fp32 value to the E4M3 grid, ties to even, saturating to
+// +-448.  The grid spacing in [2^E, 2^(E+1)) is 2^(E-3) for E >= -6 and 2^-9
+// below 2^-6 (the subnormal range), so v / spacing is an integer k whose
+// parity is the parity of the mantissa field.  Rounding k to the nearest
+// integer with ties to even is therefore the E4M3 round-to-nearest-even.
+uint8_t e4m3_encode(float v) {
+  uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  if (std::isnan(v)) return static_cast<uint8_t>(sign | 0x7F);
+  double a = std::fabs(static_cast<double>(v));
+  if (a >= 448.0) return static_cast<uint8_t>(sign | 0x7E);  // saturate
+  if (a == 0.0) return sign;
+  int E;  // a = f * 2^E2 with f in [0.5,1)  =>  a in [2^(E2-1), 2^E2)
+  std::frexp(a, &E);
+  E -= 1;                          // a in [2^E, 2^(E+1))
+  int spacing_exp = (E < -6) ? -9 : E - 3;
+  double k = std::ldexp(a, -spacing_exp);      // exact (power-of-2 scaling)
+  double r = std::nearbyint(k);                // default mode: ties to even
+  // r * 2^spacing_exp is the rounded magnitude, never above 448.
+  //  subnormal range: value r * 2^-9, r in 0..8; r == 8 is 2^-6, the first
+  //    normal (field 1, mantissa 0), which is also code 8;
+  //  normal range: value (r/8) * 2^E, r in 8..16; the code is
+  //    (E + 7) * 8 + (r - 8), and r == 16 carries into the next exponent.
+  long r_int = static_cast<long>(r);
+  if (r_int == 0) return sign;
+  long code = (E < -6) ? r_int : (E + 7) * 8 + (r_int - 8);
+  return static_cast<uint8_t>(sign | code);
+}
+
+// ------------------------------------------------------------ block scale --
+constexpr int MODE_FP32 = 0;
+constexpr int MODE_POW2 = 1;
+
+float block_scale(float amax, int mode) {
+  if (amax == 0.0f) return 1.0f;
+  if (mode == MODE_FP32) return amax / 448.0f;  // IEEE fp32 division
+  // Power of two: the smallest e with amax <= 448 * 2^e (found by search,
+  // which is the definition), clamped to the UE8M0-representable [-127,127].
+  int e = -127;
+  while (e < 127 && static_cast<double>(amax) > std::ldexp(448.0, e)) ++e;
+  return static_cast<float>(std::ldexp(1.0, e));
+}
+
+uint8_t quant_one(uint16_t xb, float s) {
+  float x = bf16_bits_to_float(xb);
+  float t = x / s;  // IEEE fp32 division, round to nearest even
+  return e4m3_encode(t);
+}
+
+}  // namespace
+
+extern "C" {
+
+double orc_e4m3_decode(uint8_t code) { return e4m3_decode(code); }
+uint8_t orc_e4m3_encode(float v) { return e4m3_encode(v); }
+float orc_block_scale(float amax, int mode) { return block_scale(amax, mode); }
+float orc_bf16_to_float(uint16_t b) { return bf16_bits_to_float(b); }
+uint16_t orc_float_to_bf16(float f) { return float_to_bf16_bits(f); }
+
+void orc_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(v[i]);
+}
+
+// Activation quantization, 1x128 blocks [P1 "Der technische Durchbruch"].
+//   x      : bf16 bits, row-major [M][ldx] (first K columns used)
+//   q_row  : [M][K] codes; s_row : [K/128][M] scales (chunk-major)
+//   q_col  : [K][M] codes of the column-wise copy, whose blocks are 128
+//            consecutive rows of one column; s_col : [M/128][K].
+//   The column-wise copy is quantized from x itself, not from q_row.
+//   q_col/s_col may be null (row-wise only).
+void orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                         int mode, uint8_t* q_row, float* s_row,
+                         uint8_t* q_col, float* s_col) {
+  const int64_t nK = K / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t kb = 0; kb < nK; ++kb) {
+      float amax = 0.0f;
+      for (int64_t j = 0; j < 128; ++j) {
+        float a = std::fabs(bf16_bits_to_float(x[m * ldx + kb * 128 + j]));
+        if (a > amax) amax = a;
+      }
+      float s = block_scale(amax, mode);
+      s_row[kb * M + m] = s;
+      for (int64_t j = 0; j < 128; ++j)
+        q_row[m * K + kb * 128 + j] = quant_one(x[m * ldx + kb * 128 + j], s);
+    }
+  }
+  if (!q_col) return;
+  const int64_t nM = M / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < K; ++k) {
+    for (int64_t mb = 0; mb < nM; ++mb) {
+      float amax = 0.0f;
+      for (int64_t i = 0; i < 128; ++i) {
+        float a = std::fabs(bf16_bits_to_float(x[(mb * 128 + i) * ldx + k]));
+        if (a > amax) amax = a;
+      }
+      float s = block_scale(amax, mode);
+      s_col[mb * K + k] = s;
+      for (int64_t i = 0; i < 128; ++i)
+        q_col[k * M + mb * 128 + i] = quant_one(x[(mb * 128 + i) * ldx + k], s);
+    }
+  }
+}
+
+// Weight quantization, 128x128 blocks [P1 "Der technische Durchbruch"].
+//   w  : bf16 bits [N][ldw]; q : [N][K]; s : [N/128][K/128];
+//   qT : [K][N], the exact byte transpose of q (may be null).
+void orc_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K,
+                              int64_t ldw, int mode, uint8_t* q, float* s,
+                              uint8_t* qT) {
+  const int64_t nN = N / 128, nK = K / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t nb = 0; nb < nN; ++nb) {
+    for (int64_t kb = 0; kb < nK; ++kb) {
+      float amax = 0.0f;
+      for (int64_t i = 0; i < 128; ++i)
+        for (int64_t j = 0; j < 128; ++j) {
+          float a = std::fabs(
+              bf16_bits_to_float(w[(nb * 128 + i) * ldw + kb * 128 + j]));
+          if (a > amax) amax = a;
+        }
+      float sc = block_scale(amax, mode);
+      s[nb * nK + kb] = sc;
+      for (int64_t i = 0; i < 128; ++i)
+        for (int64_t j = 0; j < 128; ++j)
+          q[(nb * 128 + i) * K + kb * 128 + j] =
+              quant_one(w[(nb * 128 + i) * ldw + kb * 128 + j], sc);
+    }
+  }
+  if (!qT) return;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) qT[k * N + n] = q[n * K + k];
+}
+
+// Scale of operand B for output column n at K-chunk kb, per GEMM kind:
+//   kind 0 (fprop): 128x128 block grid [N/128][K/128]
+//   kind 1 (dgrad): the weight's own grid, read transposed: [K/128][N/128]
+//   kind 2 (wgrad): 1x128 blocks along the contraction, [K/128][N]
+static double b_scale(int kind, const float* sB, int64_t N, int64_t K,
+                      int64_t n, int64_t kb) {
+  if (kind == 0) return sB[(n / 128) * (K / 128) + kb];
+  if (kind == 1) return sB[kb * (N / 128) + n / 128];
+  return sB[kb * N + n];
+}
+
+// One output element of the GEMM reference over K-chunks [kb0, kb1):
+// sum_k (qA[m][k] * sA[k/128][m]) * (qB[n][k] * sB(n, k/128)) in fp64 from
+// the dequantized operands, and sum_k |a * b|.
+static void ref_element(int kind, int64_t M, int64_t N, int64_t K,
+                        const uint8_t* A, const float* sA, const uint8_t* B,
+                        const float* sB, int64_t kb0, int64_t kb1, int64_t m,
+                        int64_t n, double* y, double* yabs) {
+  double acc = 0.0, aacc = 0.0;
+  for (int64_t kb = kb0; kb < kb1; ++kb) {
+    double sa = sA[kb * M + m];
+    double sb = b_scale(kind, sB, N, K, n, kb);
+    for (int64_t j = 0; j < 128; ++j) {
+      int64_t k = kb * 128 + j;
+      double a = e4m3_decode(A[m * K + k]) * sa;
+      double b = e4m3_decode(B[n * K + k]) * sb;
+      acc += a * b;
+      aacc += std::fabs(a * b);
+    }
+  }
+  *y = acc;
+  *yabs = aacc;
+}
+
+// GEMM reference [P1 "Der technische Durchbruch": linear layers do FP8 math]
+// over rows [m0,m1) x cols [n0,n1); y/yabs laid out [m1-m0][n1-n0].
+//   A : [M][K] codes (K-major), sA : [K/128][M]
+//   B : [N][K] codes (K-major), sB : per kind (see b_scale)
+void orc_gemm_ref_tile(int kind, int64_t M, int64_t N, int64_t K,
+                       const uint8_t* A, const float* sA, const uint8_t* B,
+                       const float* sB, int64_t m0, int64_t m1, int64_t n0,
+                       int64_t n1, double* y, double* yabs) {
+  const int64_t W = n1 - n0;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = m0; m < m1; ++m)
+    for (int64_t n = n0; n < n1; ++n)
+      ref_element(kind, M, N, K, A, sA, B, sB, 0, K / 128, m, n,
+                  &y[(m - m0) * W + (n - n0)], &yabs[(m - m0) * W + (n - n0)]);
+}
+
+// Grouped (MoE expert) GEMM reference [P1 "Leistungsgewinne in der Praxis":
+// the recipe also trains the Qwen3-30B mixture-of-experts model].  Expert g
+// owns token rows [off[g], off[g+1]) of the permuted token matrix; every
+// offset is a multiple of 128 (segments zero-padded to whole blocks).
+//   kind 0/1: rows m of the output use expert g(m)'s weight
+//             B + g*N*K, sB + g*(N/128)*(K/128); y over rows [m0,m1)
+//             (rows at or beyond off[G] are not part of the result).
+//   kind 2  : output dW_g [N][K] for one expert g = `expert`: the
+//             contraction runs over that expert's token chunks only; A is
+//             [N][Mtot] (K-major in tokens), sA [Mtot/128][N], B [K][Mtot],
+//             sB [Mtot/128][K]; y over rows [m0,m1) x cols [n0,n1) of dW_g.
+//             An empty expert gives exact zeros.
+void orc_grouped_gemm_ref_tile(int kind, int32_t G, const int32_t* off,
+                               int64_t Mtot, int64_t N, int64_t K,
+                               const uint8_t* A, const float* sA,
+                               const uint8_t* B, const float* sB,
+                               int32_t expert, int64_t m0, int64_t m1,
+                               int64_t n0, int64_t n1, double* y,
+                               double* yabs) {
+  const int64_t W = n1 - n0;
+  if (kind == 2) {
+    // GEMM dims: rows N, cols K, contraction Mtot.
+    int64_t kb0 = off[expert] / 128, kb1 = off[expert + 1] / 128;
+    for (int64_t m = m0; m < m1; ++m)
+      for (int64_t n = n0; n < n1; ++n)
+        ref_element(2, N, K, Mtot, A, sA, B, sB, kb0, kb1, m, n,
+                    &y[(m - m0) * W + (n - n0)],
+                    &yabs[(m - m0) * W + (n - n0)]);
+    return;
+  }
+  for (int64_t m = m0; m < m1; ++m) {
+    int32_t g = 0;
+    while (g < G && !(m >= off[g] && m < off[g + 1])) ++g;
+    for (int64_t n = n0; n < n1; ++n) {
+      double* py = &y[(m - m0) * W + (n - n0)];
+      double* pa = &yabs[(m - m0) * W + (n - n0)];
+      if (g == G) { *py = 0.0; *pa = 0.0; continue; }
+      const uint8_t* Bg = B + static_cast<int64_t>(g) * N * K;
+      const float* sBg = sB + static_cast<int64_t>(g) * (N / 128) * (K / 128);
+      ref_element(kind, Mtot, N, K, A, sA, Bg, sBg, 0, K / 128, m, n, py, pa);
+    }
+  }
+}
+
+// Same reference at a list of (m, n) points.
+void orc_gemm_ref_points(int kind, int64_t M, int64_t N, int64_t K,
+                         const uint8_t* A, const float* sA, const uint8_t* B,
+                         const float* sB, const int64_t* pm, const int64_t* pn,
+                         int64_t npts, double* y, double* yabs) {
+  for (int64_t p = 0; p < npts; ++p)
+    orc_gemm_ref_tile(kind, M, N, K, A, sA, B, sB, pm[p], pm[p] + 1, pn[p],
+                      pn[p] + 1, y + p, yabs + p);
+}
+
+// Diagnostic only (never a gate): the fp32 per-chunk promotion a tensor-core
+// kernel performs — fp32 chunk sums, times fp32(sa*sb), accumulated in fp32,
+// then rounded to bf16.  Returns bf16 bits [m1-m0][n1-n0].
+void orc_gemm_mimic_tile(int kind, int64_t M, int64_t N, int64_t K,
+                         const uint8_t* A, const float* sA, const uint8_t* B,
+                         const float* sB, int64_t m0, int64_t m1, int64_t n0,
+                         int64_t n1, uint16_t* y) {
+  const int64_t nK = K / 128;
+  const int64_t W = n1 - n0;
+  for (int64_t m = m0; m < m1; ++m)
+    for (int64_t n = n0; n < n1; ++n) {
+      float acc = 0.0f;
+      for (int64_t kb = 0; kb < nK; ++kb) {
+        float part = 0.0f;
+        for (int64_t j = 0; j < 128; ++j) {
+          int64_t k = kb * 128 + j;
+          part += static_cast<float>(e4m3_decode(A[m * K + k]) *
+                                     e4m3_decode(B[n * K + k]));
+        }
+        float sc = sA[kb * M + m] *
+                   static_cast<float>(b_scale(kind, sB, N, K, n, kb));
+        acc += part * sc;
+      }
+      y[(m - m0) * W + (n - n0)] = float_to_bf16_bits(acc);
+    }
+}
+
+// BF16 reference GEMM (the comparison path): y = sum_k a[m][k] * b[n][k] in
+// fp64 over bf16 operands, both K-major.
+void orc_gemm_bf16_ref_tile(int64_t M, int64_t N, int64_t K,
+                            const uint16_t* A, const uint16_t* B, int64_t m0,
+                            int64_t m1, int64_t n0, int64_t n1, double* y,
+                            double* yabs) {
+  (void)M; (void)N;
+  const int64_t W = n1 - n0;
+  for (int64_t m = m0; m < m1; ++m)
+    for (int64_t n = n0; n < n1; ++n) {
+      double acc = 0.0, aacc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = static_cast<double>(bf16_bits_to_float(A[m * K + k])) *
+                   static_cast<double>(bf16_bits_to_float(B[n * K + k]));
+        acc += p;
+        aacc += std::fabs(p);
+      }
+      y[(m - m0) * W + (n - n0)] = acc;
+      yabs[(m - m0) * W + (n - n0)] = aacc;
+    }
+}
+
+// One bf16 unit in the last place of v: the gap between the two bf16 values
+// around |v| (8 significant bits; smallest subnormal step 2^-133).
+double orc_bf16_ulp(double v) {
+  double a = std::fabs(v);
+  if (a < std::ldexp(1.0, -126)) return std::ldexp(1.0, -133);
+  int E;
+  std::frexp(a, &E);  // a in [2^(E-1), 2^E)
+  return std::ldexp(1.0, E - 1 - 7);
+}
+
+// The GEMM acceptance rule: |y - yref| <= rel * yabs + 1 bf16 ulp(yref).
+// y are bf16 bits.  Returns the number of violations; the worst ratio of
+// error to allowance is written to *worst.
+int64_t orc_check_tol(const uint16_t* y, const double* yref,
+                      const double* yabs, int64_t n, double rel,
+                      double* worst) {
+  int64_t bad = 0;
+  double w = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    double g = bf16_bits_to_float(y[i]);
+    double err = std::fabs(g - yref[i]);
+    double allow = rel * yabs[i] + orc_bf16_ulp(yref[i]);
+    if (!(err <= allow)) ++bad;
+    double r = err / allow;
+    if (std::isnan(g)) r = INFINITY;
+    if (r > w) w = r;
+  }
+  if (worst) *worst = w;
+  return bad;
+}
+
+}  // extern "C"
