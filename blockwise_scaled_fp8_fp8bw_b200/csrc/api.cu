@@ -1,0 +1,222 @@
+// C ABI of the library (declared in include/fp8bw.h): host-side argument
+// validation, device checks and kernel launches.  Nothing here allocates
+// device memory; no exception, abort or assert crosses the boundary.
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/fp8bw.h"
+
+namespace fp8bw {
+cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
+                             uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
+                             cudaStream_t st);
+cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, int mode,
+                                uint8_t* q, float* s, uint8_t* qT, cudaStream_t st);
+cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cudaStream_t st);
+cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M,
+                            int64_t N, int64_t K, const uint8_t* A, const float* sA,
+                            const uint8_t* B, const float* sB, void* D, int64_t ldd, int num_sms,
+                            cudaStream_t st);
+cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
+                             void* D, int64_t ldd, int num_sms, cudaStream_t st);
+cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
+}  // namespace fp8bw
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];  // 0 = not initialised, -1 = unsupported
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool mult128(int64_t v) { return v >= 0 && (v & 127) == 0; }
+constexpr int64_t kMaxDim = int64_t(1) << 30;  // sizes index with 32-bit tile math
+
+fp8bw_status init_device(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return FP8BW_ERR_INVALID_ARG;
+  if (g_sms[dev] > 0) return FP8BW_OK;
+  if (g_sms[dev] < 0) return FP8BW_ERR_UNSUPPORTED_ARCH;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FP8BW_ERR_CUDA;
+  if (major != 10 || minor != 0) {
+    g_sms[dev] = -1;
+    return FP8BW_ERR_UNSUPPORTED_ARCH;
+  }
+  g_sms[dev] = sms;
+  return FP8BW_OK;
+}
+
+fp8bw_status current(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8BW_ERR_CUDA;
+  fp8bw_status s = init_device(dev);
+  if (s == FP8BW_OK) *sms = g_sms[dev];
+  return s;
+}
+
+inline fp8bw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BW_OK : FP8BW_ERR_CUDA; }
+
+fp8bw_status check_weight(const void* w, int64_t N, int64_t K, int64_t ldw, const uint8_t* q,
+                          const float* s, const uint8_t* qT) {
+  if (!w || !q || !s) return FP8BW_ERR_INVALID_ARG;
+  if (N < 0 || K < 0 || ldw < K) return FP8BW_ERR_INVALID_ARG;
+  if (N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(N) || !mult128(K) || (ldw & 7) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(s) || (qT && !aligned16(qT)))
+    return FP8BW_ERR_ALIGNMENT;
+  return FP8BW_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+FP8BW_API fp8bw_status fp8bw_init(int device) { return init_device(device); }
+
+FP8BW_API const char* fp8bw_status_string(fp8bw_status s) {
+  switch (s) {
+    case FP8BW_OK: return "ok";
+    case FP8BW_ERR_INVALID_ARG: return "invalid argument";
+    case FP8BW_ERR_ALIGNMENT: return "size or pointer alignment";
+    case FP8BW_ERR_UNSUPPORTED_ARCH: return "unsupported architecture (needs sm_100)";
+    case FP8BW_ERR_CUDA: return "CUDA error";
+    case FP8BW_ERR_TIMEOUT: return "device-side wait timed out";
+    case FP8BW_ERR_DEVICE_CHECK: return "device-side argument check failed";
+    case FP8BW_ERR_TOO_LARGE: return "size exceeds the supported maximum";
+  }
+  return "unknown status";
+}
+
+FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {
+  uint32_t v = 0;
+  if (fp8bw::gemm_read_clear_error(&v, stream) != cudaSuccess) return FP8BW_ERR_CUDA;
+  if (v & 1u) return FP8BW_ERR_TIMEOUT;
+  if (v & 2u) return FP8BW_ERR_DEVICE_CHECK;
+  return FP8BW_OK;
+}
+
+FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                   fp8bw_scale_mode mode, uint8_t* q_row, float* s_row,
+                                   uint8_t* q_col, float* s_col, fp8bw_stream_t stream) {
+  if (!x || !q_row || !s_row) return FP8BW_ERR_INVALID_ARG;
+  if ((q_col == nullptr) != (s_col == nullptr)) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || K < 0 || ldx < K) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || K > kMaxDim || M / 128 > 65535) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(K) || (ldx & 7) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(q_row) || !aligned16(s_row) || (q_col && !aligned16(q_col)) ||
+      (s_col && !aligned16(s_col)))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status s = current(&sms);
+  if (s != FP8BW_OK) return s;
+  if (M == 0 || K == 0) return FP8BW_OK;
+  return from_cuda(fp8bw::launch_quant_act(x, M, K, ldx, mode, q_row, s_row, q_col, s_col,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_quant_weight_128x128(const void* w, int64_t N, int64_t K, int64_t ldw,
+                                        fp8bw_scale_mode mode, uint8_t* q, float* s, uint8_t* qT,
+                                        fp8bw_stream_t stream) {
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  fp8bw_status st = check_weight(w, N, K, ldw, q, s, qT);
+  if (st != FP8BW_OK) return st;
+  if (N / 128 > 65535) return FP8BW_ERR_TOO_LARGE;
+  int sms = 0;
+  st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (N == 0 || K == 0) return FP8BW_OK;
+  return from_cuda(fp8bw::launch_quant_weight(w, N, K, ldw, mode, q, s, qT,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_requant_weights(const fp8bw_weight_desc* descs, int32_t n,
+                                   fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  if (n < 0 || (n > 0 && !descs)) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const fp8bw_weight_desc& d = descs[i];
+    fp8bw_status st = check_weight(d.w, d.N, d.K, d.ldw, d.q, d.s, d.qT);
+    if (st != FP8BW_OK) return st;
+    total += (d.N / 128) * (d.K / 128);
+  }
+  if (total > 0x7FFFFFFF) return FP8BW_ERR_TOO_LARGE;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (n == 0) return FP8BW_OK;
+  return from_cuda(fp8bw::launch_requant(descs, n, mode, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K, const uint8_t* A,
+                        const float* sA, const uint8_t* B, const float* sB, void* D, int64_t ldd,
+                        fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  if (kind != FP8BW_FPROP && kind != FP8BW_DGRAD && kind != FP8BW_WGRAD) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (!A || !sA || !B || !sB || !D) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(N) || !mult128(K) || (ldd & 7) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sA) || !aligned16(sB))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (M == 0 || N == 0) return FP8BW_OK;
+  if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(fp8bw::launch_gemm_fp8(kind, false, 0, nullptr, M, N, K, A, sA, B, sB, D, ldd,
+                                          sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
+                                int64_t M_total_pad, int64_t N, int64_t K, const uint8_t* A,
+                                const float* sA, const uint8_t* B, const float* sB, void* D,
+                                fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  if (kind != FP8BW_FPROP && kind != FP8BW_DGRAD && kind != FP8BW_WGRAD) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (!d_offsets || !A || !sA || !B || !sB || !D) return FP8BW_ERR_INVALID_ARG;
+  if (G < 1 || M_total_pad < 0 || N < 0 || K < 0) return FP8BW_ERR_INVALID_ARG;
+  if (G > FP8BW_MAX_EXPERTS) return FP8BW_ERR_TOO_LARGE;
+  if (M_total_pad > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M_total_pad) || !mult128(N) || !mult128(K)) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sA) || !aligned16(sB) ||
+      (reinterpret_cast<uintptr_t>(d_offsets) & 3u))
+    return FP8BW_ERR_ALIGNMENT;
+  if ((int64_t)G * N * K > (int64_t(1) << 40)) return FP8BW_ERR_TOO_LARGE;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (kind == FP8BW_WGRAD) {
+    // GEMM sizes: rows = N (out), cols = K (in), contraction = tokens.
+    if (N == 0 || K == 0) return FP8BW_OK;
+    return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, N, K, M_total_pad, A, sA, B,
+                                            sB, D, K, sms, cs));
+  }
+  if (M_total_pad == 0 || N == 0) return FP8BW_OK;
+  if (K == 0) return FP8BW_ERR_INVALID_ARG;
+  return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, M_total_pad, N, K, A, sA, B,
+                                          sB, D, N, sms, cs));
+}
+
+FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,
+                             int64_t ldd, fp8bw_stream_t stream) {
+  if (!A || !B || !D) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(N) || !mult128(K) || (ldd & 7) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (M == 0 || N == 0) return FP8BW_OK;
+  if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(fp8bw::launch_gemm_bf16(M, N, K, A, B, D, ldd, sms,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,668 @@
+// Tensor-core GEMMs for sm_100a: the blockwise-scaled FP8 GEMM (dense and
+// grouped, fprop / dgrad / wgrad) and the BF16 comparison GEMM.
+//
+// Method: "NVIDIA NeMo RL erreicht 48% ..." section "Der technische
+// Durchbruch": linear layers run FP8 math on E4M3 operands with one scale per
+// 1x128 activation block and per 128x128 weight block; FP8 has twice the
+// BF16 peak.  Section "Leistungsgewinne in der Praxis": the Qwen3-30B MoE
+// model trains with the same recipe (grouped expert GEMMs).
+//
+// FP8 kernel design (one CTA per SM, persistent, 384 threads):
+//   warp 0      TMA producer: per 128-wide K chunk, one 128x128 A tile and
+//               one 256x128 B tile (E4M3, 128-byte swizzle) into a 4-stage
+//               shared-memory ring.
+//   warp 1      MMA issuer: four tcgen05.mma kind::f8f6f4 (M=128, N=256,
+//               K=32) per chunk into one of two TMEM chunk accumulators
+//               (2 x 256 columns = all 512 TMEM columns).
+//   warp 2      scale loader: the chunk's 128 A-row scales and the B scales
+//               (2 block scales, or 256 column scales for wgrad) into an
+//               8-slot shared ring with cp.async.
+//   warps 4-11  promotion: each thread owns one accumulator row and 128
+//               columns; per chunk it reads the chunk product from TMEM
+//               (tcgen05.ld), multiplies by sA*sB in fp32 and adds it to
+//               its register accumulator (packed f32x2 FMAs).  The chunk
+//               accumulator is released right after the loads, so the MMA
+//               of chunk c+1 overlaps the promotion of chunk c.  At the end
+//               of a tile the rows are rounded to bf16 and stored.
+// Registers: warpgroup 0 drops to 40 per thread, the two promotion
+// warpgroups rise to 232 (128 accumulators + staging); 40*128 + 232*256 =
+// 64512 = 384 * 168, the launch allocation (checked on the host).
+// Every wait is bounded; on a timeout the kernel latches an error bit and
+// leaves its loops.
+
+#include "common.cuh"
+
+namespace fp8bw {
+
+__device__ uint32_t g_gemm_error;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int kStages = 4;
+constexpr int kScaleStages = 8;
+constexpr int kThreads = 384;
+constexpr uint32_t kATile = BM * BK;  // 16 KB
+constexpr uint32_t kBTile = BN * BK;  // 32 KB
+constexpr uint32_t kStageBytes = kATile + kBTile;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxGroups = FP8BW_MAX_EXPERTS;
+
+constexpr uint32_t kIdescF8 = idesc_make(0, 0, BM, BN);   // E4M3 x E4M3 -> F32
+constexpr uint32_t kIdescBF16 = idesc_make(1, 1, BM, BN); // BF16 x BF16 -> F32
+
+constexpr int kRegsLow = 40, kRegsHigh = 232, kRegsLaunch = 168;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
+
+struct ScaleSlot {
+  float sa[128];
+  float sb[256];
+};
+
+struct Bars {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t sfull[kScaleStages], sempty[kScaleStages];
+  uint64_t tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t bad_offsets;
+};
+
+struct GemmArgs {
+  int M, N, K;         // GEMM sizes (grouped wgrad: M = out, N = in, K = tokens)
+  int m_tiles, n_tiles, tiles, band;
+  const float* sA;     // [K/128][M]
+  const float* sB;     // per kind
+  uint16_t* D;
+  int64_t ldd;
+  const int32_t* offsets;  // grouped: device [G+1]
+  int G;
+};
+
+constexpr size_t kSmemFp8 = 1024 + size_t(kStages) * kStageBytes +
+                            size_t(kScaleStages) * sizeof(ScaleSlot) + sizeof(Bars) +
+                            sizeof(int32_t) * (kMaxGroups + 1);
+
+struct TileInfo {
+  int mt, nt, g, kb0, kb1;
+  bool skip;
+};
+
+template <int KIND, bool GROUPED>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off) {
+  TileInfo ti;
+  ti.g = 0;
+  ti.skip = false;
+  if (GROUPED && KIND == FP8BW_WGRAD) {
+    const int per = a.m_tiles * a.n_tiles;
+    ti.g = t / per;
+    const int r = t - ti.g * per;
+    ti.mt = r % a.m_tiles;
+    ti.nt = r / a.m_tiles;
+    ti.kb0 = off[ti.g] >> 7;
+    ti.kb1 = off[ti.g + 1] >> 7;
+    return ti;
+  }
+  const int band_tiles = a.band * a.n_tiles;
+  const int band = t / band_tiles;
+  const int r = t - band * band_tiles;
+  const int rows = min(a.band, a.m_tiles - band * a.band);
+  ti.mt = band * a.band + r % rows;
+  ti.nt = r / rows;
+  ti.kb0 = 0;
+  ti.kb1 = a.K / BK;
+  if (GROUPED) {
+    const int row0 = ti.mt * BM;
+    if (row0 >= off[a.G]) {
+      ti.skip = true;
+    } else {
+      int lo = 0, hi = a.G - 1;  // last g with off[g] <= row0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= row0) lo = mid; else hi = mid - 1;
+      }
+      ti.g = lo;
+    }
+  }
+  return ti;
+}
+
+__device__ __forceinline__ void raise_timeout(Bars* bars) {
+  atomicOr(&g_gemm_error, DEV_ERR_TIMEOUT);
+  atomicExch(&bars->abort, 1);
+}
+
+template <int KIND, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(smem + kStages * kStageBytes);
+  Bars* bars = reinterpret_cast<Bars*>(slots + kScaleStages);
+  int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->empty[i]), 1);
+    }
+    for (int i = 0; i < kScaleStages; ++i) {
+      mbar_init(smem_u32(&bars->sfull[i]), 32);
+      mbar_init(smem_u32(&bars->sempty[i]), 8);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->tfull[i]), 1);
+      mbar_init(smem_u32(&bars->tempty[i]), 8);
+    }
+    bars->abort = 0;
+    bars->bad_offsets = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (GROUPED) {
+    for (int i = threadIdx.x; i <= a.G; i += kThreads) s_off[i] = a.offsets[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (GROUPED) {
+    // Offsets must start at 0, be non-decreasing multiples of 128 and end
+    // within the token matrix; otherwise nothing is computed or written.
+    for (int i = threadIdx.x; i < a.G; i += kThreads) {
+      const int o0 = s_off[i], o1 = s_off[i + 1];
+      if (o1 < o0 || (o1 & 127) || (i == 0 && o0 != 0)) bars->bad_offsets = 1;
+    }
+    if (threadIdx.x == 0) {
+      const int mtot = (KIND == FP8BW_WGRAD) ? a.K : a.M;
+      if (s_off[a.G] > mtot || s_off[a.G] < 0) bars->bad_offsets = 1;
+    }
+    __syncthreads();
+    if (bars->bad_offsets) {
+      if (threadIdx.x == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
+      if (warp == 1) tmem_dealloc(bars->tmem_base, kTmemCols);
+      return;
+    }
+  }
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ------------------------------------------------ TMA producer ----
+      if (lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        if (ti.skip) continue;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
+            raise_timeout(bars);
+            goto done;
+          }
+          if (lane == 0) {
+            const uint32_t full = smem_u32(&bars->full[stage]);
+            const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
+            mbar_arrive_expect_tx(full, kStageBytes);
+            tma_load_2d(sa, &tmA, full, kb * BK, ti.mt * BM);
+            if (GROUPED && KIND != FP8BW_WGRAD)
+              tma_load_3d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN, ti.g);
+            else
+              tma_load_2d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN);
+          }
+          __syncwarp();
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (bars->abort) break;
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------- MMA issuer -----
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t bphase = 0;
+      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        if (ti.skip) continue;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1) ||
+              !mbar_wait(smem_u32(&bars->full[stage]), phase)) {
+            raise_timeout(bars);
+            goto done;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
+            const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+            const uint32_t d = tmem + buf * BN;
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)  // +32 bytes = +2 in the >>4 address field
+              umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, kIdescF8, kk > 0 ? 1u : 0u);
+            umma_commit(smem_u32(&bars->empty[stage]));
+            umma_commit(smem_u32(&bars->tfull[buf]));
+          }
+          __syncwarp();
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (++buf == 2) { buf = 0; bphase ^= 1; }
+        }
+        if (bars->abort) break;
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------ scale loader ----
+      int ss = 0;
+      uint32_t sphase = 0;
+      const int nKb = a.K / BK, nNb = a.N / 128;
+      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        if (ti.skip) continue;
+        const float* sBg = a.sB;
+        if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&bars->sempty[ss]), sphase ^ 1)) {
+            raise_timeout(bars);
+            goto done;
+          }
+          ScaleSlot* sl = &slots[ss];
+          cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + ti.mt * BM + lane * 4);
+          if (KIND == FP8BW_WGRAD) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int n = ti.nt * BN + h * 128 + lane * 4;
+              if (n < a.N) cp_async_16(smem_u32(&sl->sb[h * 128 + lane * 4]), sBg + (size_t)kb * a.N + n);
+            }
+          } else if (lane < 2) {
+            const int nb = ti.nt * 2 + lane;
+            if (nb < nNb) {
+              const float* src = (KIND == FP8BW_FPROP) ? sBg + (size_t)nb * nKb + kb
+                                                       : sBg + (size_t)kb * nNb + nb;
+              cp_async_4(smem_u32(&sl->sb[lane]), src);
+            }
+          }
+          cp_async_mbar_arrive_noinc(smem_u32(&bars->sfull[ss]));
+          if (++ss == kScaleStages) { ss = 0; sphase ^= 1; }
+        }
+        if (bars->abort) break;
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+  } else {
+    regs_inc<kRegsHigh>();
+    // -------------------------------------------------------- promotion --
+    const int q = warp & 3;            // TMEM lane quarter of this warp
+    const int half = (warp - 4) >> 2;  // column half of the 256-wide tile
+    int ss = 0;
+    uint32_t sphase = 0;
+    int buf = 0;
+    uint32_t bphase = 0;
+    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+      if (ti.skip) continue;
+      const int row = ti.mt * BM + q * 32 + lane;
+      const int col0 = ti.nt * BN + half * 128;
+      const bool valid = col0 < a.N;
+      uint16_t* drow = a.D + (GROUPED && KIND == FP8BW_WGRAD ? (size_t)ti.g * a.M * a.N : 0) +
+                       (size_t)row * a.ldd + col0;
+      float2 acc[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.f, 0.f);
+      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        if (!mbar_wait(smem_u32(&bars->sfull[ss]), sphase) ||
+            !mbar_wait(smem_u32(&bars->tfull[buf]), bphase)) {
+          raise_timeout(bars);
+          goto done;
+        }
+        tc_fence_after();
+        const ScaleSlot* sl = &slots[ss];
+        const float sa = sl->sa[q * 32 + lane];
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          uint32_t r[32];
+          tmem_ld32(taddr + p * 32, r);
+          tmem_wait_ld();
+          if (KIND == FP8BW_WGRAD) {
+            const float2 sa2 = make_float2(sa, sa);
+            const float2* sb2 = reinterpret_cast<const float2*>(&sl->sb[half * 128 + p * 32]);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float2 sc = fmul2(sa2, sb2[j]);
+              acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+                                      sc, acc[p * 16 + j]);
+            }
+          } else {
+            const float s = sa * sl->sb[half];
+            const float2 s2 = make_float2(s, s);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+                                      s2, acc[p * 16 + j]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&bars->tempty[buf]));
+          mbar_arrive(smem_u32(&bars->sempty[ss]));
+        }
+        if (++ss == kScaleStages) { ss = 0; sphase ^= 1; }
+        if (++buf == 2) { buf = 0; bphase ^= 1; }
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(drow);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[4 * j + 0].x, acc[4 * j + 0].y);
+          o.y = pack_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y);
+          o.z = pack_bf16x2(acc[4 * j + 2].x, acc[4 * j + 2].y);
+          o.w = pack_bf16x2(acc[4 * j + 3].x, acc[4 * j + 3].y);
+          dst[j] = o;
+        }
+      }
+      if (bars->abort) break;
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ BF16 GEMM ---
+// Same pipeline without scales: BK = 64 bf16 (128-byte rows), four
+// kind::f16 MMAs (K = 16) per stage, the accumulator stays in TMEM for the
+// whole K loop, and the 8 epilogue warps drain a finished tile (double
+// buffered in TMEM) while the next tile accumulates.
+constexpr int BK16 = 64;
+constexpr size_t kSmemBf16 = 1024 + size_t(kStages) * kStageBytes + sizeof(Bars);
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->tfull[i]), 1);
+      mbar_init(smem_u32(&bars->tempty[i]), 8);
+    }
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int nkb = a.K / BK16;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false>(a, t, nullptr);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
+          raise_timeout(bars);
+          goto done;
+        }
+        if (lane == 0) {
+          const uint32_t full = smem_u32(&bars->full[stage]);
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          mbar_arrive_expect_tx(full, kStageBytes);
+          tma_load_2d(sa, &tmA, full, kb * BK16, ti.mt * BM);
+          tma_load_2d(sa + kATile, &tmB, full, kb * BK16, ti.nt * BN);
+        }
+        __syncwarp();
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (bars->abort) break;
+    }
+  } else if (warp == 1) {
+    int stage = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    uint32_t bphase = 0;
+    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1)) {
+        raise_timeout(bars);
+        goto done;
+      }
+      tc_fence_after();
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(smem_u32(&bars->full[stage]), phase)) {
+          raise_timeout(bars);
+          goto done;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+#pragma unroll
+          for (int kk = 0; kk < BK16 / 16; ++kk)
+            umma_f16(tmem + buf * BN, da + 2 * kk, db + 2 * kk, kIdescBF16,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&bars->empty[stage]));
+          if (kb == nkb - 1) umma_commit(smem_u32(&bars->tfull[buf]));
+        }
+        __syncwarp();
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (++buf == 2) { buf = 0; bphase ^= 1; }
+      if (bars->abort) break;
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3, half = (warp - 4) >> 2;
+    int buf = 0;
+    uint32_t bphase = 0;
+    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false>(a, t, nullptr);
+      if (!mbar_wait(smem_u32(&bars->tfull[buf]), bphase)) {
+        raise_timeout(bars);
+        goto done;
+      }
+      tc_fence_after();
+      const int row = ti.mt * BM + q * 32 + lane;
+      const int col0 = ti.nt * BN + half * 128;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
+      uint4* dst = reinterpret_cast<uint4*>(a.D + (size_t)row * a.ldd + col0);
+      const bool valid = col0 < a.N;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        uint32_t r[32];
+        tmem_ld32(taddr + p * 32, r);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+            o.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+            o.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+            o.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+            dst[p * 4 + j] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->tempty[buf]));
+      if (++buf == 2) { buf = 0; bphase ^= 1; }
+      if (bars->abort) break;
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// -------------------------------------------------------------- host ------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major [rows][inner] (inner contiguous, `ld` elements per row), box
+// [box_rows][box_inner], 128-byte swizzle.  Optional third dim (groups).
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+              uint64_t rows, uint64_t ld, uint32_t box_inner, uint32_t box_rows,
+              uint64_t groups = 0) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, groups};
+  cuuint64_t strides[2] = {ld * esize, ld * esize * rows};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = groups ? 3 : 2;
+  return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t prepare(K kernel, size_t smem) {
+  static thread_local int done_dev = -1;
+  (void)done_dev;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kernel);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg draws on the launch allocation: refuse to launch if the
+  // compiled register count could not cover the split.
+  if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+int gemm_band_rows = 16;
+
+cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
+                            int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
+                            const float* sB, void* D, int64_t ldd, int num_sms, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  GemmArgs a;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.m_tiles = (int)(M / BM);
+  a.n_tiles = (int)((N + BN - 1) / BN);
+  a.band = gemm_band_rows;
+  a.sA = sA;
+  a.sB = sB;
+  a.D = static_cast<uint16_t*>(D);
+  a.ldd = ldd;
+  a.offsets = d_off;
+  a.G = G;
+  if (grouped && kind == FP8BW_WGRAD) a.tiles = G * a.m_tiles * a.n_tiles;
+  else a.tiles = a.m_tiles * a.n_tiles;
+  if (a.tiles == 0) return cudaSuccess;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, K, BK, BM)) return cudaErrorInvalidValue;
+  const bool b3 = grouped && kind != FP8BW_WGRAD;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, BN, b3 ? (uint64_t)G : 0))
+    return cudaErrorInvalidValue;
+  const int grid = a.tiles < num_sms ? a.tiles : num_sms;
+#define FP8BW_LAUNCH(KD, GR)                                                  \
+  do {                                                                        \
+    auto kern = k_gemm_fp8<KD, GR>;                                           \
+    cudaError_t e = prepare(kern, kSmemFp8);                                  \
+    if (e != cudaSuccess) return e;                                           \
+    kern<<<grid, kThreads, kSmemFp8, st>>>(ta, tb, a);                        \
+  } while (0)
+  if (!grouped) {
+    if (kind == FP8BW_FPROP) FP8BW_LAUNCH(FP8BW_FPROP, false);
+    else if (kind == FP8BW_DGRAD) FP8BW_LAUNCH(FP8BW_DGRAD, false);
+    else FP8BW_LAUNCH(FP8BW_WGRAD, false);
+  } else {
+    if (kind == FP8BW_FPROP) FP8BW_LAUNCH(FP8BW_FPROP, true);
+    else if (kind == FP8BW_DGRAD) FP8BW_LAUNCH(FP8BW_DGRAD, true);
+    else FP8BW_LAUNCH(FP8BW_WGRAD, true);
+  }
+#undef FP8BW_LAUNCH
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,
+                             int64_t ldd, int num_sms, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  GemmArgs a;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.m_tiles = (int)(M / BM);
+  a.n_tiles = (int)((N + BN - 1) / BN);
+  a.band = gemm_band_rows;
+  a.tiles = a.m_tiles * a.n_tiles;
+  a.sA = a.sB = nullptr;
+  a.D = static_cast<uint16_t*>(D);
+  a.ldd = ldd;
+  a.offsets = nullptr;
+  a.G = 0;
+  if (a.tiles == 0) return cudaSuccess;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, K, BK16, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, K, BK16, BN)) return cudaErrorInvalidValue;
+  const int grid = a.tiles < num_sms ? a.tiles : num_sms;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBf16);
+  if (e != cudaSuccess) return e;
+  k_gemm_bf16<<<grid, kThreads, kSmemBf16, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st) {
+  uint32_t v = 0, z = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_gemm_error, sizeof v, 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbolAsync(g_gemm_error, &z, sizeof z, 0, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *out = v;
+  return e;
+}
+
+}  // namespace fp8bw

@@ -1,0 +1,190 @@
+/*
+ * fp8bw — blockwise-scaled FP8 linear layer for B200 (sm_100a).
+ *
+ * The method (page "NVIDIA NeMo RL erreicht 48% Geschwindigkeitssteigerung
+ * mit End-to-End FP8-Präzisionstraining", section "Der technische
+ * Durchbruch"): linear layers run FP8 math on E4M3 operands that carry one
+ * scale per 128x128 block of a weight and one per 1x128 block of an
+ * activation; section "Leistungsgewinne in der Praxis": the weight scales are
+ * recalibrated after every training step; section "Warum dies für die
+ * KI-Ökonomie wichtig ist": optionally the scales are powers of two.  E4M3
+ * itself (page "FP8 Trainingsinfrastructuur", section "Het landschap van
+ * numerieke precisie"): 4 exponent bits, 3 mantissa bits, values up to +-448.
+ *
+ * Conventions for every call below
+ *  - All tensor arguments are DEVICE pointers to caller-owned memory; the
+ *    library allocates no device memory and keeps no pointer after the call.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The returned status covers host-side validation and
+ *    launch errors; errors seen inside a kernel (a bounded wait that ran out,
+ *    a failed device-side check) are latched in a device error word and read
+ *    with fp8bw_last_device_error().
+ *  - Shapes: M, N, K are multiples of 128 (else FP8BW_ERR_ALIGNMENT), and
+ *    every pointer is 16-byte aligned with leading dimensions that keep rows
+ *    16-byte aligned.  Invalid arguments never reach the GPU.
+ *  - bf16 tensors are IEEE bfloat16 bit patterns; E4M3 codes are bytes
+ *    (sign | 4-bit exponent field, bias 7 | 3-bit mantissa; 0x7F/0xFF NaN).
+ *  - Scale rule (identical in every quantizer): amax = max |x| over the block;
+ *      FP8BW_SCALE_FP32: s = fp32(amax / 448)
+ *      FP8BW_SCALE_POW2: s = 2^e, e the smallest integer with amax <= 448*2^e,
+ *                        clamped to [-127, 127]
+ *      an all-zero block has s = 1;
+ *    codes q = E4M3(fp32(x / s)) with IEEE fp32 division, round to nearest
+ *    even, magnitudes above 448 saturating to 448, the sign of zero kept.
+ *    Dequantized value = decode(q) * s.
+ */
+#ifndef FP8BW_H_
+#define FP8BW_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FP8BW_API __attribute__((visibility("default")))
+#else
+#define FP8BW_API
+#endif
+
+typedef struct CUstream_st* fp8bw_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  FP8BW_OK = 0,
+  FP8BW_ERR_INVALID_ARG = 1,     /* null pointer, bad enum, negative size   */
+  FP8BW_ERR_ALIGNMENT = 2,       /* size not a multiple of 128, misaligned  */
+  FP8BW_ERR_UNSUPPORTED_ARCH = 3,/* device is not compute capability 10.0   */
+  FP8BW_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed       */
+  FP8BW_ERR_TIMEOUT = 5,         /* a device-side bounded wait ran out      */
+  FP8BW_ERR_DEVICE_CHECK = 6,    /* a device-side argument check failed     */
+  FP8BW_ERR_TOO_LARGE = 7        /* a size exceeds a documented maximum     */
+} fp8bw_status;
+
+typedef enum { FP8BW_SCALE_FP32 = 0, FP8BW_SCALE_POW2 = 1 } fp8bw_scale_mode;
+
+typedef enum { FP8BW_FPROP = 0, FP8BW_DGRAD = 1, FP8BW_WGRAD = 2 } fp8bw_gemm_kind;
+
+/* Checks that `device` is an sm_100 part and caches its SM count.  Called
+ * implicitly by every entry point for the current device; calling it
+ * explicitly first keeps that one-time query out of timed regions. */
+FP8BW_API fp8bw_status fp8bw_init(int device);
+
+/* Static, human-readable name of a status. */
+FP8BW_API const char* fp8bw_status_string(fp8bw_status s);
+
+/* Synchronizes `stream`, then returns (and clears) the device error word of
+ * the current device: FP8BW_ERR_TIMEOUT if a kernel's bounded wait ran out,
+ * FP8BW_ERR_DEVICE_CHECK if a kernel rejected its device-side arguments
+ * (e.g. grouped offsets), else FP8BW_OK.  FP8BW_ERR_CUDA if the sync failed. */
+FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream);
+
+/* Activation quantization with 1x128 blocks ("Der technische Durchbruch":
+ * 1x128 granularity for activations), plus the column-wise copy the weight
+ * gradient needs.
+ *   x      [M][ldx] bf16, row-major; the first K columns are quantized.
+ *   q_row  [M][K]   E4M3 codes; block (m, kb) = x[m][128kb .. 128kb+127]
+ *   s_row  [K/128][M] fp32 scales, chunk-major (s_row[kb*M + m])
+ *   q_col  [K][M]   E4M3 codes of the column-wise copy: block (mb, k) =
+ *                   x[128mb .. 128mb+127][k], quantized from x itself and
+ *                   stored transposed (q_col[k*M + m]) so that the weight
+ *                   gradient reads it K-major in tokens
+ *   s_col  [M/128][K] fp32 scales of the column-wise copy
+ *   q_col and s_col are both NULL for a row-wise-only call.
+ * For mixture-of-experts tokens grouped by expert, pad each expert's segment
+ * to a multiple of 128 rows (zero rows): column blocks then never straddle
+ * two experts and zero rows change no block's amax.
+ * Requires M, K multiples of 128, ldx >= K, ldx a multiple of 8. */
+FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                   fp8bw_scale_mode mode, uint8_t* q_row, float* s_row,
+                                   uint8_t* q_col, float* s_col, fp8bw_stream_t stream);
+
+/* Weight quantization with 128x128 blocks ("Der technische Durchbruch":
+ * 128x128 granularity for weights).
+ *   w   [N][ldw] bf16 row-major (nn.Linear layout: N = out, K = in features)
+ *   q   [N][K]   E4M3 codes
+ *   s   [N/128][K/128] fp32 scales, row-major
+ *   qT  [K][N]   the exact byte transpose of q (the data-gradient operand),
+ *                or NULL.  Its scale grid is s read transposed.
+ * Requires N, K multiples of 128, ldw >= K, ldw a multiple of 8. */
+FP8BW_API fp8bw_status fp8bw_quant_weight_128x128(const void* w, int64_t N, int64_t K, int64_t ldw,
+                                        fp8bw_scale_mode mode, uint8_t* q, float* s,
+                                        uint8_t* qT, fp8bw_stream_t stream);
+
+/* One weight of a batched requantization. */
+typedef struct {
+  const void* w;   /* [N][ldw] bf16 */
+  int64_t N, K, ldw;
+  uint8_t* q;      /* [N][K]            */
+  float* s;        /* [N/128][K/128]    */
+  uint8_t* qT;     /* [K][N] or NULL    */
+} fp8bw_weight_desc;
+
+/* Per-step scale recalibration ("Leistungsgewinne in der Praxis": the scales
+ * are recalibrated after every training step): requantizes every weight in
+ * `descs` (a HOST array of n descriptors, read during the call only) exactly
+ * as fp8bw_quant_weight_128x128 would, in one launch per up to
+ * FP8BW_REQUANT_MAX_PER_LAUNCH weights.  Output is bit-identical to n
+ * separate fp8bw_quant_weight_128x128 calls. */
+#define FP8BW_REQUANT_MAX_PER_LAUNCH 256
+FP8BW_API fp8bw_status fp8bw_requant_weights(const fp8bw_weight_desc* descs, int32_t n,
+                                   fp8bw_scale_mode mode, fp8bw_stream_t stream);
+
+/* Blockwise-scaled FP8 GEMM ("Der technische Durchbruch": linear layers run
+ * FP8 math), FP32 accumulation, bf16 output:
+ *   D[m][n] = bf16( sum_kb sA(m,kb) * sB(n,kb) * sum_{k in chunk kb} A[m][k] B[n][k] )
+ * with codes decoded from E4M3 and chunk kb = columns 128kb .. 128kb+127.
+ * M, N, K are the GEMM's own sizes:
+ *   FPROP  Y  = X W^T : A = q_row(X) [M][K], sA = s_row(X); B = q(W) [N][K],
+ *                       sB = s(W) [N/128][K/128]
+ *   DGRAD  dX = dY W  : A = q_row(dY) [M][K=out], sA = s_row(dY);
+ *                       B = qT(W) [N=in][K=out], sB = s(W) of the layer,
+ *                       i.e. [K/128][N/128] in this call's sizes
+ *   WGRAD  dW = dY^T X: A = q_col(dY) [M=out][K=tokens], sA = s_col(dY);
+ *                       B = q_col(X) [N=in][K=tokens], sB = s_col(X) [K/128][N]
+ *   A  [M][K] codes, K-major; sA [K/128][M]
+ *   B  [N][K] codes, K-major; sB as above
+ *   D  [M][ldd] bf16; ldd >= N, a multiple of 8
+ * `mode` states how the scales were made; FP8BW_SCALE_POW2 promises exact
+ * powers of two (the kernel may then fold them into the tensor-core MMA).
+ * The result is within |D - ref| <= 1e-2 * sum_k |a_k b_k| + 1 bf16 ulp(ref)
+ * of the fp64 product of the dequantized operands. */
+FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                        const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                        void* D, int64_t ldd, fp8bw_scale_mode mode, fp8bw_stream_t stream);
+
+/* Grouped GEMM for mixture-of-experts layers ("Leistungsgewinne in der
+ * Praxis": the recipe also trains the Qwen3-30B MoE model).  Tokens are
+ * grouped by expert: expert g owns rows [off[g], off[g+1]) of the permuted
+ * token matrix, with every offset a multiple of 128 (segments zero-padded),
+ * off[0] = 0 and off[G] <= M_total_pad.  `d_offsets` is a DEVICE array of
+ * G+1 int32 values, so routing never synchronizes the host; a kernel that
+ * finds them invalid writes nothing and latches FP8BW_ERR_DEVICE_CHECK.
+ *   FPROP/DGRAD: A [M_total_pad][K], sA [K/128][M_total_pad];
+ *                B [G][N][K] (FPROP: q(W_g); DGRAD: qT(W_g)),
+ *                sB [G][...] the per-expert grid as in fp8bw_gemm;
+ *                D [M_total_pad][N]; rows at or beyond off[G] are untouched.
+ *   WGRAD:       A = q_col(dY) [N][M_total_pad], sA [M_total_pad/128][N];
+ *                B = q_col(X)  [K][M_total_pad], sB [M_total_pad/128][K];
+ *                D [G][N][K]: expert g contracts only its own tokens; an
+ *                expert with no tokens gets exact zeros.
+ * Requires G <= FP8BW_MAX_EXPERTS. */
+#define FP8BW_MAX_EXPERTS 1024
+FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
+                                int64_t M_total_pad, int64_t N, int64_t K,
+                                const uint8_t* A, const float* sA, const uint8_t* B,
+                                const float* sB, void* D, fp8bw_scale_mode mode,
+                                fp8bw_stream_t stream);
+
+/* BF16 GEMM, the comparison path of "Der technische Durchbruch" (FP8 linear
+ * layers have twice the BF16 peak): D[m][n] = bf16( sum_k A[m][k] B[n][k] )
+ * with FP32 accumulation.  A [M][K], B [N][K] bf16, K-major (dense rows);
+ * D [M][ldd] bf16.  M, N, K multiples of 128. */
+FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
+                             void* D, int64_t ldd, fp8bw_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BW_H_ */

@@ -17,3 +17,15 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def fb():
+    """The CUDA library (fails loudly if it is missing or no GPU is visible)."""
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from blockwise_scaled_fp8_fp8bw_b200 import build
+    build.build()
+    import blockwise_scaled_fp8_fp8bw_b200 as lib
+    lib.fp8bw_init(torch.cuda.current_device())
+    return lib

@@ -1,0 +1,80 @@
+"""The C-ABI library loads, exports every call its header declares, and
+rejects invalid arguments on the host (no GPU needed: none of these calls
+reaches the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bw.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FP8BW_API\s+[\w\s\*]+?\b(fp8bw_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from blockwise_scaled_fp8_fp8bw_b200 import build
+    build.build()
+    import blockwise_scaled_fp8_fp8bw_b200 as fb
+    return fb
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for n in ["fp8bw_quant_act_1x128", "fp8bw_quant_weight_128x128", "fp8bw_requant_weights",
+              "fp8bw_gemm", "fp8bw_grouped_gemm", "fp8bw_gemm_bf16", "fp8bw_init",
+              "fp8bw_status_string", "fp8bw_last_device_error"]:
+        assert n in names
+
+
+def test_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in _declared():
+        assert hasattr(so, n), n
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.status_string(s) and lib.status_string(s) != "unknown status"
+    assert lib.status_string(99) == "unknown status"
+
+
+def test_host_validation(lib):
+    r = lib.raw
+    p = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+    odd = ctypes.c_void_p(0x10008)    # misaligned
+    N = None
+    # null pointers
+    assert r.fp8bw_gemm(0, 128, 128, 128, N, p, p, p, p, 128, 0, N) == 1
+    assert r.fp8bw_quant_act_1x128(N, 128, 128, 128, 0, p, p, N, N, N) == 1
+    # q_col without s_col
+    assert r.fp8bw_quant_act_1x128(p, 128, 128, 128, 0, p, p, p, N, N) == 1
+    # bad enums
+    assert r.fp8bw_gemm(3, 128, 128, 128, p, p, p, p, p, 128, 0, N) == 1
+    assert r.fp8bw_gemm(0, 128, 128, 128, p, p, p, p, p, 128, 2, N) == 1
+    assert r.fp8bw_quant_weight_128x128(p, 128, 128, 128, 5, p, p, N, N) == 1
+    # sizes not multiples of 128, misaligned pointers, bad leading dims
+    assert r.fp8bw_gemm(0, 130, 128, 128, p, p, p, p, p, 128, 0, N) == 2
+    assert r.fp8bw_gemm(0, 128, 128, 128, odd, p, p, p, p, 128, 0, N) == 2
+    assert r.fp8bw_gemm(0, 128, 128, 128, p, p, p, p, p, 132, 0, N) == 2
+    assert r.fp8bw_gemm(0, 128, 256, 128, p, p, p, p, p, 128, 0, N) == 1   # ldd < N
+    assert r.fp8bw_quant_act_1x128(p, 128, 200, 256, 0, p, p, N, N, N) == 2
+    assert r.fp8bw_quant_act_1x128(p, 128, 128, 100, 0, p, p, N, N, N) == 1   # ldx < K
+    assert r.fp8bw_gemm_bf16(128, 128, 100, p, p, p, 128, N) == 2
+    # grouped: bad G, too many experts, misaligned offsets
+    assert r.fp8bw_grouped_gemm(0, 0, p, 128, 128, 128, p, p, p, p, p, 0, N) == 1
+    assert r.fp8bw_grouped_gemm(0, 2000, p, 128, 128, 128, p, p, p, p, p, 0, N) == 7
+    assert r.fp8bw_grouped_gemm(0, 4, ctypes.c_void_p(0x10002), 128, 128, 128, p, p, p, p, p, 0, N) == 2
+    # too large
+    assert r.fp8bw_gemm(0, 1 << 31, 128, 128, p, p, p, p, p, 128, 0, N) == 7
+    # requant: a bad descriptor anywhere rejects the whole batch
+    d = (lib.fp8bw_weight_desc * 2)()
+    d[0] = lib.fp8bw_weight_desc(0x10000, 128, 128, 128, 0x10000, 0x10000, None)
+    d[1] = lib.fp8bw_weight_desc(0x10000, 128, 136, 136, 0x10000, 0x10000, None)
+    assert r.fp8bw_requant_weights(d, 2, 0, N) == 2
+    assert r.fp8bw_requant_weights(None, 1, 0, N) == 1

@@ -1,0 +1,137 @@
+"""GPU parity of the blockwise FP8 GEMMs (fprop / dgrad / wgrad) and of the
+BF16 comparison GEMM against the oracle's fp64 reference.
+
+Method: "NVIDIA NeMo RL erreicht 48% ..." section "Der technische
+Durchbruch": FP8 linear layers on 1x128 / 128x128 blockwise-scaled E4M3
+operands.  Acceptance: |y - y_ref| <= 1e-2 * sum_k |a_k b_k| + 1 bf16 ulp(y_ref),
+y_ref the fp64 product of the dequantized operands.  The operands come from
+the oracle's quantizer, so these tests do not depend on the GPU quantizers.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from util import bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def gpu_gemm(fb, kind, A, sA, B, sB, mode=0):
+    M, N = A.shape[0], B.shape[0]
+    D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_gemm(kind, dev(A), dev(sA), dev(B), dev(sB), D, mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    return bits(D)
+
+
+def operands(orc, X, W, dY, mode):
+    """Quantized operands of the three GEMMs of one linear layer."""
+    qx, sx, qxc, sxc = orc.quant_act_1x128(bits(X), mode)
+    qw, sw, qwT = orc.quant_weight_128x128(bits(W), mode)
+    qd, sd, qdc, sdc = orc.quant_act_1x128(bits(dY), mode)
+    return {
+        0: (qx, sx, qw, sw),          # fprop:  Y  = X W^T
+        1: (qd, sd, qwT, sw),         # dgrad:  dX = dY W
+        2: (qdc, sdc, qxc, sxc),      # wgrad:  dW = dY^T X
+    }
+
+
+def check(orc, y, kind, A, sA, B, sB):
+    yr, ya = orc.gemm_ref_tile(kind, A, sA, B, sB, 0, A.shape[0], 0, B.shape[0])
+    bad, worst = orc.check_tol(y, yr, ya)
+    assert bad == 0, f"kind {kind}: {bad} elements out of tolerance (worst ratio {worst:.3g})"
+    return worst
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_tiny_layer(fb, orc, kind, mode):
+    X, W, dY = workloads.tiny(0)
+    ops = operands(orc, X, W, dY, mode)[kind]
+    y = gpu_gemm(fb, kind, *ops, mode=mode)
+    worst = check(orc, y, kind, *ops)
+    assert worst < 0.05, worst   # fp32 promotion is far inside the 1% bound
+
+
+def rand_ops(rng, M, N, K, kind):
+    A = rng.integers(0, 0x7E, (M, K), dtype=np.uint8) | (rng.integers(0, 2, (M, K), dtype=np.uint8) << 7)
+    B = rng.integers(0, 0x7E, (N, K), dtype=np.uint8) | (rng.integers(0, 2, (N, K), dtype=np.uint8) << 7)
+    nK = K // 128
+    sA = (2.0 ** rng.uniform(-10, 4, (nK, M))).astype(np.float32)
+    shp = {0: (N // 128, nK), 1: (nK, N // 128), 2: (nK, N)}[kind]
+    sB = (2.0 ** rng.uniform(-10, 4, shp)).astype(np.float32)
+    return A, sA, B, sB
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("MNK", [(128, 128, 128), (384, 640, 384), (256, 384, 1024), (640, 256, 256)])
+def test_shapes(fb, orc, kind, MNK):
+    rng = np.random.default_rng(hash((kind,) + MNK) % 2**32)
+    ops = rand_ops(rng, *MNK, kind)
+    y = gpu_gemm(fb, kind, *ops)
+    check(orc, y, kind, *ops)
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_small_integers_exact(fb, orc, kind):
+    rng = np.random.default_rng(21 + kind)
+    pool = np.array([0x00, 0x38, 0x40, 0x44, 0xB8, 0xC0], np.uint8)   # 0, 1, 2, 3, -1, -2
+    M, N, K = 256, 384, 256
+    A = rng.choice(pool, (M, K))
+    B = rng.choice(pool, (N, K))
+    sA = np.ones((K // 128, M), np.float32)
+    sB = {0: np.ones((N // 128, K // 128)), 1: np.ones((K // 128, N // 128)),
+          2: np.ones((K // 128, N))}[kind].astype(np.float32)
+    y = gpu_gemm(fb, kind, A, sA, B, sB)
+    yr, _ = orc.gemm_ref_tile(kind, A, sA, B, sB, 0, M, 0, N)
+    assert np.abs(yr).max() <= 256
+    got = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got, yr)
+
+
+def test_identity_and_zero_rows(fb, orc):
+    rng = np.random.default_rng(2)
+    M = N = K = 256
+    A, sA, _, _ = rand_ops(rng, M, N, K, 0)
+    A[128:] = 0
+    B = np.zeros((N, K), np.uint8)
+    np.fill_diagonal(B, 0x38)
+    sB = np.ones((N // 128, K // 128), np.float32)
+    y = gpu_gemm(fb, 0, A, sA, B, sB)
+    got = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).float().numpy()
+    yr, _ = orc.gemm_ref_tile(0, A, sA, B, sB, 0, M, 0, N)
+    want = torch.from_numpy(yr).float().to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(got, want)
+    assert np.all(got[128:] == 0)
+
+
+def test_ldd(fb, orc):
+    rng = np.random.default_rng(4)
+    A, sA, B, sB = rand_ops(rng, 256, 256, 256, 0)
+    Dbig = torch.zeros((256, 512), dtype=torch.bfloat16, device=DEV)
+    D = Dbig[:, 128:384]
+    fb.fp8bw_gemm(0, dev(A), dev(sA), dev(B), dev(sB), D)
+    torch.cuda.synchronize()
+    check(orc, bits(D), 0, A, sA, B, sB)
+    assert torch.all(Dbig[:, :128] == 0) and torch.all(Dbig[:, 384:] == 0)
+
+
+@pytest.mark.parametrize("MNK", [(256, 512, 512), (128, 384, 256)])
+def test_bf16_gemm(fb, orc, MNK):
+    M, N, K = MNK
+    g = torch.Generator().manual_seed(M + N + K)
+    A = torch.randn((M, K), generator=g).to(torch.bfloat16)
+    B = torch.randn((N, K), generator=g).to(torch.bfloat16)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_gemm_bf16(A.to(DEV), B.to(DEV), D)
+    torch.cuda.synchronize()
+    yr, ya = orc.gemm_bf16_ref_tile(bits(A), bits(B), 0, M, 0, N)
+    bad, worst = orc.check_tol(bits(D), yr, ya, rel=1e-3)
+    assert bad == 0, worst
