@@ -1,0 +1,440 @@
+#!/usr/bin/env python3
+"""Benchmark of the blockwise-scaled FP8 linear-layer hot path on B200.
+
+One step = one training pass of the four Llama-3.1-8B-like linear layers
+(tokens M = 8192; qkv 4096->6144, o_proj 4096->4096, gate_up 4096->28672,
+down 14336->4096) through the library:
+  requant all four weights (one batched call, the per-step recalibration),
+  then per layer: quantize X (row-wise + column-wise copy), fprop,
+  quantize dY (row-wise + column-wise copy), dgrad, wgrad.
+Metric: FP8 blockwise linear TFLOP/s (fprop+dgrad+wgrad FLOPs / step time).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+With N > 1 (launched by torchrun) every rank runs an independent replica
+(the path has no exchange step); value = all ranks' FLOPs / max time.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 blockwise linear TFLOP/s (fprop+dgrad+wgrad) & % FP8 peak; quant GB/s"
+WORKLOAD = "llama3.1-8b-like linear layers, M=8192 tokens, fprop+dgrad+wgrad + act/weight quant + per-step requant"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="fp8bw", choices=["fp8bw", "reference"])
+    p.add_argument("--mode", default="fp32", choices=["fp32", "pow2"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_burst": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_burst": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+# ------------------------------------------------------------ clocks ------
+class ClockSampler:
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------- workload -----
+class Layer:
+    def __init__(self, name, K, N, M, dev, seed=0):
+        self.name, self.K, self.N, self.M = name, K, N, M
+        X, W, dY = workloads.llama_layer(name, seed=seed, device=dev, M=M)
+        self.X, self.W, self.dY = X, W, dY
+        u8, f32 = torch.uint8, torch.float32
+        e = lambda *s, dt=u8: torch.empty(s, dtype=dt, device=dev)  # noqa: E731
+        self.qx, self.sx, self.qxc, self.sxc = e(M, K), e(K // 128, M, dt=f32), e(K, M), e(M // 128, K, dt=f32)
+        self.qd, self.sd, self.qdc, self.sdc = e(M, N), e(N // 128, M, dt=f32), e(N, M), e(M // 128, N, dt=f32)
+        self.qw, self.sw, self.qwT = e(N, K), e(N // 128, K // 128, dt=f32), e(K, N)
+        bf = torch.bfloat16
+        self.Y, self.dX, self.dW = e(M, N, dt=bf), e(M, K, dt=bf), e(N, K, dt=bf)
+
+    @property
+    def flops(self):
+        return 3 * 2 * self.M * self.N * self.K
+
+    def act_bytes(self, rows, cols):
+        # read bf16 + row codes + col codes + two fp32 scale grids
+        return rows * cols * (2 + 1 + 1) + 2 * 4 * rows * cols // 128
+
+    @property
+    def weight_bytes(self):
+        return self.N * self.K * (2 + 1 + 1) + 4 * self.N * self.K // (128 * 128)
+
+
+def build_layers(dev, M=workloads.LLAMA8B_TOKENS):
+    return [Layer(n, K, N, M, dev) for (n, K, N) in workloads.LLAMA8B_LAYERS]
+
+
+def run_step(fb, layers, mode, ev=None):
+    """One step; if `ev` is a dict, records (start, end) events per call kind."""
+    def rec(kind, fn):
+        if ev is None:
+            fn()
+            return
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        ev.setdefault(kind, []).append((s, e))
+
+    rec("requant", lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT) for l in layers], mode))
+    for l in layers:
+        rec("quant_act", lambda: fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc))
+        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode))
+        rec("quant_act", lambda: fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc))
+        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode))
+        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode))
+
+
+LAUNCHES_PER_STEP = 1 + 4 * 5   # requant + per layer (2 quant_act + 3 gemm)
+
+
+def bf16_ratio(fb, layers, reps=3):
+    """Same three GEMMs per layer through the library's BF16 path."""
+    dev = layers[0].X.device
+    tot_flops, tot_ms = 0.0, 0.0
+    for l in layers:
+        WT = l.W.t().contiguous()
+        dYT = l.dY.t().contiguous()
+        XT = l.X.t().contiguous()
+        D1 = torch.empty((l.M, l.N), dtype=torch.bfloat16, device=dev)
+        D2 = torch.empty((l.M, l.K), dtype=torch.bfloat16, device=dev)
+        D3 = torch.empty((l.N, l.K), dtype=torch.bfloat16, device=dev)
+        calls = [lambda: fb.fp8bw_gemm_bf16(l.X, l.W, D1), lambda: fb.fp8bw_gemm_bf16(l.dY, WT, D2),
+                 lambda: fb.fp8bw_gemm_bf16(dYT, XT, D3)]
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            for c in calls:
+                c()
+        e.record()
+        torch.cuda.synchronize()
+        tot_ms += s.elapsed_time(e) / reps
+        tot_flops += l.flops
+        del WT, dYT, XT, D1, D2, D3
+    return tot_flops / (tot_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------- CPU oracle ----
+_ORC = {}
+
+
+def _oracle_operands(name):
+    """The oracle's quantized operands for a slice of one layer's fprop: the
+    first 128 token rows of X and the first 512 rows of W (full K)."""
+    if name not in _ORC:
+        import oracle
+        X, W, _ = workloads.llama_layer(name, seed=0, device="cpu", M=128)
+        xb = X.view(torch.int16).numpy().view(np.uint16)
+        wb = np.ascontiguousarray(W[:512].view(torch.int16).numpy().view(np.uint16))
+        qx, sx, _, _ = oracle.quant_act_1x128(xb, 0, colwise=False)
+        qw, sw, _ = oracle.quant_weight_128x128(wb, 0, transposed=False)
+        _ORC[name] = (qx, sx, qw, sw)
+    return _ORC[name]
+
+
+def _oracle_gemm(name, rows, cols):
+    import oracle
+    qx, sx, qw, sw = _oracle_operands(name)
+    t0 = time.perf_counter()
+    oracle.gemm_ref_tile(0, qx, sx, qw, sw, 0, rows, 0, cols)
+    dt = time.perf_counter() - t0
+    return 2.0 * rows * cols * qx.shape[1], dt
+
+
+def _cores():
+    cores = len(os.sched_getaffinity(0))
+    return min(cores, int(os.environ.get("OMP_NUM_THREADS", cores)))
+
+
+def oracle_sample(target_s=10.0, rows=8, cols=512):
+    """Times the CPU oracle's fp64 reference GEMM on a bounded sample of the
+    step (blocks of `rows` x `cols` outputs of each layer's fprop, full K),
+    cycling through the layers until about `target_s` seconds of GEMM work."""
+    names = [n for n, _, _ in workloads.LLAMA8B_LAYERS]
+    for n in names:
+        _oracle_operands(n)
+    flops = secs = 0.0
+    done = []
+    i = 0
+    while secs < target_s and i < 1000:
+        n = names[i % len(names)]
+        f, dt = _oracle_gemm(n, rows, cols)
+        flops += f
+        secs += dt
+        done.append(n)
+        i += 1
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"fp64 reference GEMM (oracle.gemm_ref_tile, fprop) on {i} blocks of "
+                      f"{rows} rows x {cols} cols x full K cycling over the four layers "
+                      f"({secs:.1f} s of CPU work), operands quantized by the oracle; "
+                      "TFLOP/s = 2*rows*cols*K / time"}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    names = [n for n, _, _ in workloads.LLAMA8B_LAYERS]
+    for n in names:
+        _oracle_operands(n)
+    flops = secs = 0.0
+    for i in range(args.warmup + args.steps):
+        f, dt = _oracle_gemm(names[i % 4], 2, 256)
+        if i >= args.warmup:
+            flops += f
+            secs += dt
+    val = flops / secs / 1e12
+    sample = ("one step = fp64 reference GEMM (oracle.gemm_ref_tile, fprop) of 2 rows x 256 "
+              "cols x full K of one layer, cycling over the four layers")
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs * 1e3 / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD + " (CPU oracle, bounded sample)"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- main -----
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist:
+            dist.barrier()
+
+    from blockwise_scaled_fp8_fp8bw_b200 import build as _b
+    if rank == 0 and not os.path.exists(os.path.join(ROOT, "blockwise_scaled_fp8_fp8bw_b200", "libfp8bw.so")):
+        _b.build()
+    barrier()
+    import blockwise_scaled_fp8_fp8bw_b200 as fb
+    fb.fp8bw_init(local)
+    mode = fb.FP8BW_SCALE_POW2 if args.mode == "pow2" else fb.FP8BW_SCALE_FP32
+    dev = torch.device("cuda", local)
+    layers = build_layers(dev)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        run_step(fb, layers, mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+
+    # ---- timed region: K steps, per-call events, clocks sampled meanwhile
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = {}
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        run_step(fb, layers, mode, ev)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ck = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    st = fb.fp8bw_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error: {fb.status_string(st)}")
+    if dist:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    step_flops = sum(l.flops for l in layers)
+    value = step_flops * args.steps * world / (ms_total * 1e-3) / 1e12
+
+    def kind_ms(k):
+        return sum(s.elapsed_time(e) for s, e in ev[k])
+
+    gemm_ms = kind_ms("gemm") / (args.steps)
+    quant_ms = kind_ms("quant_act") / args.steps
+    req_ms = kind_ms("requant") / args.steps
+    gemm_tflops = step_flops / (gemm_ms * 1e-3) / 1e12
+    gemm_launch_ms = kind_ms("gemm") / len(ev["gemm"])
+    quant_bytes = sum(l.act_bytes(l.M, l.K) + l.act_bytes(l.M, l.N) for l in layers)
+    req_bytes = sum(l.weight_bytes for l in layers)
+    pk = peaks()
+    timed_long = ms_total > 1000.0
+    fp8_peak = 2.0 * (pk["bf16_sustained"] if timed_long else pk["bf16_burst"])
+
+    # ---- BF16 comparison GEMMs (outside the timed region)
+    bf16 = bf16_ratio(fb, layers) if rank == 0 else None
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = [(l.X.cpu().pin_memory(), l.W.cpu().pin_memory(), l.dY.cpu().pin_memory()) for l in layers]
+        host_out = [(torch.empty_like(l.Y, device="cpu").pin_memory(), torch.empty_like(l.dX, device="cpu").pin_memory(),
+                     torch.empty_like(l.dW, device="cpu").pin_memory()) for l in layers]
+        h2d = sum(x.numel() * 2 + w.numel() * 2 + d.numel() * 2 for x, w, d in host_in)
+        d2h = sum(a.numel() * 2 + b.numel() * 2 + c.numel() * 2 for a, b, c in host_out)
+
+        def e2e_step():
+            for l, (x, w, d) in zip(layers, host_in):
+                l.X.copy_(x, non_blocking=True)
+                l.W.copy_(w, non_blocking=True)
+                l.dY.copy_(d, non_blocking=True)
+            run_step(fb, layers, mode)
+            for l, (a, b, c) in zip(layers, host_out):
+                a.copy_(l.Y, non_blocking=True)
+                b.copy_(l.dX, non_blocking=True)
+                c.copy_(l.dW, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e.record()
+        torch.cuda.synchronize()
+        e_ms = s.elapsed_time(e)
+        if dist:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": step_flops * args.e2e_steps * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample(target_s=10.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": workloads.LLAMA8B_TOKENS,
+                       "layers": [f"{n}:{K}->{N}" for n, K, N in workloads.LLAMA8B_LAYERS],
+                       "scale_mode": args.mode, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (per-step working set > 1.5 GB)"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp8_peak, "traffic": None,
+                         "kernel": "k_gemm_fp8 (all fprop/dgrad/wgrad launches)",
+                         "peak_note": f"FP8 = 2 x {pk['src']} cuBLAS bf16 "
+                                      f"({'sustained' if timed_long else 'burst'})",
+                         "avg_launch_ms": gemm_launch_ms},
+            "calls": {"gemm_ms_per_step": gemm_ms, "gemm_tflops": gemm_tflops,
+                      "quant_act_ms_per_step": quant_ms, "quant_act_gbs": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                      "requant_ms_per_step": req_ms, "requant_gbs": req_bytes / (req_ms * 1e-3) / 1e9,
+                      "hbm_peak_gbs": pk["hbm_gbs"],
+                      "bf16_gemm_tflops": bf16, "fp8_over_bf16": (gemm_tflops / bf16) if bf16 else None,
+                      "requant_over_step": req_ms / ms_step},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": ck,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -56,8 +56,12 @@ def test_tiny_layer(fb, orc, kind, mode):
     X, W, dY = workloads.tiny(0)
     ops = operands(orc, X, W, dY, mode)[kind]
     y = gpu_gemm(fb, kind, *ops, mode=mode)
-    worst = check(orc, y, kind, *ops)
-    assert worst < 0.05, worst   # fp32 promotion is far inside the 1% bound
+    check(orc, y, kind, *ops)
+    # FP32 accumulation and promotion leave the result far inside the 1%
+    # gate: within 1e-3 * sum|ab| + 1 ulp (bf16 output rounding dominates).
+    yr, ya = orc.gemm_ref_tile(kind, *ops, 0, ops[0].shape[0], 0, ops[2].shape[0])
+    bad, worst = orc.check_tol(y, yr, ya, rel=1e-3)
+    assert bad == 0, worst
 
 
 def rand_ops(rng, M, N, K, kind):
@@ -91,9 +95,10 @@ def test_small_integers_exact(fb, orc, kind):
           2: np.ones((K // 128, N))}[kind].astype(np.float32)
     y = gpu_gemm(fb, kind, A, sA, B, sB)
     yr, _ = orc.gemm_ref_tile(kind, A, sA, B, sB, 0, M, 0, N)
-    assert np.abs(yr).max() <= 256
+    # integer sums are exact in fp32, so the only rounding is the final bf16
+    want = torch.from_numpy(yr).float().to(torch.bfloat16).double().numpy()
     got = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).double().numpy()
-    np.testing.assert_array_equal(got, yr)
+    np.testing.assert_array_equal(got, want)
 
 
 def test_identity_and_zero_rows(fb, orc):
