@@ -47,6 +47,10 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--case", default=None,
+                   help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
+                        "requant|bf16_fprop, on --layer")
+    p.add_argument("--layer", default="gate_up", choices=[n for n, _, _ in workloads.LLAMA8B_LAYERS])
     return p.parse_args()
 
 
@@ -281,11 +285,52 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------- one case -----
+def run_case(args):
+    """Times a single call of one layer (used for ncu captures and sweeps)."""
+    import blockwise_scaled_fp8_fp8bw_b200 as fb
+    torch.cuda.set_device(0)
+    fb.fp8bw_init(0)
+    mode = fb.FP8BW_SCALE_POW2 if args.mode == "pow2" else fb.FP8BW_SCALE_FP32
+    name = args.layer
+    K, N = [(k, n) for nm, k, n in workloads.LLAMA8B_LAYERS if nm == name][0]
+    l = Layer(name, K, N, workloads.LLAMA8B_TOKENS, torch.device("cuda", 0))
+    fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode)
+    fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)
+    fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)
+    calls = {
+        "fprop": (lambda: fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode), l.flops / 3, "TFLOP/s"),
+        "dgrad": (lambda: fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode), l.flops / 3, "TFLOP/s"),
+        "wgrad": (lambda: fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode), l.flops / 3, "TFLOP/s"),
+        "quant_x": (lambda: fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc), l.act_bytes(l.M, l.K), "GB/s"),
+        "quant_dy": (lambda: fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc), l.act_bytes(l.M, l.N), "GB/s"),
+        "requant": (lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode), l.weight_bytes, "GB/s"),
+        "bf16_fprop": (lambda: fb.fp8bw_gemm_bf16(l.X, l.W, l.Y), l.flops / 3, "TFLOP/s"),
+    }
+    fn, work, unit = calls[args.case]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    ms = s.elapsed_time(e) / max(args.steps, 1)
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"case": args.case, "layer": name, "mode": args.mode, "ms": ms, unit: rate}), flush=True)
+
+
 # --------------------------------------------------------------- main -----
 def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.case:
+        run_case(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

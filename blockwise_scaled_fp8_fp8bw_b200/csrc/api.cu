@@ -10,7 +10,7 @@
 namespace fp8bw {
 cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
                              uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
-                             cudaStream_t st);
+                             int num_sms, cudaStream_t st);
 cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, int mode,
                                 uint8_t* q, float* s, uint8_t* qT, cudaStream_t st);
 cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cudaStream_t st);
@@ -114,7 +114,7 @@ FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K
   fp8bw_status s = current(&sms);
   if (s != FP8BW_OK) return s;
   if (M == 0 || K == 0) return FP8BW_OK;
-  return from_cuda(fp8bw::launch_quant_act(x, M, K, ldx, mode, q_row, s_row, q_col, s_col,
+  return from_cuda(fp8bw::launch_quant_act(x, M, K, ldx, mode, q_row, s_row, q_col, s_col, sms,
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 

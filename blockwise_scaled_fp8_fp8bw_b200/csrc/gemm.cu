@@ -7,30 +7,37 @@
 // BF16 peak.  Section "Leistungsgewinne in der Praxis": the Qwen3-30B MoE
 // model trains with the same recipe (grouped expert GEMMs).
 //
-// FP8 kernel design (one CTA per SM, persistent, 384 threads):
-//   warp 0      TMA producer: per 128-wide K chunk, one 128x128 A tile and
-//               one 256x128 B tile (E4M3, 128-byte swizzle) into a 4-stage
-//               shared-memory ring.
-//   warp 1      MMA issuer: four tcgen05.mma kind::f8f6f4 (M=128, N=256,
-//               K=32) per chunk into one of two TMEM chunk accumulators
-//               (2 x 256 columns = all 512 TMEM columns).
+// FP8 kernel (persistent, 384 threads per CTA, one CTA per SM).  Output tile
+// 256x256 per CTA pair (PAIR: a 2-CTA cluster, tcgen05 cta_group::2, M=256
+// split over the two SMs, each SM holding its own 128 A rows and half of the
+// 256 B rows) or 128x256 per CTA (grouped fprop/dgrad, whose 128-row expert
+// segments cannot share a 256-row tile).  Roles per CTA:
+//   warp 0      TMA producer: per 128-wide K chunk, the CTA's 128x128 A tile
+//               and its B tile (128 or 256 rows) into a shared-memory ring
+//               (E4M3, 128-byte swizzle).  In a pair both CTAs count their
+//               bytes on the first CTA's barrier.
+//   warp 1      MMA issuer (first CTA of a pair only): four tcgen05.mma
+//               kind::f8f6f4 (K = 32) per chunk into one of two TMEM chunk
+//               accumulators (2 x 256 columns = all of TMEM), then commits
+//               to the stage-empty and chunk-full barriers of both CTAs.
 //   warp 2      scale loader: the chunk's 128 A-row scales and the B scales
 //               (2 block scales, or 256 column scales for wgrad) into an
 //               8-slot shared ring with cp.async.
 //   warps 4-11  promotion: each thread owns one accumulator row and 128
-//               columns; per chunk it reads the chunk product from TMEM
-//               (tcgen05.ld), multiplies by sA*sB in fp32 and adds it to
-//               its register accumulator (packed f32x2 FMAs).  The chunk
-//               accumulator is released right after the loads, so the MMA
-//               of chunk c+1 overlaps the promotion of chunk c.  At the end
-//               of a tile the rows are rounded to bf16 and stored.
-// Registers: warpgroup 0 drops to 40 per thread, the two promotion
-// warpgroups rise to 232 (128 accumulators + staging); 40*128 + 232*256 =
-// 64512 = 384 * 168, the launch allocation (checked on the host).
+//               columns; per chunk it reads the chunk product from TMEM,
+//               multiplies by sA*sB in fp32 and adds it to its registers
+//               (packed f32x2 FMAs), releasing the TMEM buffer as soon as it
+//               is read so the MMA of the next chunk overlaps.  At the end
+//               of a tile the rows are rounded to bf16, staged in shared
+//               memory (64-byte swizzle) and written by TMA stores.
+// Registers: warpgroup 0 drops to 40 per thread, the promotion warpgroups
+// rise to 232 (128 accumulators + 64 staging); 40*128 + 232*256 = 64512 =
+// 384 * 168, the launch allocation (checked on the host before launch).
 // Every wait is bounded; on a timeout the kernel latches an error bit and
 // leaves its loops.
 
 #include "common.cuh"
+#include "tmap.cuh"
 
 namespace fp8bw {
 
@@ -39,19 +46,25 @@ __device__ uint32_t g_gemm_error;
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 128;
-constexpr int kStages = 4;
-constexpr int kScaleStages = 8;
 constexpr int kThreads = 384;
-constexpr uint32_t kATile = BM * BK;  // 16 KB
-constexpr uint32_t kBTile = BN * BK;  // 32 KB
-constexpr uint32_t kStageBytes = kATile + kBTile;
+constexpr int kScaleStages = 8;
+constexpr uint32_t kATile = BM * BK;  // 16 KB: one CTA's A rows
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = FP8BW_MAX_EXPERTS;
+constexpr uint32_t kEpiBytes = 2048;  // per promotion warp: 32 rows x 32 bf16
 
-constexpr uint32_t kIdescF8 = idesc_make(0, 0, BM, BN);   // E4M3 x E4M3 -> F32
-constexpr uint32_t kIdescBF16 = idesc_make(1, 1, BM, BN); // BF16 x BF16 -> F32
+template <bool PAIR>
+struct Cfg {
+  static constexpr uint32_t kBTile = PAIR ? (BN / 2) * BK : BN * BK;  // this CTA's B rows
+  static constexpr uint32_t kStageBytes = kATile + kBTile;
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr uint32_t kIdesc = idesc_make(0, 0, PAIR ? 2 * BM : BM, BN);  // E4M3 -> F32
+  static constexpr uint32_t kTemptyCount = PAIR ? 16 : 8;
+};
 
-constexpr int kRegsLow = 40, kRegsHigh = 232, kRegsLaunch = 168;
+constexpr uint32_t kIdescBF16 = idesc_make(1, 1, BM, BN);  // BF16 x BF16 -> F32
+
+constexpr int kRegsLow = 56, kRegsHigh = 224, kRegsLaunch = 168;
 static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
 
 struct ScaleSlot {
@@ -59,8 +72,9 @@ struct ScaleSlot {
   float sb[256];
 };
 
+constexpr int kMaxStages = 6;
 struct Bars {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t sfull[kScaleStages], sempty[kScaleStages];
   uint64_t tfull[2], tempty[2];
   uint32_t tmem_base;
@@ -73,21 +87,28 @@ struct GemmArgs {
   int m_tiles, n_tiles, tiles, band;
   const float* sA;     // [K/128][M]
   const float* sB;     // per kind
-  uint16_t* D;
-  int64_t ldd;
   const int32_t* offsets;  // grouped: device [G+1]
   int G;
+  uint16_t* D;         // BF16 kernel only (the FP8 kernel stores through a tensor map)
+  int64_t ldd;
 };
 
-constexpr size_t kSmemFp8 = 1024 + size_t(kStages) * kStageBytes +
-                            size_t(kScaleStages) * sizeof(ScaleSlot) + sizeof(Bars) +
-                            sizeof(int32_t) * (kMaxGroups + 1);
+template <bool PAIR>
+constexpr size_t smem_fp8() {
+  return 1024 + size_t(Cfg<PAIR>::kStages) * Cfg<PAIR>::kStageBytes +
+         size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * kEpiBytes + sizeof(Bars) +
+         sizeof(int32_t) * (kMaxGroups + 1);
+}
+static_assert(smem_fp8<true>() <= 232448 && smem_fp8<false>() <= 232448, "shared memory budget");
 
 struct TileInfo {
   int mt, nt, g, kb0, kb1;
   bool skip;
 };
 
+// Tile t -> (m tile, n tile, expert, K-chunk range).  M tiles are 256 rows
+// for a pair, 128 otherwise; dense tiles go in bands of `band` M tiles so
+// that the CTAs running at once share A and B panels in L2.
 template <int KIND, bool GROUPED>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off) {
   TileInfo ti;
@@ -132,22 +153,28 @@ __device__ __forceinline__ void raise_timeout(Bars* bars) {
   atomicExch(&bars->abort, 1);
 }
 
-template <int KIND, bool GROUPED>
+template <int KIND, bool GROUPED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const GemmArgs a) {
+               const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
+  using C = Cfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(smem + kStages * kStageBytes);
+  uint8_t* epi_base = smem + C::kStages * C::kStageBytes;  // 1024-aligned
+  ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kEpiBytes);
   Bars* bars = reinterpret_cast<Bars*>(slots + kScaleStages);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int cta_slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile-loop index
+  const int cta_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
@@ -157,41 +184,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->tfull[i]), 1);
-      mbar_init(smem_u32(&bars->tempty[i]), 8);
+      mbar_init(smem_u32(&bars->tempty[i]), C::kTemptyCount);
     }
     bars->abort = 0;
     bars->bad_offsets = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (GROUPED) {
     for (int i = threadIdx.x; i <= a.G; i += kThreads) s_off[i] = a.offsets[i];
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (GROUPED) {
     // Offsets must start at 0, be non-decreasing multiples of 128 and end
     // within the token matrix; otherwise nothing is computed or written.
+    int bad = 0;
     for (int i = threadIdx.x; i < a.G; i += kThreads) {
       const int o0 = s_off[i], o1 = s_off[i + 1];
-      if (o1 < o0 || (o1 & 127) || (i == 0 && o0 != 0)) bars->bad_offsets = 1;
+      if (o1 < o0 || (o1 & 127) || (i == 0 && o0 != 0)) bad = 1;
     }
     if (threadIdx.x == 0) {
       const int mtot = (KIND == FP8BW_WGRAD) ? a.K : a.M;
-      if (s_off[a.G] > mtot || s_off[a.G] < 0) bars->bad_offsets = 1;
+      if (s_off[a.G] > mtot || s_off[a.G] < 0) bad = 1;
     }
-    __syncthreads();
-    if (bars->bad_offsets) {
+    if (__syncthreads_or(bad)) {
       if (threadIdx.x == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
-      if (warp == 1) tmem_dealloc(bars->tmem_base, kTmemCols);
+      tc_fence_before();
+      if (PAIR) cluster_sync();
+      if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(bars->tmem_base, kTmemCols);
+        else tmem_dealloc(bars->tmem_base, kTmemCols);
+      }
       return;
     }
   }
   const uint32_t tmem = bars->tmem_base;
+  // Barriers the MMA waits on live in the first CTA of a pair.
+  const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&bars->full[0]), 0) : smem_u32(&bars->full[0]);
+  const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&bars->tempty[0]), 0) : smem_u32(&bars->tempty[0]);
 
   if (warp < 4) {
     regs_dec<kRegsLow>();
@@ -203,69 +243,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
         const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
         if (ti.skip) continue;
+        const int arow = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
             raise_timeout(bars);
             goto done;
           }
           if (lane == 0) {
-            const uint32_t full = smem_u32(&bars->full[stage]);
-            const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
-            mbar_arrive_expect_tx(full, kStageBytes);
-            tma_load_2d(sa, &tmA, full, kb * BK, ti.mt * BM);
-            if (GROUPED && KIND != FP8BW_WGRAD)
-              tma_load_3d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN, ti.g);
-            else
-              tma_load_2d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN);
+            const uint32_t full = full0 + stage * 8;
+            const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+            if (PAIR) {
+              if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[stage]), 2 * C::kStageBytes);
+              tma_load_2d_pair(sa, &tmA, full, kb * BK, arow);
+              tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
+            } else {
+              mbar_arrive_expect_tx(full, C::kStageBytes);
+              tma_load_2d(sa, &tmA, full, kb * BK, arow);
+              if (GROUPED && KIND != FP8BW_WGRAD)
+                tma_load_3d(sa + kATile, &tmB, full, kb * BK, brow, ti.g);
+              else
+                tma_load_2d(sa + kATile, &tmB, full, kb * BK, brow);
+            }
           }
           __syncwarp();
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (bars->abort) break;
       }
     } else if (warp == 1) {
       // ------------------------------------------------- MMA issuer -----
-      int stage = 0;
-      uint32_t phase = 0;
-      int buf = 0;
-      uint32_t bphase = 0;
-      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
-        if (ti.skip) continue;
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1) ||
-              !mbar_wait(smem_u32(&bars->full[stage]), phase)) {
-            raise_timeout(bars);
-            goto done;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
-            const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
-            const uint32_t d = tmem + buf * BN;
+      if (leader) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int t = cta_slot; t < a.tiles; t += cta_step) {
+          const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          if (ti.skip) continue;
+          for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+            if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1) ||
+                !mbar_wait(smem_u32(&bars->full[stage]), phase)) {
+              raise_timeout(bars);
+              goto done;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+              const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+              const uint32_t d = tmem + buf * BN;
 #pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)  // +32 bytes = +2 in the >>4 address field
-              umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, kIdescF8, kk > 0 ? 1u : 0u);
-            umma_commit(smem_u32(&bars->empty[stage]));
-            umma_commit(smem_u32(&bars->tfull[buf]));
+              for (int kk = 0; kk < BK / 32; ++kk) {  // +32 bytes = +2 in the >>4 address field
+                if (PAIR) umma_f8f6f4_pair(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
+                else umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
+              }
+              if (PAIR) {
+                umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
+                umma_commit_pair(smem_u32(&bars->tfull[buf]), 0x3);
+              } else {
+                umma_commit(smem_u32(&bars->empty[stage]));
+                umma_commit(smem_u32(&bars->tfull[buf]));
+              }
+            }
+            __syncwarp();
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            if (++buf == 2) { buf = 0; bphase ^= 1; }
           }
-          __syncwarp();
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-          if (++buf == 2) { buf = 0; bphase ^= 1; }
+          if (bars->abort) break;
         }
-        if (bars->abort) break;
       }
     } else if (warp == 2) {
       // ------------------------------------------------ scale loader ----
       int ss = 0;
       uint32_t sphase = 0;
       const int nKb = a.K / BK, nNb = a.N / 128;
-      for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
         const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
         if (ti.skip) continue;
+        const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const bool rows_ok = row0 < a.M;
         const float* sBg = a.sB;
         if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
@@ -274,7 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             goto done;
           }
           ScaleSlot* sl = &slots[ss];
-          cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + ti.mt * BM + lane * 4);
+          if (rows_ok)
+            cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + row0 + lane * 4);
           if (KIND == FP8BW_WGRAD) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -301,18 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------- promotion --
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int half = (warp - 4) >> 2;  // column half of the 256-wide tile
+    uint8_t* epi = epi_base + (warp - 4) * kEpiBytes;
+    const uint32_t epi_s = smem_u32(epi);
     int ss = 0;
     uint32_t sphase = 0;
     int buf = 0;
     uint32_t bphase = 0;
-    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
+    for (int t = cta_slot; t < a.tiles; t += cta_step) {
       const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
       if (ti.skip) continue;
-      const int row = ti.mt * BM + q * 32 + lane;
+      const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
       const int col0 = ti.nt * BN + half * 128;
-      const bool valid = col0 < a.N;
-      uint16_t* drow = a.D + (GROUPED && KIND == FP8BW_WGRAD ? (size_t)ti.g * a.M * a.N : 0) +
-                       (size_t)row * a.ldd + col0;
       float2 acc[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.f, 0.f);
@@ -326,59 +385,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         const ScaleSlot* sl = &slots[ss];
         const float sa = sl->sa[q * 32 + lane];
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
+        // Two rounds of two 32-column loads: one wait per 64 columns keeps
+        // the staging at 64 registers next to the 128 accumulators.
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          uint32_t r[32];
-          tmem_ld32(taddr + p * 32, r);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[2][32];
+          tmem_ld32(taddr + h2 * 64, r[0]);
+          tmem_ld32(taddr + h2 * 64 + 32, r[1]);
           tmem_wait_ld();
-          if (KIND == FP8BW_WGRAD) {
-            const float2 sa2 = make_float2(sa, sa);
-            const float2* sb2 = reinterpret_cast<const float2*>(&sl->sb[half * 128 + p * 32]);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float2 sc = fmul2(sa2, sb2[j]);
-              acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
-                                      sc, acc[p * 16 + j]);
+          if (h2 == 1) {
+            // chunk fully read: hand the TMEM buffer back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
+              else mbar_arrive(smem_u32(&bars->tempty[buf]));
             }
-          } else {
-            const float s = sa * sl->sb[half];
-            const float2 s2 = make_float2(s, s);
+          }
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
-                                      s2, acc[p * 16 + j]);
+          for (int p2 = 0; p2 < 2; ++p2) {
+            const int p = h2 * 2 + p2;
+            if (KIND == FP8BW_WGRAD) {
+              const float2 sa2 = make_float2(sa, sa);
+              const float2* sb2 = reinterpret_cast<const float2*>(&sl->sb[half * 128 + p * 32]);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float2 sc = fmul2(sa2, sb2[j]);
+                acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1])),
+                                        sc, acc[p * 16 + j]);
+              }
+            } else {
+              const float s = sa * sl->sb[half];
+              const float2 s2 = make_float2(s, s);
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1])),
+                                        s2, acc[p * 16 + j]);
+            }
           }
         }
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&bars->tempty[buf]));
-          mbar_arrive(smem_u32(&bars->sempty[ss]));
-        }
+        if (lane == 0) mbar_arrive(smem_u32(&bars->sempty[ss]));
         if (++ss == kScaleStages) { ss = 0; sphase ^= 1; }
         if (++buf == 2) { buf = 0; bphase ^= 1; }
       }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(drow);
+      // ---- epilogue: bf16 rows through shared memory, TMA stores of 32x32
+      // pieces (rows / columns outside the output are clipped by the TMA).
+      const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
+      // (a pair's second CTA past the last row of M computed nothing real)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+      for (int p = 0; p < 4 && row0 < a.M; ++p) {
+        if (lane == 0) bulk_wait_read0();   // the previous piece has left the buffer
+        __syncwarp();
+        // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
           uint4 o;
-          o.x = pack_bf16x2(acc[4 * j + 0].x, acc[4 * j + 0].y);
-          o.y = pack_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y);
-          o.z = pack_bf16x2(acc[4 * j + 2].x, acc[4 * j + 2].y);
-          o.w = pack_bf16x2(acc[4 * j + 3].x, acc[4 * j + 3].y);
-          dst[j] = o;
+          o.x = pack_bf16x2(acc[p * 16 + 4 * c + 0].x, acc[p * 16 + 4 * c + 0].y);
+          o.y = pack_bf16x2(acc[p * 16 + 4 * c + 1].x, acc[p * 16 + 4 * c + 1].y);
+          o.z = pack_bf16x2(acc[p * 16 + 4 * c + 2].x, acc[p * 16 + 4 * c + 2].y);
+          o.w = pack_bf16x2(acc[p * 16 + 4 * c + 3].x, acc[p * 16 + 4 * c + 3].y);
+          *reinterpret_cast<uint4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, epi_s, col0 + p * 32, drow);
+          bulk_commit();
         }
       }
       if (bars->abort) break;
     }
   }
 done:
+  if (warp >= 4 && lane == 0) bulk_wait0();  // TMA stores have finished
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -388,6 +474,8 @@ done:
 // whole K loop, and the 8 epilogue warps drain a finished tile (double
 // buffered in TMEM) while the next tile accumulates.
 constexpr int BK16 = 64;
+constexpr int kStages = 4;
+constexpr uint32_t kStageBytes = kATile + BN * BK16 * 2;  // 16 KB + 32 KB
 constexpr size_t kSmemBf16 = 1024 + size_t(kStages) * kStageBytes + sizeof(Bars);
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -529,47 +617,11 @@ done:
 }
 
 // -------------------------------------------------------------- host ------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// Row-major [rows][inner] (inner contiguous, `ld` elements per row), box
-// [box_rows][box_inner], 128-byte swizzle.  Optional third dim (groups).
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
-              uint64_t rows, uint64_t ld, uint32_t box_inner, uint32_t box_rows,
-              uint64_t groups = 0) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {inner, rows, groups};
-  cuuint64_t strides[2] = {ld * esize, ld * esize * rows};
-  cuuint32_t box[3] = {box_inner, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  const cuuint32_t rank = groups ? 3 : 2;
-  return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename K>
-cudaError_t prepare(K kernel, size_t smem) {
-  static thread_local int done_dev = -1;
-  (void)done_dev;
+cudaError_t prepare(K kernel, size_t smem, bool check_regs) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (!check_regs) return cudaSuccess;
   cudaFuncAttributes attr;
   e = cudaFuncGetAttributes(&attr, kernel);
   if (e != cudaSuccess) return e;
@@ -579,6 +631,30 @@ cudaError_t prepare(K kernel, size_t smem) {
   return cudaSuccess;
 }
 
+template <int KIND, bool GROUPED, bool PAIR>
+cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                       const GemmArgs& a, int grid, cudaStream_t st) {
+  auto kern = k_gemm_fp8<KIND, GROUPED, PAIR>;
+  const size_t smem = smem_fp8<PAIR>();
+  cudaError_t e = prepare(kern, smem, true);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
+}
+
 }  // namespace
 
 int gemm_band_rows = 16;
@@ -586,45 +662,51 @@ int gemm_band_rows = 16;
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
                             const float* sB, void* D, int64_t ldd, int num_sms, cudaStream_t st) {
-  CUtensorMap ta, tb;
-  GemmArgs a;
+  // CTA pairs everywhere except grouped fprop/dgrad (128-row expert segments)
+  const bool pair = !(grouped && kind != FP8BW_WGRAD);
+  GemmArgs a = {};
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
-  a.m_tiles = (int)(M / BM);
+  a.m_tiles = (int)(pair ? (M + 2 * BM - 1) / (2 * BM) : M / BM);
   a.n_tiles = (int)((N + BN - 1) / BN);
-  a.band = gemm_band_rows;
+  a.band = pair ? (gemm_band_rows + 1) / 2 : gemm_band_rows;
   a.sA = sA;
   a.sB = sB;
-  a.D = static_cast<uint16_t*>(D);
-  a.ldd = ldd;
   a.offsets = d_off;
   a.G = G;
   if (grouped && kind == FP8BW_WGRAD) a.tiles = G * a.m_tiles * a.n_tiles;
   else a.tiles = a.m_tiles * a.n_tiles;
   if (a.tiles == 0) return cudaSuccess;
-  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, K, BK, BM)) return cudaErrorInvalidValue;
-  const bool b3 = grouped && kind != FP8BW_WGRAD;
-  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, BN, b3 ? (uint64_t)G : 0))
+  CUtensorMap ta, tb, td;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const int grid = a.tiles < num_sms ? a.tiles : num_sms;
-#define FP8BW_LAUNCH(KD, GR)                                                  \
-  do {                                                                        \
-    auto kern = k_gemm_fp8<KD, GR>;                                           \
-    cudaError_t e = prepare(kern, kSmemFp8);                                  \
-    if (e != cudaSuccess) return e;                                           \
-    kern<<<grid, kThreads, kSmemFp8, st>>>(ta, tb, a);                        \
-  } while (0)
-  if (!grouped) {
-    if (kind == FP8BW_FPROP) FP8BW_LAUNCH(FP8BW_FPROP, false);
-    else if (kind == FP8BW_DGRAD) FP8BW_LAUNCH(FP8BW_DGRAD, false);
-    else FP8BW_LAUNCH(FP8BW_WGRAD, false);
+  const bool b3 = grouped && kind != FP8BW_WGRAD;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, pair ? BN / 2 : BN,
+                CU_TENSOR_MAP_SWIZZLE_128B, b3 ? (uint64_t)G : 0))
+    return cudaErrorInvalidValue;
+  const uint64_t drows = (grouped && kind == FP8BW_WGRAD) ? (uint64_t)G * M : (uint64_t)M;
+  if (!make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, drows, ldd, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  int grid;
+  if (pair) {
+    const int clusters = num_sms / 2;
+    grid = 2 * (a.tiles < clusters ? a.tiles : clusters);
   } else {
-    if (kind == FP8BW_FPROP) FP8BW_LAUNCH(FP8BW_FPROP, true);
-    else if (kind == FP8BW_DGRAD) FP8BW_LAUNCH(FP8BW_DGRAD, true);
-    else FP8BW_LAUNCH(FP8BW_WGRAD, true);
+    grid = a.tiles < num_sms ? a.tiles : num_sms;
   }
-#undef FP8BW_LAUNCH
+  cudaError_t e;
+  if (!grouped) {
+    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true>(ta, tb, td, a, grid, st);
+    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true>(ta, tb, td, a, grid, st);
+    else e = launch_one<FP8BW_WGRAD, false, true>(ta, tb, td, a, grid, st);
+  } else {
+    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, true, false>(ta, tb, td, a, grid, st);
+    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, true, false>(ta, tb, td, a, grid, st);
+    else e = launch_one<FP8BW_WGRAD, true, true>(ta, tb, td, a, grid, st);
+  }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -645,8 +727,10 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, con
   a.offsets = nullptr;
   a.G = 0;
   if (a.tiles == 0) return cudaSuccess;
-  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, K, BK16, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, K, BK16, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, K, BK16, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, K, BK16, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   const int grid = a.tiles < num_sms ? a.tiles : num_sms;
   cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBf16);
