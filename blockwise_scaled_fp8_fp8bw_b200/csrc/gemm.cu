@@ -51,13 +51,15 @@ constexpr int kScaleStages = 8;
 constexpr uint32_t kATile = BM * BK;  // 16 KB: one CTA's A rows
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = FP8BW_MAX_EXPERTS;
-constexpr uint32_t kEpiBytes = 2048;  // per promotion warp: 32 rows x 32 bf16
+constexpr uint32_t kEpiPiece = 2048;  // 32 rows x 32 bf16: one TMA store
 
 template <bool PAIR>
 struct Cfg {
   static constexpr uint32_t kBTile = PAIR ? (BN / 2) * BK : BN * BK;  // this CTA's B rows
   static constexpr uint32_t kStageBytes = kATile + kBTile;
-  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kStages = PAIR ? 5 : 4;
+  static constexpr int kEpiBufs = PAIR ? 2 : 1;  // staging pieces per promotion warp
+  static constexpr uint32_t kEpiBytes = kEpiBufs * kEpiPiece;
   static constexpr uint32_t kIdesc = idesc_make(0, 0, PAIR ? 2 * BM : BM, BN);  // E4M3 -> F32
   static constexpr uint32_t kTemptyCount = PAIR ? 16 : 8;
 };
@@ -96,7 +98,7 @@ struct GemmArgs {
 template <bool PAIR>
 constexpr size_t smem_fp8() {
   return 1024 + size_t(Cfg<PAIR>::kStages) * Cfg<PAIR>::kStageBytes +
-         size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * kEpiBytes + sizeof(Bars) +
+         size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * Cfg<PAIR>::kEpiBytes + sizeof(Bars) +
          sizeof(int32_t) * (kMaxGroups + 1);
 }
 static_assert(smem_fp8<true>() <= 232448 && smem_fp8<false>() <= 232448, "shared memory budget");
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + C::kStages * C::kStageBytes;  // 1024-aligned
-  ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kEpiBytes);
+  ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(epi_base + 8 * C::kEpiBytes);
   Bars* bars = reinterpret_cast<Bars*>(slots + kScaleStages);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
 
@@ -276,11 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ------------------------------------------------- MMA issuer -----
-      if (leader) {
-        int stage = 0;
-        uint32_t phase = 0;
-        int buf = 0;
-        uint32_t bphase = 0;
+      if (leader && lane == 0) {
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, bphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
           const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
           if (ti.skip) continue;
@@ -291,24 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               goto done;
             }
             tc_fence_after();
-            if (lane == 0) {
-              const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
-              const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
-              const uint32_t d = tmem + buf * BN;
+            const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+            const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+            const uint32_t d = tmem + buf * BN;
 #pragma unroll
-              for (int kk = 0; kk < BK / 32; ++kk) {  // +32 bytes = +2 in the >>4 address field
-                if (PAIR) umma_f8f6f4_pair(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
-                else umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
-              }
-              if (PAIR) {
-                umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
-                umma_commit_pair(smem_u32(&bars->tfull[buf]), 0x3);
-              } else {
-                umma_commit(smem_u32(&bars->empty[stage]));
-                umma_commit(smem_u32(&bars->tfull[buf]));
-              }
+            for (int kk = 0; kk < BK / 32; ++kk) {  // +32 bytes = +2 in the >>4 address field
+              if (PAIR) umma_f8f6f4_pair(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
+              else umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
             }
-            __syncwarp();
+            if (PAIR) {
+              umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
+              umma_commit_pair(smem_u32(&bars->tfull[buf]), 0x3);
+            } else {
+              umma_commit(smem_u32(&bars->empty[stage]));
+              umma_commit(smem_u32(&bars->tfull[buf]));
+            }
             if (++stage == C::kStages) { stage = 0; phase ^= 1; }
             if (++buf == 2) { buf = 0; bphase ^= 1; }
           }
@@ -361,8 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------- promotion --
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int half = (warp - 4) >> 2;  // column half of the 256-wide tile
-    uint8_t* epi = epi_base + (warp - 4) * kEpiBytes;
-    const uint32_t epi_s = smem_u32(epi);
+    uint8_t* epi0 = epi_base + (warp - 4) * C::kEpiBytes;
     int ss = 0;
     uint32_t sphase = 0;
     int buf = 0;
@@ -390,8 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           uint32_t r[2][32];
-          tmem_ld32(taddr + h2 * 64, r[0]);
-          tmem_ld32(taddr + h2 * 64 + 32, r[1]);
+          tmem_ld64(taddr + h2 * 64, r[0], r[1]);
           tmem_wait_ld();
           if (h2 == 1) {
             // chunk fully read: hand the TMEM buffer back to the MMA warp
@@ -407,12 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int p = h2 * 2 + p2;
             if (KIND == FP8BW_WGRAD) {
               const float2 sa2 = make_float2(sa, sa);
-              const float2* sb2 = reinterpret_cast<const float2*>(&sl->sb[half * 128 + p * 32]);
+              const float4* sb4 = reinterpret_cast<const float4*>(&sl->sb[half * 128 + p * 32]);
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float2 sc = fmul2(sa2, sb2[j]);
-                acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1])),
-                                        sc, acc[p * 16 + j]);
+              for (int j = 0; j < 8; ++j) {
+                const float4 b4 = sb4[j];  // one broadcast load serves four columns
+                const float2 sc0 = fmul2(sa2, make_float2(b4.x, b4.y));
+                const float2 sc1 = fmul2(sa2, make_float2(b4.z, b4.w));
+                acc[p * 16 + 2 * j] = ffma2(make_float2(__uint_as_float(r[p2][4 * j]), __uint_as_float(r[p2][4 * j + 1])),
+                                            sc0, acc[p * 16 + 2 * j]);
+                acc[p * 16 + 2 * j + 1] = ffma2(make_float2(__uint_as_float(r[p2][4 * j + 2]), __uint_as_float(r[p2][4 * j + 3])),
+                                                sc1, acc[p * 16 + 2 * j + 1]);
               }
             } else {
               const float s = sa * sl->sb[half];
@@ -435,7 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (a pair's second CTA past the last row of M computed nothing real)
 #pragma unroll
       for (int p = 0; p < 4 && row0 < a.M; ++p) {
-        if (lane == 0) bulk_wait_read0();   // the previous piece has left the buffer
+        uint8_t* epi = epi0 + (p % C::kEpiBufs) * kEpiPiece;
+        // the store that last used this staging piece has read it
+        if (lane == 0) {
+          if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
+        }
         __syncwarp();
         // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
 #pragma unroll
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmD, epi_s, col0 + p * 32, drow);
+          tma_store_2d(&tmD, smem_u32(epi), col0 + p * 32, drow);
           bulk_commit();
         }
       }
