@@ -1,0 +1,153 @@
+"""GPU parity of the grouped (mixture-of-experts) blockwise FP8 GEMM against
+the oracle.  Method: "NVIDIA NeMo RL erreicht 48% ..." section
+"Leistungsgewinne in der Praxis" (the recipe trains the Qwen3-30B MoE model
+with the same FP8 linear layers).  Tokens are grouped by expert, each
+segment zero-padded to a multiple of 128 rows."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from util import bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def moe_case(orc, seed, lens, K, N, mode):
+    """Permuted tokens (zero-padded segments), expert weights and dY, all
+    quantized by the oracle.  Returns every operand the three GEMMs need."""
+    g = torch.Generator().manual_seed(seed)
+    pad = [((l + 127) // 128) * 128 for l in lens]
+    off = np.concatenate([[0], np.cumsum(pad)]).astype(np.int32)
+    Mtot = int(off[-1]) + 128          # a tail of rows beyond the last expert
+    G = len(lens)
+    X = torch.zeros((Mtot, K), dtype=torch.float32)
+    dY = torch.zeros((Mtot, N), dtype=torch.float32)
+    for e, l in enumerate(lens):
+        X[off[e]:off[e] + l] = torch.randn((l, K), generator=g)
+        dY[off[e]:off[e] + l] = torch.randn((l, N), generator=g) * 1e-3
+    X, dY = X.to(torch.bfloat16), dY.to(torch.bfloat16)
+    W = (torch.randn((G, N, K), generator=g) * 0.02).to(torch.bfloat16)
+    qx, sx, qxc, sxc = orc.quant_act_1x128(bits(X), mode)
+    qd, sd, qdc, sdc = orc.quant_act_1x128(bits(dY), mode)
+    qw = np.empty((G, N, K), np.uint8)
+    qwT = np.empty((G, K, N), np.uint8)
+    sw = np.empty((G, N // 128, K // 128), np.float32)
+    for e in range(G):
+        qw[e], sw[e], qwT[e] = orc.quant_weight_128x128(bits(W[e]), mode)
+    return dict(off=off, Mtot=Mtot, G=G, qx=qx, sx=sx, qxc=qxc, sxc=sxc, qd=qd, sd=sd, qdc=qdc,
+                sdc=sdc, qw=qw, sw=sw, qwT=qwT)
+
+
+def run_grouped(fb, kind, c, mode, D_shape):
+    off = dev(c["off"])
+    if kind == 0:
+        A, sA, B, sB = c["qx"], c["sx"], c["qw"], c["sw"]
+    elif kind == 1:
+        A, sA, B, sB = c["qd"], c["sd"], c["qwT"], c["sw"]
+    else:
+        A, sA, B, sB = c["qdc"], c["sdc"], c["qxc"], c["sxc"]
+    D = torch.full(D_shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_grouped_gemm(kind, off, dev(A), dev(sA), dev(B), dev(sB), D, mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    return D, (A, sA, B, sB)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_grouped_small(fb, orc, mode):
+    lens = [300, 0, 128, 1, 517, 0, 256, 77]          # empty experts and ragged segments
+    K, N = 256, 384
+    c = moe_case(orc, 11 + mode, lens, K, N, mode)
+    off, Mtot, G = c["off"], c["Mtot"], c["G"]
+    # fprop: Y = X W_g^T per segment;  dgrad: dX = dY W_g
+    for kind, Nout, Kin in [(0, N, K), (1, K, N)]:
+        D, ops = run_grouped(fb, kind, c, mode, (Mtot, Nout))
+        y, ya = orc.grouped_gemm_ref_tile(kind, off, *ops, 0, 0, int(off[-1]), 0, Nout)
+        bad, worst = orc.check_tol(bits(D)[:int(off[-1])], y, ya)
+        assert bad == 0, (kind, worst)
+        # rows past the last expert are not part of the result: untouched
+        assert torch.isnan(D[int(off[-1]):].float()).all()
+    # wgrad: dW_g = dY_g^T X_g over the expert's own tokens; empty experts -> 0
+    D, ops = run_grouped(fb, 2, c, mode, (G, N, K))
+    for e in range(G):
+        y, ya = orc.grouped_gemm_ref_tile(2, off, *ops, e, 0, N, 0, K)
+        bad, worst = orc.check_tol(bits(D[e]), y, ya)
+        assert bad == 0, (e, worst)
+        if lens[e] == 0:
+            assert torch.all(D[e] == 0)
+
+
+def test_grouped_bad_offsets(fb, orc):
+    """Offsets that are not multiples of 128 are rejected on the device: the
+    kernel writes nothing and latches FP8BW_ERR_DEVICE_CHECK."""
+    lens = [128, 256]
+    c = moe_case(orc, 3, lens, 128, 128, 0)
+    bad = np.array([0, 100, 384], np.int32)
+    D = torch.full((c["Mtot"], 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_grouped_gemm(0, dev(bad), dev(c["qx"]), dev(c["sx"]), dev(c["qw"]), dev(c["sw"]), D, 0)
+    assert fb.fp8bw_last_device_error() == 6
+    assert torch.all(D == 7.0)
+    assert fb.fp8bw_last_device_error() == 0   # the error word was cleared
+
+
+def test_grouped_moe_full_size_sampled(fb, orc):
+    """Qwen3-30B-A3B-like expert layer (hidden 2048 -> 1536, 128 experts,
+    top-8 of 16384 tokens, Zipf(1.1) popularity) at full size, in the launch
+    configuration the benchmark uses; one 128x128 output tile per expert is
+    checked against the oracle (smallest and largest experts included)."""
+    r = workloads.moe_routing(0)
+    G, K, N = workloads.MOE_EXPERTS, workloads.MOE_HIDDEN, 2 * workloads.MOE_INTER
+    X = workloads.moe_permuted(r, K, 1.0, seed=5, device=DEV)
+    W = workloads.moe_experts(G, N, K, seed=6, device=DEV)
+    Mtot = r.m_total_pad
+    qx = torch.empty((Mtot, K), dtype=torch.uint8, device=DEV)
+    sx = torch.empty((K // 128, Mtot), dtype=torch.float32, device=DEV)
+    fb.fp8bw_quant_act_1x128(X, 0, qx, sx)
+    qw = torch.empty((G, N, K), dtype=torch.uint8, device=DEV)
+    sw = torch.empty((G, N // 128, K // 128), dtype=torch.float32, device=DEV)
+    fb.fp8bw_requant_weights([(W[e], qw[e], sw[e], None) for e in range(G)], 0)
+    off = torch.tensor(r.offsets, dtype=torch.int32, device=DEV)
+    D = torch.empty((Mtot, N), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_grouped_gemm(0, off, qx, sx, qw, sw, D, 0)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    qx_h, sx_h, qw_h, sw_h = qx.cpu().numpy(), sx.cpu().numpy(), qw.cpu().numpy(), sw.cpu().numpy()
+    Dh = bits(D)
+    rng = np.random.default_rng(0)
+    counts = np.array(r.counts)
+    offs = np.array(r.offsets, np.int32)
+    for e in range(G):
+        if counts[e] == 0:
+            continue
+        nblk = (offs[e + 1] - offs[e]) // 128
+        rb = int(offs[e]) + 128 * int(rng.integers(0, nblk)) + 32 * int(rng.integers(0, 4))
+        cb = 32 * int(rng.integers(0, N // 32))
+        y, ya = orc.grouped_gemm_ref_tile(0, offs, qx_h, sx_h, qw_h, sw_h, 0, rb, rb + 32, cb, cb + 32)
+        bad, worst = orc.check_tol(np.ascontiguousarray(Dh[rb:rb + 32, cb:cb + 32]), y, ya)
+        assert bad == 0, (e, worst)
+    # wgrad for the largest and smallest experts: dW_g = dY_g^T X_g
+    dY = workloads.moe_permuted(r, N, 1e-3, seed=7, device=DEV)
+    qxc = torch.empty((K, Mtot), dtype=torch.uint8, device=DEV)
+    sxc = torch.empty((Mtot // 128, K), dtype=torch.float32, device=DEV)
+    qd = torch.empty((Mtot, N), dtype=torch.uint8, device=DEV)
+    sd = torch.empty((N // 128, Mtot), dtype=torch.float32, device=DEV)
+    qdc = torch.empty((N, Mtot), dtype=torch.uint8, device=DEV)
+    sdc = torch.empty((Mtot // 128, N), dtype=torch.float32, device=DEV)
+    fb.fp8bw_quant_act_1x128(X, 0, qx, sx, qxc, sxc)
+    fb.fp8bw_quant_act_1x128(dY, 0, qd, sd, qdc, sdc)
+    dW = torch.empty((G, N, K), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_grouped_gemm(2, off, qdc, sdc, qxc, sxc, dW, 0)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    A, sA, B, sB = qdc.cpu().numpy(), sdc.cpu().numpy(), qxc.cpu().numpy(), sxc.cpu().numpy()
+    for e in [int(np.argmax(counts)), int(np.argmin(counts))]:
+        nb, kb = 32 * int(rng.integers(0, N // 32)), 32 * int(rng.integers(0, K // 32))
+        y, ya = orc.grouped_gemm_ref_tile(2, offs, A, sA, B, sB, e, nb, nb + 32, kb, kb + 32)
+        bad, worst = orc.check_tol(np.ascontiguousarray(bits(dW[e])[nb:nb + 32, kb:kb + 32]), y, ya)
+        assert bad == 0, (e, worst)

@@ -195,8 +195,10 @@ def packed_rows_mask(seed: int = 0, total: int = PACKED_TOKENS):
 
 
 def packed_activations(K: int, seed: int = 0, device="cpu", total: int = PACKED_TOKENS,
-                       scale: float = 1.0):
-    mask = packed_rows_mask(seed, total).to(device)
+                       scale: float = 1.0, mask_seed: int = 0):
+    """[total, K] Student-t (nu=3) values times `scale`, zero on the padding
+    rows of the packing drawn with `mask_seed` (shared by X and dY)."""
+    mask = packed_rows_mask(mask_seed, total).to(device)
     x = student_t_bf16((total, K), 3, scale, seed * 97 + K, device)
     x[~mask] = 0
     return x
