@@ -64,6 +64,22 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_burst": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
 
 
+def gemm_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None if
+    the kernel source changed since those counters were taken."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "k_gemm_fp8_llama8b_step.md")
+    src = os.path.join(ROOT, "blockwise_scaled_fp8_fp8bw_b200", "csrc", "gemm.cu")
+    try:
+        text = open(prof).read()
+        want = [l.split(":", 1)[1].strip() for l in text.splitlines() if l.startswith("gemm_cu_sha256_16:")][0]
+        val = [l.split(":", 1)[1].strip() for l in text.splitlines() if l.startswith("traffic_bytes_per_launch:")][0]
+        have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return int(val) if have == want else None
+    except (OSError, IndexError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------ clocks ------
 class ClockSampler:
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -459,7 +475,7 @@ def main():
                        "scale_mode": args.mode, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (per-step working set > 1.5 GB)"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": gemm_tflops / fp8_peak, "traffic": None,
+                         "frac": gemm_tflops / fp8_peak, "traffic": gemm_traffic(),
                          "kernel": "k_gemm_fp8 (all fprop/dgrad/wgrad launches)",
                          "peak_note": f"FP8 = 2 x {pk['src']} cuBLAS bf16 "
                                       f"({'sustained' if timed_long else 'burst'})",

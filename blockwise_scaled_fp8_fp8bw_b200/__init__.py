@@ -8,6 +8,8 @@ torch stream and raises ``Fp8bwError`` on a non-OK status.  There is no CPU
 fallback: if the library is missing this module fails to import.
 
 ``raw`` is the ctypes handle with the C prototypes, for pointer-level calls.
+The library is loaded on first use (``load()``), so that building it does not
+require an already-built copy.
 """
 from __future__ import annotations
 
@@ -48,24 +50,43 @@ def _load():
     L.fp8bw_status_string.argtypes = [i32]
     L.fp8bw_status_string.restype = ctypes.c_char_p
     L.fp8bw_last_device_error.argtypes = [vp]
+    L.fp8bw_testing_stall_next_gemm.argtypes = [ctypes.c_int32]
     L.fp8bw_quant_act_1x128.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp]
     L.fp8bw_quant_weight_128x128.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp]
     L.fp8bw_requant_weights.argtypes = [ctypes.POINTER(fp8bw_weight_desc), ctypes.c_int32, i32, vp]
     L.fp8bw_gemm.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, vp, i64, i32, vp]
     L.fp8bw_grouped_gemm.argtypes = [i32, ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
-    for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_quant_act_1x128",
+    for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm",
+              "fp8bw_quant_act_1x128",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
               "fp8bw_grouped_gemm", "fp8bw_gemm_bf16"):
         getattr(L, f).restype = i32
     return L
 
 
-raw = _load()
+_raw = None
+
+
+def load():
+    """Loads libfp8bw.so (raises ImportError if it is missing or stale)."""
+    global _raw
+    if _raw is None:
+        try:
+            _raw = _load()
+        except AttributeError as e:  # a symbol of the header is missing: stale build
+            raise ImportError(f"{LIB_PATH} is stale ({e}); rebuild it") from e
+    return _raw
+
+
+def __getattr__(name):
+    if name == "raw":
+        return load()
+    raise AttributeError(name)
 
 
 def status_string(status: int) -> str:
-    return raw.fp8bw_status_string(int(status)).decode()
+    return load().fp8bw_status_string(int(status)).decode()
 
 
 def _check(fn: str, status: int) -> None:
@@ -86,12 +107,17 @@ def _stream(stream):
 
 # --------------------------------------------------------------- calls ----
 def fp8bw_init(device: int = 0) -> None:
-    _check("fp8bw_init", raw.fp8bw_init(int(device)))
+    _check("fp8bw_init", load().fp8bw_init(int(device)))
 
 
 def fp8bw_last_device_error(stream=None) -> int:
     """Status of the device error word (synchronizes the stream, clears it)."""
-    return raw.fp8bw_last_device_error(_stream(stream))
+    return load().fp8bw_last_device_error(_stream(stream))
+
+
+def fp8bw_testing_stall_next_gemm(chunk: int) -> None:
+    """Testing hook: the next GEMM launch stalls at `chunk` and times out."""
+    _check("fp8bw_testing_stall_next_gemm", load().fp8bw_testing_stall_next_gemm(int(chunk)))
 
 
 def fp8bw_quant_act_1x128(x, mode, q_row, s_row, q_col=None, s_col=None, stream=None, K=None):
@@ -99,7 +125,7 @@ def fp8bw_quant_act_1x128(x, mode, q_row, s_row, q_col=None, s_col=None, stream=
     q_col [K,M] u8 / s_col [M/128,K] f32 or both None."""
     M, ldx = x.shape[0], x.stride(0)
     K = x.shape[1] if K is None else K
-    _check("fp8bw_quant_act_1x128", raw.fp8bw_quant_act_1x128(
+    _check("fp8bw_quant_act_1x128", load().fp8bw_quant_act_1x128(
         _ptr(x), M, K, ldx, int(mode), _ptr(q_row), _ptr(s_row), _ptr(q_col), _ptr(s_col),
         _stream(stream)))
 
@@ -107,7 +133,7 @@ def fp8bw_quant_act_1x128(x, mode, q_row, s_row, q_col=None, s_col=None, stream=
 def fp8bw_quant_weight_128x128(w, mode, q, s, qT=None, stream=None):
     """w [N, ldw] bf16; q [N,K] u8; s [N/128,K/128] f32; qT [K,N] u8 or None."""
     N, K = w.shape
-    _check("fp8bw_quant_weight_128x128", raw.fp8bw_quant_weight_128x128(
+    _check("fp8bw_quant_weight_128x128", load().fp8bw_quant_weight_128x128(
         _ptr(w), N, K, w.stride(0), int(mode), _ptr(q), _ptr(s), _ptr(qT), _stream(stream)))
 
 
@@ -118,14 +144,14 @@ def fp8bw_requant_weights(items, mode, stream=None):
     for i, (w, q, s, qT) in enumerate(items):
         arr[i] = fp8bw_weight_desc(w.data_ptr(), w.shape[0], w.shape[1], w.stride(0), q.data_ptr(),
                                    s.data_ptr(), qT.data_ptr() if qT is not None else None)
-    _check("fp8bw_requant_weights", raw.fp8bw_requant_weights(arr, n, int(mode), _stream(stream)))
+    _check("fp8bw_requant_weights", load().fp8bw_requant_weights(arr, n, int(mode), _stream(stream)))
 
 
 def fp8bw_gemm(kind, A, sA, B, sB, D, mode=FP8BW_SCALE_FP32, stream=None):
     """A [M,K] u8, sA [K/128,M]; B [N,K] u8, sB per kind; D [M, ldd>=N] bf16."""
     M, K = A.shape
     N = B.shape[0]
-    _check("fp8bw_gemm", raw.fp8bw_gemm(int(kind), M, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
+    _check("fp8bw_gemm", load().fp8bw_gemm(int(kind), M, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
                                         _ptr(D), D.stride(0), int(mode), _stream(stream)))
 
 
@@ -139,7 +165,7 @@ def fp8bw_grouped_gemm(kind, offsets, A, sA, B, sB, D, mode=FP8BW_SCALE_FP32, st
     else:
         Mtot, K = A.shape
         N = B.shape[1]
-    _check("fp8bw_grouped_gemm", raw.fp8bw_grouped_gemm(
+    _check("fp8bw_grouped_gemm", load().fp8bw_grouped_gemm(
         int(kind), G, _ptr(offsets), Mtot, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(D),
         int(mode), _stream(stream)))
 
@@ -148,5 +174,5 @@ def fp8bw_gemm_bf16(A, B, D, stream=None):
     """A [M,K] bf16, B [N,K] bf16, D [M, ldd>=N] bf16."""
     M, K = A.shape
     N = B.shape[0]
-    _check("fp8bw_gemm_bf16", raw.fp8bw_gemm_bf16(M, N, K, _ptr(A), _ptr(B), _ptr(D), D.stride(0),
+    _check("fp8bw_gemm_bf16", load().fp8bw_gemm_bf16(M, N, K, _ptr(A), _ptr(B), _ptr(D), D.stride(0),
                                                   _stream(stream)))

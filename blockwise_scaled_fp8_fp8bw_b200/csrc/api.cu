@@ -21,6 +21,7 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
+extern int gemm_stall_chunk;
 }  // namespace fp8bw
 
 namespace {
@@ -88,6 +89,12 @@ FP8BW_API const char* fp8bw_status_string(fp8bw_status s) {
     case FP8BW_ERR_TOO_LARGE: return "size exceeds the supported maximum";
   }
   return "unknown status";
+}
+
+FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk) {
+  if (chunk < -1) return FP8BW_ERR_INVALID_ARG;
+  fp8bw::gemm_stall_chunk = chunk;
+  return FP8BW_OK;
 }
 
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {

@@ -93,6 +93,7 @@ struct GemmArgs {
   int G;
   uint16_t* D;         // BF16 kernel only (the FP8 kernel stores through a tensor map)
   int64_t ldd;
+  int stall_chunk;     // testing: CTA 0's producer never fills this chunk (-1: off)
 };
 
 template <bool PAIR>
@@ -243,19 +244,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
       }
-      int stage = 0;
+      int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
         const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
         if (ti.skip) continue;
         const int arow = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++chunk) {
           if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
             raise_timeout(bars);
             goto done;
           }
-          if (lane == 0) {
+          if (lane == 0 && !(blockIdx.x == 0 && chunk == a.stall_chunk)) {
             const uint32_t full = full0 + stage * 8;
             const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
             if (PAIR) {
@@ -661,6 +662,7 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
 }  // namespace
 
 int gemm_band_rows = 16;
+int gemm_stall_chunk = -1;  // testing hook, consumed by the next FP8 GEMM launch
 
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
@@ -678,6 +680,8 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   a.sB = sB;
   a.offsets = d_off;
   a.G = G;
+  a.stall_chunk = gemm_stall_chunk;
+  gemm_stall_chunk = -1;
   if (grouped && kind == FP8BW_WGRAD) a.tiles = G * a.m_tiles * a.n_tiles;
   else a.tiles = a.m_tiles * a.n_tiles;
   if (a.tiles == 0) return cudaSuccess;

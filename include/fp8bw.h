@@ -79,6 +79,15 @@ FP8BW_API const char* fp8bw_status_string(fp8bw_status s);
  * (e.g. grouped offsets), else FP8BW_OK.  FP8BW_ERR_CUDA if the sync failed. */
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream);
 
+/* Testing hook for the failure path (not part of the method): the next
+ * fp8bw_gemm / fp8bw_grouped_gemm launch on this host thread's process has
+ * its first CTA's operand producer skip K-chunk number `chunk` (counted over
+ * that CTA's tiles), so the kernel's bounded waits run out: it abandons its
+ * loops within a few seconds, writes an incomplete result and latches
+ * FP8BW_ERR_TIMEOUT for fp8bw_last_device_error(); the context stays usable.
+ * chunk = -1 cancels a pending stall.  FP8BW_ERR_INVALID_ARG if chunk < -1. */
+FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk);
+
 /* Activation quantization with 1x128 blocks ("Der technische Durchbruch":
  * 1x128 granularity for activations), plus the column-wise copy the weight
  * gradient needs.

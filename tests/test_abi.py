@@ -78,3 +78,6 @@ def test_host_validation(lib):
     d[1] = lib.fp8bw_weight_desc(0x10000, 128, 136, 136, 0x10000, 0x10000, None)
     assert r.fp8bw_requant_weights(d, 2, 0, N) == 2
     assert r.fp8bw_requant_weights(None, 1, 0, N) == 1
+    # testing hook: only chunk >= -1 is accepted; -1 cancels
+    assert r.fp8bw_testing_stall_next_gemm(-2) == 1
+    assert r.fp8bw_testing_stall_next_gemm(-1) == 0

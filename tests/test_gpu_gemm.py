@@ -140,3 +140,18 @@ def test_bf16_gemm(fb, orc, MNK):
     yr, ya = orc.gemm_bf16_ref_tile(bits(A), bits(B), 0, M, 0, N)
     bad, worst = orc.check_tol(bits(D), yr, ya, rel=1e-3)
     assert bad == 0, worst
+
+
+def test_bounded_wait_timeout_is_reported(fb, orc):
+    """Failure path: a producer that never fills one K-chunk makes the GEMM's
+    bounded waits run out; the call comes back with FP8BW_ERR_TIMEOUT and
+    the context stays usable for the next (correct) GEMM."""
+    rng = np.random.default_rng(12)
+    A, sA, B, sB = rand_ops(rng, 256, 256, 512, 0)
+    D = torch.zeros((256, 256), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_testing_stall_next_gemm(1)
+    fb.fp8bw_gemm(0, dev(A), dev(sA), dev(B), dev(sB), D)
+    assert fb.fp8bw_last_device_error() == 5          # FP8BW_ERR_TIMEOUT
+    assert fb.fp8bw_last_device_error() == 0          # cleared
+    y = gpu_gemm(fb, 0, A, sA, B, sB)
+    check(orc, y, 0, A, sA, B, sB)
