@@ -16,8 +16,8 @@ cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw
 cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cudaStream_t st);
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M,
                             int64_t N, int64_t K, const uint8_t* A, const float* sA,
-                            const uint8_t* B, const float* sB, void* D, int64_t ldd, int num_sms,
-                            cudaStream_t st);
+                            const uint8_t* B, const float* sB, void* D, int64_t ldd, int mode,
+                            int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
@@ -176,7 +176,7 @@ FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, in
   if (M == 0 || N == 0) return FP8BW_OK;
   if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
   return from_cuda(fp8bw::launch_gemm_fp8(kind, false, 0, nullptr, M, N, K, A, sA, B, sB, D, ldd,
-                                          sms, reinterpret_cast<cudaStream_t>(stream)));
+                                          mode, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
@@ -202,12 +202,12 @@ FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const
     // GEMM sizes: rows = N (out), cols = K (in), contraction = tokens.
     if (N == 0 || K == 0) return FP8BW_OK;
     return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, N, K, M_total_pad, A, sA, B,
-                                            sB, D, K, sms, cs));
+                                            sB, D, K, mode, sms, cs));
   }
   if (M_total_pad == 0 || N == 0) return FP8BW_OK;
   if (K == 0) return FP8BW_ERR_INVALID_ARG;
   return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, M_total_pad, N, K, A, sA, B,
-                                          sB, D, N, sms, cs));
+                                          sB, D, N, mode, sms, cs));
 }
 
 FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,

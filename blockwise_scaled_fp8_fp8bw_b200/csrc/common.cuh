@@ -202,6 +202,36 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// Block-scaled MMA (kind::mxf8f6f4, one UE8M0 scale per row and per 32-K
+// block of A and B, read from TMEM at sfa / sfb): D (+)= (A*sA)(B*sB).
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared memory -> TMEM: 32 rows x 128 bits, written to all four 32-lane
+// quarters of TMEM (lanes i, 32+i, 64+i, 96+i get row i), 4 columns.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a plain (unswizzled) K-major tile of 16-byte
+// rows: 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_k_noswz_16B(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128u >> 4) << 16;  // leading byte offset (single 16-byte column)
+  d |= (uint64_t)(128u >> 4) << 32;  // stride byte offset: next 8-row core matrix
+  d |= (uint64_t)1 << 46;
+  return d;                          // layout type 0: no swizzle
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
@@ -369,6 +399,13 @@ __device__ __forceinline__ void bulk_wait_read1() {
 }
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: B scale-factor id [4,6),
+// A/B formats (E4M3 = 0) at [7,10)/[10,13), N>>3 at [17,23), scale format
+// [23] (1 = UE8M0), M>>4 at [24,29), A scale-factor id [29,31).
+__host__ __device__ constexpr uint32_t idesc_mx(uint32_t M, uint32_t N, uint32_t sf_id) {
+  return (sf_id << 4) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) | (sf_id << 29);
 }
 
 // ----------------------------------------------------------- setmaxnreg ---

@@ -156,6 +156,12 @@ __device__ __forceinline__ void raise_timeout(Bars* bars) {
   atomicExch(&bars->abort, 1);
 }
 
+template <typename B>
+__device__ __forceinline__ void raise_timeout_mx(B* bars) {
+  atomicOr(&g_gemm_error, DEV_ERR_TIMEOUT);
+  atomicExch(&bars->abort, 1);
+}
+
 template <int KIND, bool GROUPED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -472,6 +478,338 @@ done:
   }
 }
 
+// ----------------------------------------------- block-scaled (MX) GEMM ---
+// Power-of-2 scales (FP8BW_SCALE_POW2, "Warum dies für die KI-Ökonomie
+// wichtig ist": power-of-2 scale factors as an optimization) are exactly
+// UE8M0 values, so the tensor core applies them itself
+// (tcgen05.mma.kind::mxf8f6f4.block_scale): each 128-wide scale block is one
+// UE8M0 byte replicated over its four 32-element MMA blocks, and the whole K
+// loop accumulates in one TMEM accumulator with no promotion.
+// One CTA per SM, 128x256 tiles, 384 threads:
+//   warp 0      TMA producer (4-stage ring of 48 KB stages)
+//   warp 1      MMA issuer: per chunk, tcgen05.cp of the chunk's scale
+//               bytes (A: 128 rows, B: 256 rows) from shared memory into a
+//               per-stage TMEM slot, then four block-scaled MMAs
+//   warp 2      scale loader: fp32 scales by cp.async into a raw ring, then
+//               converted to UE8M0 bytes in the tcgen05.cp layout (row r of a
+//               128-row group at lane r%32, word r/32; the four bytes of a
+//               word are the four 32-K blocks); a scale that is not a power
+//               of two latches FP8BW_ERR_DEVICE_CHECK
+//   warps 4-11  epilogue: drain the accumulator (tcgen05.ld), release it,
+//               round to bf16 and TMA-store (as in the promotion kernel)
+constexpr int kMxStages = 4;
+constexpr int kMxRaw = 4;                       // raw scale slots; lookahead kMxRaw-1
+constexpr uint32_t kMxStageBytes = kATile + BN * BK;  // 16 KB A + 32 KB B
+constexpr uint32_t kSfCol0 = 256;               // TMEM: accumulator [0,256), scales after
+constexpr uint32_t kSfCols = 12;                // per stage: A 4 columns + B 8 columns
+
+struct MxBars {
+  uint64_t full[kMxStages], empty[kMxStages], sffull[kMxStages];
+  uint64_t tfull, tempty;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct SfSlot {
+  uint32_t a[32][4];     // A rows: row i + 32b at [i][b]
+  uint32_t b[2][32][4];  // B rows 0..127 and 128..255
+};
+
+constexpr size_t kSmemMx = 1024 + size_t(kMxStages) * kMxStageBytes + 8 * kEpiPiece +
+                           size_t(kMxRaw) * sizeof(ScaleSlot) + size_t(kMxStages) * sizeof(SfSlot) +
+                           sizeof(MxBars) + sizeof(int32_t) * (kMaxGroups + 1);
+static_assert(kSmemMx <= 232448, "shared memory budget (MX)");
+
+// UE8M0 byte of a power-of-2 fp32 scale (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ uint32_t ue8m0_x4(float s, bool& bad) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t e = b >> 23;
+  if ((b & 0x7FFFFFu) != 0u && b != 0x00400000u) bad = true;
+  return (e & 0xFFu) * 0x01010101u;
+}
+
+template <int KIND, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint8_t* epi_base = smem + kMxStages * kMxStageBytes;
+  ScaleSlot* raw = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kEpiPiece);
+  SfSlot* sf = reinterpret_cast<SfSlot*>(raw + kMxRaw);
+  MxBars* bars = reinterpret_cast<MxBars*>(sf + kMxStages);
+  int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMxStages; ++i) {
+      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->empty[i]), 1);
+      mbar_init(smem_u32(&bars->sffull[i]), 1);
+    }
+    mbar_init(smem_u32(&bars->tfull), 1);
+    mbar_init(smem_u32(&bars->tempty), 8);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (GROUPED) {
+    for (int i = threadIdx.x; i <= a.G; i += kThreads) s_off[i] = a.offsets[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (GROUPED) {
+    int bad = 0;
+    for (int i = threadIdx.x; i < a.G; i += kThreads) {
+      const int o0 = s_off[i], o1 = s_off[i + 1];
+      if (o1 < o0 || (o1 & 127) || (i == 0 && o0 != 0)) bad = 1;
+    }
+    if (threadIdx.x == 0) {
+      const int mtot = (KIND == FP8BW_WGRAD) ? a.K : a.M;
+      if (s_off[a.G] > mtot || s_off[a.G] < 0) bad = 1;
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
+      tc_fence_before();
+      if (warp == 1) tmem_dealloc(bars->tmem_base, kTmemCols);
+      return;
+    }
+  }
+  const uint32_t tmem = bars->tmem_base;
+  const int cta_slot = blockIdx.x, cta_step = gridDim.x;
+
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ------------------------------------------------ TMA producer ----
+      if (lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+      }
+      int stage = 0, chunk = 0;
+      uint32_t phase = 0;
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
+        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        if (ti.skip) continue;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++chunk) {
+          if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
+            raise_timeout_mx(bars);
+            goto done;
+          }
+          if (lane == 0 && !(blockIdx.x == 0 && chunk == a.stall_chunk)) {
+            const uint32_t full = smem_u32(&bars->full[stage]);
+            const uint32_t sa = smem_u32(stage_base + stage * kMxStageBytes);
+            mbar_arrive_expect_tx(full, kMxStageBytes);
+            tma_load_2d(sa, &tmA, full, kb * BK, ti.mt * BM);
+            if (GROUPED && KIND != FP8BW_WGRAD)
+              tma_load_3d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN, ti.g);
+            else
+              tma_load_2d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN);
+          }
+          __syncwarp();
+          if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+        }
+        if (bars->abort) break;
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------- MMA issuer -----
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0, tphase = 0;
+        for (int t = cta_slot; t < a.tiles; t += cta_step) {
+          const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          if (ti.skip || ti.kb0 == ti.kb1) continue;
+          if (!mbar_wait(smem_u32(&bars->tempty), tphase ^ 1)) {
+            raise_timeout_mx(bars);
+            goto done;
+          }
+          tc_fence_after();
+          for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+            if (!mbar_wait(smem_u32(&bars->full[stage]), phase) ||
+                !mbar_wait(smem_u32(&bars->sffull[stage]), phase)) {
+              raise_timeout_mx(bars);
+              goto done;
+            }
+            tc_fence_after();
+            const uint32_t tsf = tmem + kSfCol0 + stage * kSfCols;
+            tmem_cp_32x128b_x4(tsf, sdesc_k_noswz_16B(smem_u32(&sf[stage].a[0][0])));
+            tmem_cp_32x128b_x4(tsf + 4, sdesc_k_noswz_16B(smem_u32(&sf[stage].b[0][0][0])));
+            tmem_cp_32x128b_x4(tsf + 8, sdesc_k_noswz_16B(smem_u32(&sf[stage].b[1][0][0])));
+            const uint32_t sa = smem_u32(stage_base + stage * kMxStageBytes);
+            const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              umma_mx(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(BM, BN, kk), tsf, tsf + 4,
+                      (kb > ti.kb0 || kk > 0) ? 1u : 0u);
+            umma_commit(smem_u32(&bars->empty[stage]));
+            if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+          }
+          umma_commit(smem_u32(&bars->tfull));
+          tphase ^= 1;
+          if (bars->abort) break;
+        }
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------ scale loader ----
+      // Chunk c's fp32 scales go to raw slot c % kMxRaw by cp.async; chunk
+      // c - (kMxRaw - 1) is converted once its copies have landed.
+      constexpr int L = kMxRaw - 1;
+      const int nKb = a.K / BK, nNb = a.N / 128;
+      int issued = 0, done_c = 0, sstage = 0;
+      uint32_t sphase = 0;
+      bool bad = false;
+      auto convert = [&](int d) -> bool {
+        __syncwarp();
+        if (!mbar_wait(smem_u32(&bars->empty[sstage]), sphase ^ 1)) return false;
+        const ScaleSlot* r = &raw[d % kMxRaw];
+        SfSlot* o = &sf[sstage];
+        uint4 wa;
+        wa.x = ue8m0_x4(r->sa[lane], bad);
+        wa.y = ue8m0_x4(r->sa[lane + 32], bad);
+        wa.z = ue8m0_x4(r->sa[lane + 64], bad);
+        wa.w = ue8m0_x4(r->sa[lane + 96], bad);
+        *reinterpret_cast<uint4*>(&o->a[lane][0]) = wa;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4 wb;
+          if (KIND == FP8BW_WGRAD) {
+            wb.x = ue8m0_x4(r->sb[h * 128 + lane], bad);
+            wb.y = ue8m0_x4(r->sb[h * 128 + lane + 32], bad);
+            wb.z = ue8m0_x4(r->sb[h * 128 + lane + 64], bad);
+            wb.w = ue8m0_x4(r->sb[h * 128 + lane + 96], bad);
+          } else {
+            wb.x = wb.y = wb.z = wb.w = ue8m0_x4(r->sb[h], bad);
+          }
+          *reinterpret_cast<uint4*>(&o->b[h][lane][0]) = wb;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->sffull[sstage]));
+        if (++sstage == kMxStages) { sstage = 0; sphase ^= 1; }
+        return true;
+      };
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
+        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        if (ti.skip) continue;
+        const float* sBg = a.sB;
+        if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          ScaleSlot* sl = &raw[issued % kMxRaw];
+          // unused entries hold 1.0 (byte 127) so no stale value is checked
+          cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + ti.mt * BM + lane * 4);
+          if (KIND == FP8BW_WGRAD) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int n = ti.nt * BN + h * 128 + lane * 4;
+              if (n < a.N) cp_async_16(smem_u32(&sl->sb[h * 128 + lane * 4]), sBg + (size_t)kb * a.N + n);
+              else *reinterpret_cast<float4*>(&sl->sb[h * 128 + lane * 4]) = make_float4(1.f, 1.f, 1.f, 1.f);
+            }
+          } else if (lane < 2) {
+            const int nb = ti.nt * 2 + lane;
+            if (nb < nNb) {
+              const float* src = (KIND == FP8BW_FPROP) ? sBg + (size_t)nb * nKb + kb
+                                                       : sBg + (size_t)kb * nNb + nb;
+              cp_async_4(smem_u32(&sl->sb[lane]), src);
+            } else {
+              sl->sb[lane] = 1.f;
+            }
+          }
+          asm volatile("cp.async.commit_group;" ::: "memory");
+          ++issued;
+          if (issued - done_c > L) {
+            asm volatile("cp.async.wait_group %0;" ::"n"(L) : "memory");
+            if (!convert(done_c)) { raise_timeout_mx(bars); goto done; }
+            ++done_c;
+          }
+        }
+        if (bars->abort) break;
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      while (done_c < issued) {
+        if (!convert(done_c)) { raise_timeout_mx(bars); goto done; }
+        ++done_c;
+      }
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
+    }
+  } else {
+    regs_inc<kRegsHigh>();
+    // -------------------------------------------------------- epilogue ---
+    const int q = warp & 3, half = (warp - 4) >> 2;
+    uint8_t* epi = epi_base + (warp - 4) * kEpiPiece;
+    uint32_t tphase = 0;
+    for (int t = cta_slot; t < a.tiles; t += cta_step) {
+      const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+      if (ti.skip) continue;
+      const int row0 = ti.mt * BM;
+      const int col0 = ti.nt * BN + half * 128;
+      float2 acc[64];
+      if (ti.kb0 == ti.kb1) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.f, 0.f);
+      } else {
+        if (!mbar_wait(smem_u32(&bars->tfull), tphase)) {
+          raise_timeout_mx(bars);
+          goto done;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + half * 128;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[2][32];
+          tmem_ld64(taddr + h2 * 64, r[0], r[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int p2 = 0; p2 < 2; ++p2)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[(h2 * 2 + p2) * 16 + j] =
+                  make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->tempty));
+        tphase ^= 1;
+      }
+      const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[p * 16 + 4 * c + 0].x, acc[p * 16 + 4 * c + 0].y);
+          o.y = pack_bf16x2(acc[p * 16 + 4 * c + 1].x, acc[p * 16 + 4 * c + 1].y);
+          o.z = pack_bf16x2(acc[p * 16 + 4 * c + 2].x, acc[p * 16 + 4 * c + 2].y);
+          o.w = pack_bf16x2(acc[p * 16 + 4 * c + 3].x, acc[p * 16 + 4 * c + 3].y);
+          *reinterpret_cast<uint4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, smem_u32(epi), col0 + p * 32, drow);
+          bulk_commit();
+        }
+      }
+      if (bars->abort) break;
+    }
+  }
+done:
+  if (warp >= 4 && lane == 0) bulk_wait0();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------ BF16 GEMM ---
 // Same pipeline without scales: BK = 64 bf16 (128-byte rows), four
 // kind::f16 MMAs (K = 16) per stage, the accumulator stays in TMEM for the
@@ -659,6 +997,16 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
 }
 
+template <int KIND, bool GROUPED>
+cudaError_t launch_mx(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                      const GemmArgs& a, int grid, cudaStream_t st) {
+  auto kern = k_gemm_mx<KIND, GROUPED>;
+  cudaError_t e = prepare(kern, kSmemMx, true);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemMx, st>>>(ta, tb, td, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int gemm_band_rows = 16;
@@ -666,7 +1014,8 @@ int gemm_stall_chunk = -1;  // testing hook, consumed by the next FP8 GEMM launc
 
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
-                            const float* sB, void* D, int64_t ldd, int num_sms, cudaStream_t st) {
+                            const float* sB, void* D, int64_t ldd, int mode, int num_sms,
+                            cudaStream_t st) {
   // CTA pairs everywhere except grouped fprop/dgrad (128-row expert segments)
   const bool pair = !(grouped && kind != FP8BW_WGRAD);
   GemmArgs a = {};
@@ -697,13 +1046,34 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
                 CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   int grid;
+  cudaError_t e;
+  if (mode == FP8BW_SCALE_POW2) {
+    // 1-CTA 128x256 tiles over the whole problem
+    a.m_tiles = (int)(M / BM);
+    a.band = gemm_band_rows;
+    a.tiles = (grouped && kind == FP8BW_WGRAD) ? G * a.m_tiles * a.n_tiles : a.m_tiles * a.n_tiles;
+    if (pair && !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, BN,
+                          CU_TENSOR_MAP_SWIZZLE_128B, 0))
+      return cudaErrorInvalidValue;
+    grid = a.tiles < num_sms ? a.tiles : num_sms;
+    if (!grouped) {
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false>(ta, tb, td, a, grid, st);
+      else e = launch_mx<FP8BW_WGRAD, false>(ta, tb, td, a, grid, st);
+    } else {
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, true>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, true>(ta, tb, td, a, grid, st);
+      else e = launch_mx<FP8BW_WGRAD, true>(ta, tb, td, a, grid, st);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (pair) {
     const int clusters = num_sms / 2;
     grid = 2 * (a.tiles < clusters ? a.tiles : clusters);
   } else {
     grid = a.tiles < num_sms ? a.tiles : num_sms;
   }
-  cudaError_t e;
   if (!grouped) {
     if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true>(ta, tb, td, a, grid, st);
     else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true>(ta, tb, td, a, grid, st);

@@ -155,3 +155,35 @@ def test_bounded_wait_timeout_is_reported(fb, orc):
     assert fb.fp8bw_last_device_error() == 0          # cleared
     y = gpu_gemm(fb, 0, A, sA, B, sB)
     check(orc, y, 0, A, sA, B, sB)
+
+
+def rand_ops_pow2(rng, M, N, K, kind):
+    A, _, B, _ = rand_ops(rng, M, N, K, kind)
+    nK = K // 128
+    sA = (2.0 ** rng.integers(-20, 6, (nK, M))).astype(np.float32)
+    shp = {0: (N // 128, nK), 1: (nK, N // 128), 2: (nK, N)}[kind]
+    sB = (2.0 ** rng.integers(-20, 6, shp)).astype(np.float32)
+    return A, sA, B, sB
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("MNK", [(128, 128, 128), (384, 640, 384), (256, 384, 1024)])
+def test_shapes_pow2(fb, orc, kind, MNK):
+    """Power-of-2 scales (the tensor core's block-scaled MMA applies them)."""
+    rng = np.random.default_rng(hash((kind, 7) + MNK) % 2**32)
+    ops = rand_ops_pow2(rng, *MNK, kind)
+    y = gpu_gemm(fb, kind, *ops, mode=1)
+    check(orc, y, kind, *ops)
+    yr, ya = orc.gemm_ref_tile(kind, *ops, 0, MNK[0], 0, MNK[1])
+    assert orc.check_tol(y, yr, ya, rel=1e-3)[0] == 0
+
+
+def test_pow2_mode_rejects_other_scales(fb, orc):
+    """A scale that is not a power of two in FP8BW_SCALE_POW2 mode is latched
+    as FP8BW_ERR_DEVICE_CHECK."""
+    rng = np.random.default_rng(1)
+    A, sA, B, sB = rand_ops_pow2(rng, 128, 256, 256, 0)
+    sA[1, 5] = 0.75
+    D = torch.zeros((128, 256), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_gemm(0, dev(A), dev(sA), dev(B), dev(sB), D, 1)
+    assert fb.fp8bw_last_device_error() == 6
