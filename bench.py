@@ -421,6 +421,31 @@ def main():
     timed_long = ms_total > 1000.0
     fp8_peak = 2.0 * (pk["bf16_sustained"] if timed_long else pk["bf16_burst"])
 
+    # ---- the same step with power-of-2 scales (block-scaled MMA path)
+    pow2 = None
+    if args.mode == "fp32":
+        for _ in range(max(args.warmup, 3)):
+            run_step(fb, layers, fb.FP8BW_SCALE_POW2)
+        torch.cuda.synchronize()
+        barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        for _ in range(args.steps):
+            run_step(fb, layers, fb.FP8BW_SCALE_POW2)
+        p1.record()
+        torch.cuda.synchronize()
+        p_ms = p0.elapsed_time(p1)
+        if dist:
+            t = torch.tensor([p_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            p_ms = float(t.item())
+        st = fb.fp8bw_last_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error (pow2): {fb.status_string(st)}")
+        pow2 = {"value": step_flops * args.steps * world / (p_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": p_ms / args.steps,
+                "note": "same step with power-of-2 scales (GEMMs on the block-scaled MMA)"}
+
     # ---- BF16 comparison GEMMs (outside the timed region)
     bf16 = bf16_ratio(fb, layers) if rank == 0 else None
 
@@ -433,16 +458,43 @@ def main():
         h2d = sum(x.numel() * 2 + w.numel() * 2 + d.numel() * 2 for x, w, d in host_in)
         d2h = sum(a.numel() * 2 + b.numel() * 2 + c.numel() * 2 for a, b, c in host_out)
 
+        # Copies overlap the compute: host->device on one stream, device->host
+        # on another, the layers in order on the compute stream; a step's
+        # uploads start once the previous step's compute has finished.
+        comp = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
         def e2e_step():
-            for l, (x, w, d) in zip(layers, host_in):
-                l.X.copy_(x, non_blocking=True)
-                l.W.copy_(w, non_blocking=True)
-                l.dY.copy_(d, non_blocking=True)
-            run_step(fb, layers, mode)
-            for l, (a, b, c) in zip(layers, host_out):
-                a.copy_(l.Y, non_blocking=True)
-                b.copy_(l.dX, non_blocking=True)
-                c.copy_(l.dW, non_blocking=True)
+            s_in.wait_stream(comp)
+            with torch.cuda.stream(s_in):
+                for l, (x, w, d) in zip(layers, host_in):
+                    l.W.copy_(w, non_blocking=True)
+                ev_w = torch.cuda.Event()
+                ev_w.record(s_in)
+                ev_in = []
+                for l, (x, w, d) in zip(layers, host_in):
+                    l.X.copy_(x, non_blocking=True)
+                    l.dY.copy_(d, non_blocking=True)
+                    ev_in.append(torch.cuda.Event())
+                    ev_in[-1].record(s_in)
+            comp.wait_event(ev_w)
+            fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT) for l in layers], mode)
+            for i, l in enumerate(layers):
+                comp.wait_event(ev_in[i])
+                fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)
+                fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode)
+                fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)
+                fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode)
+                fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode)
+                ev = torch.cuda.Event()
+                ev.record(comp)
+                s_out.wait_event(ev)
+                with torch.cuda.stream(s_out):
+                    a, b, c = host_out[i]
+                    a.copy_(l.Y, non_blocking=True)
+                    b.copy_(l.dX, non_blocking=True)
+                    c.copy_(l.dW, non_blocking=True)
+            comp.wait_stream(s_out)
         e2e_step()
         torch.cuda.synchronize()
         barrier()
@@ -486,6 +538,7 @@ def main():
                       "hbm_peak_gbs": pk["hbm_gbs"],
                       "bf16_gemm_tflops": bf16, "fp8_over_bf16": (gemm_tflops / bf16) if bf16 else None,
                       "requant_over_step": req_ms / ms_step},
+            "pow2_scales": pow2,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": ck,
             "e2e": e2e,

@@ -23,7 +23,7 @@ FP8BW_OK = 0
 FP8BW_SCALE_FP32, FP8BW_SCALE_POW2 = 0, 1
 FP8BW_FPROP, FP8BW_DGRAD, FP8BW_WGRAD = 0, 1, 2
 FP8BW_REQUANT_MAX_PER_LAUNCH = 256
-FP8BW_MAX_EXPERTS = 1024
+FP8BW_MAX_EXPERTS = 512
 STATUS = {0: "FP8BW_OK", 1: "FP8BW_ERR_INVALID_ARG", 2: "FP8BW_ERR_ALIGNMENT",
           3: "FP8BW_ERR_UNSUPPORTED_ARCH", 4: "FP8BW_ERR_CUDA", 5: "FP8BW_ERR_TIMEOUT",
           6: "FP8BW_ERR_DEVICE_CHECK", 7: "FP8BW_ERR_TOO_LARGE"}

@@ -215,6 +215,24 @@ __device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t adesc, uint64_
       : "memory");
 }
 
+// Pair form: issued by the first CTA of a pair, D in both CTAs' TMEM.
+__device__ __forceinline__ void umma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Pair form of the copy below: each CTA of the pair copies from its own
+// shared memory into its own TMEM (issued by the first CTA).
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Shared memory -> TMEM: 32 rows x 128 bits, written to all four 32-lane
 // quarters of TMEM (lanes i, 32+i, 64+i, 96+i get row i), 4 columns.
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {

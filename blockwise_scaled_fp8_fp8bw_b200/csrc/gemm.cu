@@ -485,11 +485,14 @@ done:
 // (tcgen05.mma.kind::mxf8f6f4.block_scale): each 128-wide scale block is one
 // UE8M0 byte replicated over its four 32-element MMA blocks, and the whole K
 // loop accumulates in one TMEM accumulator with no promotion.
-// One CTA per SM, 128x256 tiles, 384 threads:
-//   warp 0      TMA producer (4-stage ring of 48 KB stages)
-//   warp 1      MMA issuer: per chunk, tcgen05.cp of the chunk's scale
-//               bytes (A: 128 rows, B: 256 rows) from shared memory into a
-//               per-stage TMEM slot, then four block-scaled MMAs
+// Tiles as in the promotion kernel: 256x256 per CTA pair (cta_group::2) for
+// dense GEMMs and grouped wgrad, 128x256 per CTA for grouped fprop/dgrad.
+// 384 threads per CTA:
+//   warp 0      TMA producer
+//   warp 1      MMA issuer (first CTA of a pair): per chunk, tcgen05.cp of
+//               the chunk's scale bytes (A: the CTA's 128 rows, B: all 256
+//               rows) from shared memory into a per-stage TMEM slot of each
+//               CTA, then four block-scaled MMAs
 //   warp 2      scale loader: fp32 scales by cp.async into a raw ring, then
 //               converted to UE8M0 bytes in the tcgen05.cp layout (row r of a
 //               128-row group at lane r%32, word r/32; the four bytes of a
@@ -497,14 +500,26 @@ done:
 //               of two latches FP8BW_ERR_DEVICE_CHECK
 //   warps 4-11  epilogue: drain the accumulator (tcgen05.ld), release it,
 //               round to bf16 and TMA-store (as in the promotion kernel)
-constexpr int kMxStages = 4;
-constexpr int kMxRaw = 4;                       // raw scale slots; lookahead kMxRaw-1
-constexpr uint32_t kMxStageBytes = kATile + BN * BK;  // 16 KB A + 32 KB B
+// Scales of 4 consecutive chunks share one TMEM word per row (byte j = chunk
+// j of the group; the MMAs of a chunk select their byte), so one tcgen05.cp
+// per matrix serves 4 chunks.
+constexpr int kSfGroup = 4;                     // chunks per scale group
+constexpr int kSfSlots = 2;                     // scale groups in flight
+constexpr int kMxRaw = kSfGroup * kSfSlots;     // raw fp32 chunk slots
 constexpr uint32_t kSfCol0 = 256;               // TMEM: accumulator [0,256), scales after
-constexpr uint32_t kSfCols = 12;                // per stage: A 4 columns + B 8 columns
+constexpr uint32_t kSfCols = 12;                // per group: A 4 columns + B 8 columns
+constexpr int kMxMaxStages = 6;
+
+template <bool PAIR>
+struct MxCfg {
+  static constexpr uint32_t kStageBytes = kATile + (PAIR ? (BN / 2) * BK : BN * BK);
+  static constexpr int kStages = PAIR ? 5 : 4;
+  static constexpr uint32_t kIdescM = PAIR ? 2 * BM : BM;
+};
 
 struct MxBars {
-  uint64_t full[kMxStages], empty[kMxStages], sffull[kMxStages];
+  uint64_t full[kMxMaxStages], empty[kMxMaxStages];
+  uint64_t sffull[kSfSlots], sfempty[kSfSlots];
   uint64_t tfull, tempty;
   uint32_t tmem_base;
   int32_t abort;
@@ -515,54 +530,103 @@ struct SfSlot {
   uint32_t b[2][32][4];  // B rows 0..127 and 128..255
 };
 
-constexpr size_t kSmemMx = 1024 + size_t(kMxStages) * kMxStageBytes + 8 * kEpiPiece +
-                           size_t(kMxRaw) * sizeof(ScaleSlot) + size_t(kMxStages) * sizeof(SfSlot) +
-                           sizeof(MxBars) + sizeof(int32_t) * (kMaxGroups + 1);
-static_assert(kSmemMx <= 232448, "shared memory budget (MX)");
+template <bool PAIR>
+constexpr size_t smem_mx() {
+  return 1024 + size_t(MxCfg<PAIR>::kStages) * MxCfg<PAIR>::kStageBytes + 8 * kEpiPiece +
+         size_t(kMxRaw) * sizeof(ScaleSlot) + size_t(kSfSlots) * sizeof(SfSlot) +
+         sizeof(MxBars) + sizeof(int32_t) * (kMaxGroups + 1);
+}
+static_assert(smem_mx<true>() <= 232448 && smem_mx<false>() <= 232448, "shared memory budget (MX)");
 
-// UE8M0 byte of a power-of-2 fp32 scale (2^-127 is the subnormal 0x00400000).
+// UE8M0 byte of a power-of-2 fp32 scale (2^-127 is the subnormal 0x00400000),
+// replicated into the four bytes of a word.
 __device__ __forceinline__ uint32_t ue8m0_x4(float s, bool& bad) {
   const uint32_t b = __float_as_uint(s);
-  const uint32_t e = b >> 23;
   if ((b & 0x7FFFFFu) != 0u && b != 0x00400000u) bad = true;
-  return (e & 0xFFu) * 0x01010101u;
+  return ((b >> 23) & 0xFFu) * 0x01010101u;
 }
 
-template <int KIND, bool GROUPED>
+// Builds one scale group: byte j of every word comes from chunk j of the
+// group (raw slots r[0..n-1]); bytes of absent chunks hold 127 (1.0).
+template <int KIND>
+__device__ __forceinline__ void sf_convert(const ScaleSlot* const* r, int n, SfSlot* o, int lane,
+                                           bool& bad) {
+  uint32_t wa[4] = {0, 0, 0, 0}, wb[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+#pragma unroll
+  for (int j = 0; j < kSfGroup; ++j) {
+    const uint32_t sh = 8 * j;
+    if (j < n) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) wa[b] |= (ue8m0_x4(r[j]->sa[lane + 32 * b], bad) & 0xFFu) << sh;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float v = (KIND == FP8BW_WGRAD) ? r[j]->sb[h * 128 + lane + 32 * b] : r[j]->sb[h];
+          wb[h][b] |= (ue8m0_x4(v, bad) & 0xFFu) << sh;
+        }
+    } else {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        wa[b] |= 127u << sh;
+        wb[0][b] |= 127u << sh;
+        wb[1][b] |= 127u << sh;
+      }
+    }
+  }
+  *reinterpret_cast<uint4*>(&o->a[lane][0]) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+  *reinterpret_cast<uint4*>(&o->b[0][lane][0]) = make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
+  *reinterpret_cast<uint4*>(&o->b[1][lane][0]) = make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
+}
+
+template <int KIND, bool GROUPED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
+  using C = MxCfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint8_t* epi_base = smem + kMxStages * kMxStageBytes;
+  uint8_t* epi_base = smem + C::kStages * C::kStageBytes;
   ScaleSlot* raw = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kEpiPiece);
   SfSlot* sf = reinterpret_cast<SfSlot*>(raw + kMxRaw);
-  MxBars* bars = reinterpret_cast<MxBars*>(sf + kMxStages);
+  MxBars* bars = reinterpret_cast<MxBars*>(sf + kSfSlots);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int cta_slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int cta_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMxStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
-      mbar_init(smem_u32(&bars->sffull[i]), 1);
+    }
+    for (int i = 0; i < kSfSlots; ++i) {
+      mbar_init(smem_u32(&bars->sffull[i]), PAIR ? 2 : 1);
+      mbar_init(smem_u32(&bars->sfempty[i]), 1);
     }
     mbar_init(smem_u32(&bars->tfull), 1);
-    mbar_init(smem_u32(&bars->tempty), 8);
+    mbar_init(smem_u32(&bars->tempty), PAIR ? 16 : 8);
     bars->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (GROUPED) {
     for (int i = threadIdx.x; i <= a.G; i += kThreads) s_off[i] = a.offsets[i];
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (GROUPED) {
     int bad = 0;
@@ -577,12 +641,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__syncthreads_or(bad)) {
       if (threadIdx.x == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
       tc_fence_before();
-      if (warp == 1) tmem_dealloc(bars->tmem_base, kTmemCols);
+      if (PAIR) cluster_sync();
+      if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(bars->tmem_base, kTmemCols);
+        else tmem_dealloc(bars->tmem_base, kTmemCols);
+      }
       return;
     }
   }
   const uint32_t tmem = bars->tmem_base;
-  const int cta_slot = blockIdx.x, cta_step = gridDim.x;
+  // Barriers the MMA waits on live in the first CTA of a pair.
+  const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&bars->full[0]), 0) : smem_u32(&bars->full[0]);
+  const uint32_t sffull0 = PAIR ? mapa_shared(smem_u32(&bars->sffull[0]), 0) : smem_u32(&bars->sffull[0]);
+  const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(&bars->tempty), 0) : smem_u32(&bars->tempty);
 
   if (warp < 4) {
     regs_dec<kRegsLow>();
@@ -597,31 +668,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
         const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
         if (ti.skip) continue;
+        const int arow = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++chunk) {
           if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
             raise_timeout_mx(bars);
             goto done;
           }
           if (lane == 0 && !(blockIdx.x == 0 && chunk == a.stall_chunk)) {
-            const uint32_t full = smem_u32(&bars->full[stage]);
-            const uint32_t sa = smem_u32(stage_base + stage * kMxStageBytes);
-            mbar_arrive_expect_tx(full, kMxStageBytes);
-            tma_load_2d(sa, &tmA, full, kb * BK, ti.mt * BM);
-            if (GROUPED && KIND != FP8BW_WGRAD)
-              tma_load_3d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN, ti.g);
-            else
-              tma_load_2d(sa + kATile, &tmB, full, kb * BK, ti.nt * BN);
+            const uint32_t full = full0 + stage * 8;
+            const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+            if (PAIR) {
+              if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[stage]), 2 * C::kStageBytes);
+              tma_load_2d_pair(sa, &tmA, full, kb * BK, arow);
+              tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
+            } else {
+              mbar_arrive_expect_tx(full, C::kStageBytes);
+              tma_load_2d(sa, &tmA, full, kb * BK, arow);
+              if (GROUPED && KIND != FP8BW_WGRAD)
+                tma_load_3d(sa + kATile, &tmB, full, kb * BK, brow, ti.g);
+              else
+                tma_load_2d(sa + kATile, &tmB, full, kb * BK, brow);
+            }
           }
           __syncwarp();
-          if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (bars->abort) break;
       }
     } else if (warp == 1) {
       // ------------------------------------------------- MMA issuer -----
-      if (lane == 0) {
-        int stage = 0;
-        uint32_t phase = 0, tphase = 0;
+      if (leader && lane == 0) {
+        int stage = 0, gslot = 0;
+        uint32_t phase = 0, tphase = 0, gphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
           const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
           if (ti.skip || ti.kb0 == ti.kb1) continue;
@@ -631,109 +710,134 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-            if (!mbar_wait(smem_u32(&bars->full[stage]), phase) ||
-                !mbar_wait(smem_u32(&bars->sffull[stage]), phase)) {
+            const int i = kb - ti.kb0, j = i % kSfGroup;
+            const uint32_t tsf = tmem + kSfCol0 + gslot * kSfCols;
+            if (j == 0) {
+              if (!mbar_wait(smem_u32(&bars->sffull[gslot]), gphase)) {
+                raise_timeout_mx(bars);
+                goto done;
+              }
+              tc_fence_after();
+              const uint64_t sda = sdesc_k_noswz_16B(smem_u32(&sf[gslot].a[0][0]));
+              const uint64_t sdb0 = sdesc_k_noswz_16B(smem_u32(&sf[gslot].b[0][0][0]));
+              const uint64_t sdb1 = sdesc_k_noswz_16B(smem_u32(&sf[gslot].b[1][0][0]));
+              if (PAIR) {
+                tmem_cp_32x128b_x4_pair(tsf, sda);
+                tmem_cp_32x128b_x4_pair(tsf + 4, sdb0);
+                tmem_cp_32x128b_x4_pair(tsf + 8, sdb1);
+              } else {
+                tmem_cp_32x128b_x4(tsf, sda);
+                tmem_cp_32x128b_x4(tsf + 4, sdb0);
+                tmem_cp_32x128b_x4(tsf + 8, sdb1);
+              }
+            }
+            if (!mbar_wait(smem_u32(&bars->full[stage]), phase)) {
               raise_timeout_mx(bars);
               goto done;
             }
             tc_fence_after();
-            const uint32_t tsf = tmem + kSfCol0 + stage * kSfCols;
-            tmem_cp_32x128b_x4(tsf, sdesc_k_noswz_16B(smem_u32(&sf[stage].a[0][0])));
-            tmem_cp_32x128b_x4(tsf + 4, sdesc_k_noswz_16B(smem_u32(&sf[stage].b[0][0][0])));
-            tmem_cp_32x128b_x4(tsf + 8, sdesc_k_noswz_16B(smem_u32(&sf[stage].b[1][0][0])));
-            const uint32_t sa = smem_u32(stage_base + stage * kMxStageBytes);
+            const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
             const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
 #pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              umma_mx(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(BM, BN, kk), tsf, tsf + 4,
-                      (kb > ti.kb0 || kk > 0) ? 1u : 0u);
-            umma_commit(smem_u32(&bars->empty[stage]));
-            if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              const uint32_t acc = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
+              if (PAIR)
+                umma_mx_pair(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j), tsf, tsf + 4, acc);
+              else
+                umma_mx(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j), tsf, tsf + 4, acc);
+            }
+            if (PAIR) umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
+            else umma_commit(smem_u32(&bars->empty[stage]));
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            if (j == kSfGroup - 1 || kb + 1 == ti.kb1) {
+              // the group's scales may be replaced once these MMAs are done
+              if (PAIR) umma_commit_pair(smem_u32(&bars->sfempty[gslot]), 0x3);
+              else umma_commit(smem_u32(&bars->sfempty[gslot]));
+              if (++gslot == kSfSlots) { gslot = 0; gphase ^= 1; }
+            }
           }
-          umma_commit(smem_u32(&bars->tfull));
+          if (PAIR) umma_commit_pair(smem_u32(&bars->tfull), 0x3);
+          else umma_commit(smem_u32(&bars->tfull));
           tphase ^= 1;
           if (bars->abort) break;
         }
       }
     } else if (warp == 2) {
       // ------------------------------------------------ scale loader ----
-      // Chunk c's fp32 scales go to raw slot c % kMxRaw by cp.async; chunk
-      // c - (kMxRaw - 1) is converted once its copies have landed.
-      constexpr int L = kMxRaw - 1;
+      // Per scale group (up to 4 chunks of one tile): the chunks' fp32 scales
+      // go to raw slots by cp.async as one copy group; the previous group is
+      // converted once its copies have landed and its SF slot is free.
       const int nKb = a.K / BK, nNb = a.N / 128;
-      int issued = 0, done_c = 0, sstage = 0;
-      uint32_t sphase = 0;
-      bool bad = false;
-      auto convert = [&](int d) -> bool {
-        __syncwarp();
-        if (!mbar_wait(smem_u32(&bars->empty[sstage]), sphase ^ 1)) return false;
-        const ScaleSlot* r = &raw[d % kMxRaw];
-        SfSlot* o = &sf[sstage];
-        uint4 wa;
-        wa.x = ue8m0_x4(r->sa[lane], bad);
-        wa.y = ue8m0_x4(r->sa[lane + 32], bad);
-        wa.z = ue8m0_x4(r->sa[lane + 64], bad);
-        wa.w = ue8m0_x4(r->sa[lane + 96], bad);
-        *reinterpret_cast<uint4*>(&o->a[lane][0]) = wa;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4 wb;
-          if (KIND == FP8BW_WGRAD) {
-            wb.x = ue8m0_x4(r->sb[h * 128 + lane], bad);
-            wb.y = ue8m0_x4(r->sb[h * 128 + lane + 32], bad);
-            wb.z = ue8m0_x4(r->sb[h * 128 + lane + 64], bad);
-            wb.w = ue8m0_x4(r->sb[h * 128 + lane + 96], bad);
-          } else {
-            wb.x = wb.y = wb.z = wb.w = ue8m0_x4(r->sb[h], bad);
-          }
-          *reinterpret_cast<uint4*>(&o->b[h][lane][0]) = wb;
+      int rbase = 0, gslot = 0, pend_n = 0, pend_base = 0;
+      uint32_t gphase = 0;
+      bool bad = false, pend = false;
+      for (int t = cta_slot;; t += cta_step) {
+        const bool have = t < a.tiles;
+        TileInfo ti = {};
+        if (have) {
+          ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          if (ti.skip) continue;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->sffull[sstage]));
-        if (++sstage == kMxStages) { sstage = 0; sphase ^= 1; }
-        return true;
-      };
-      for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
-        if (ti.skip) continue;
+        const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
         const float* sBg = a.sB;
         if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          ScaleSlot* sl = &raw[issued % kMxRaw];
-          // unused entries hold 1.0 (byte 127) so no stale value is checked
-          cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + ti.mt * BM + lane * 4);
-          if (KIND == FP8BW_WGRAD) {
+        for (int kg = ti.kb0; have ? kg < ti.kb1 : pend; kg += kSfGroup) {
+          int n = 0;
+          if (have) {
+            n = min(kSfGroup, ti.kb1 - kg);
+            for (int j = 0; j < n; ++j) {
+              const int kb = kg + j;
+              ScaleSlot* sl = &raw[(rbase + j) % kMxRaw];
+              if (row0 < a.M)
+                cp_async_16(smem_u32(&sl->sa[lane * 4]), a.sA + (size_t)kb * a.M + row0 + lane * 4);
+              else
+                *reinterpret_cast<float4*>(&sl->sa[lane * 4]) = make_float4(1.f, 1.f, 1.f, 1.f);
+              if (KIND == FP8BW_WGRAD) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int n = ti.nt * BN + h * 128 + lane * 4;
-              if (n < a.N) cp_async_16(smem_u32(&sl->sb[h * 128 + lane * 4]), sBg + (size_t)kb * a.N + n);
-              else *reinterpret_cast<float4*>(&sl->sb[h * 128 + lane * 4]) = make_float4(1.f, 1.f, 1.f, 1.f);
+                for (int h = 0; h < 2; ++h) {
+                  const int nn = ti.nt * BN + h * 128 + lane * 4;
+                  if (nn < a.N) cp_async_16(smem_u32(&sl->sb[h * 128 + lane * 4]), sBg + (size_t)kb * a.N + nn);
+                  else *reinterpret_cast<float4*>(&sl->sb[h * 128 + lane * 4]) = make_float4(1.f, 1.f, 1.f, 1.f);
+                }
+              } else if (lane < 2) {
+                const int nb = ti.nt * 2 + lane;
+                if (nb < nNb)
+                  cp_async_4(smem_u32(&sl->sb[lane]), (KIND == FP8BW_FPROP) ? sBg + (size_t)nb * nKb + kb
+                                                                            : sBg + (size_t)kb * nNb + nb);
+                else
+                  sl->sb[lane] = 1.f;
+              }
             }
-          } else if (lane < 2) {
-            const int nb = ti.nt * 2 + lane;
-            if (nb < nNb) {
-              const float* src = (KIND == FP8BW_FPROP) ? sBg + (size_t)nb * nKb + kb
-                                                       : sBg + (size_t)kb * nNb + nb;
-              cp_async_4(smem_u32(&sl->sb[lane]), src);
-            } else {
-              sl->sb[lane] = 1.f;
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 1;" ::: "memory");  // the previous group has landed
+          } else {
+            asm volatile("cp.async.wait_all;" ::: "memory");
+          }
+          __syncwarp();
+          if (pend) {
+            if (!mbar_wait(smem_u32(&bars->sfempty[gslot]), gphase ^ 1)) {
+              raise_timeout_mx(bars);
+              goto done;
             }
+            const ScaleSlot* r[kSfGroup];
+#pragma unroll
+            for (int j = 0; j < kSfGroup; ++j) r[j] = &raw[(pend_base + j) % kMxRaw];
+            sf_convert<KIND>(r, pend_n, &sf[gslot], lane, bad);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (PAIR && !leader) mbar_arrive_cluster(sffull0 + gslot * 8);
+              else mbar_arrive(smem_u32(&bars->sffull[gslot]));
+            }
+            if (++gslot == kSfSlots) { gslot = 0; gphase ^= 1; }
           }
-          asm volatile("cp.async.commit_group;" ::: "memory");
-          ++issued;
-          if (issued - done_c > L) {
-            asm volatile("cp.async.wait_group %0;" ::"n"(L) : "memory");
-            if (!convert(done_c)) { raise_timeout_mx(bars); goto done; }
-            ++done_c;
-          }
+          pend = have;
+          pend_n = n;
+          pend_base = rbase;
+          rbase = (rbase + kSfGroup) % kMxRaw;
+          if (!have) break;
         }
-        if (bars->abort) break;
-      }
-      asm volatile("cp.async.wait_all;" ::: "memory");
-      while (done_c < issued) {
-        if (!convert(done_c)) { raise_timeout_mx(bars); goto done; }
-        ++done_c;
+        if (!have || bars->abort) break;
       }
       if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_gemm_error, DEV_ERR_CHECK);
     }
@@ -746,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
       const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
       if (ti.skip) continue;
-      const int row0 = ti.mt * BM;
+      const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
       const int col0 = ti.nt * BN + half * 128;
       float2 acc[64];
       if (ti.kb0 == ti.kb1) {
@@ -773,12 +877,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->tempty));
+        if (lane == 0) {
+          if (PAIR && !leader) mbar_arrive_cluster(tempty0);
+          else mbar_arrive(smem_u32(&bars->tempty));
+        }
         tphase ^= 1;
       }
       const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < 4 && row0 < a.M; ++p) {
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
 #pragma unroll
@@ -803,10 +910,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 done:
   if (warp >= 4 && lane == 0) bulk_wait0();
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -997,14 +1105,28 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
 }
 
-template <int KIND, bool GROUPED>
+template <int KIND, bool GROUPED, bool PAIR>
 cudaError_t launch_mx(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                       const GemmArgs& a, int grid, cudaStream_t st) {
-  auto kern = k_gemm_mx<KIND, GROUPED>;
-  cudaError_t e = prepare(kern, kSmemMx, true);
+  auto kern = k_gemm_mx<KIND, GROUPED, PAIR>;
+  const size_t smem = smem_mx<PAIR>();
+  cudaError_t e = prepare(kern, smem, true);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemMx, st>>>(ta, tb, td, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
 }
 
 }  // namespace
@@ -1047,32 +1169,24 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
     return cudaErrorInvalidValue;
   int grid;
   cudaError_t e;
-  if (mode == FP8BW_SCALE_POW2) {
-    // 1-CTA 128x256 tiles over the whole problem
-    a.m_tiles = (int)(M / BM);
-    a.band = gemm_band_rows;
-    a.tiles = (grouped && kind == FP8BW_WGRAD) ? G * a.m_tiles * a.n_tiles : a.m_tiles * a.n_tiles;
-    if (pair && !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, BN,
-                          CU_TENSOR_MAP_SWIZZLE_128B, 0))
-      return cudaErrorInvalidValue;
-    grid = a.tiles < num_sms ? a.tiles : num_sms;
-    if (!grouped) {
-      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false>(ta, tb, td, a, grid, st);
-      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false>(ta, tb, td, a, grid, st);
-      else e = launch_mx<FP8BW_WGRAD, false>(ta, tb, td, a, grid, st);
-    } else {
-      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, true>(ta, tb, td, a, grid, st);
-      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, true>(ta, tb, td, a, grid, st);
-      else e = launch_mx<FP8BW_WGRAD, true>(ta, tb, td, a, grid, st);
-    }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-  }
   if (pair) {
     const int clusters = num_sms / 2;
     grid = 2 * (a.tiles < clusters ? a.tiles : clusters);
   } else {
     grid = a.tiles < num_sms ? a.tiles : num_sms;
+  }
+  if (mode == FP8BW_SCALE_POW2) {
+    if (!grouped) {
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false, true>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false, true>(ta, tb, td, a, grid, st);
+      else e = launch_mx<FP8BW_WGRAD, false, true>(ta, tb, td, a, grid, st);
+    } else {
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, true, false>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, true, false>(ta, tb, td, a, grid, st);
+      else e = launch_mx<FP8BW_WGRAD, true, true>(ta, tb, td, a, grid, st);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
   }
   if (!grouped) {
     if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true>(ta, tb, td, a, grid, st);

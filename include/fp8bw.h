@@ -178,7 +178,7 @@ FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, in
  *                D [G][N][K]: expert g contracts only its own tokens; an
  *                expert with no tokens gets exact zeros.
  * Requires G <= FP8BW_MAX_EXPERTS. */
-#define FP8BW_MAX_EXPERTS 1024
+#define FP8BW_MAX_EXPERTS 512
 FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
                                 int64_t M_total_pad, int64_t N, int64_t K,
                                 const uint8_t* A, const float* sA, const uint8_t* B,
