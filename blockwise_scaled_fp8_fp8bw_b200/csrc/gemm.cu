@@ -386,43 +386,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const ScaleSlot* sl = &slots[ss];
-        const float sa = sl->sa[q * 32 + lane];
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
-        // Two rounds of two 32-column loads: one wait per 64 columns keeps
-        // the staging at 64 registers next to the 128 accumulators.
+        if (KIND == FP8BW_WGRAD) {
+          // Column scales change with every column, so each thread needs the
+          // scale of every column it holds.  The 16x256b TMEM shape gives a
+          // thread 4 rows x 32 columns (instead of 1 row x 128 columns), so
+          // a chunk costs 4 row-scale and 16 column-pair loads from shared
+          // memory instead of 128 column-scale loads.
+          // acc[16 * i + g] holds row 8i + lane/4 of the quarter and columns
+          // 8g + 2(lane%4) + {0, 1} of the warp's 128.
+          float sa[4];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t r[2][32];
-          tmem_ld64(taddr + h2 * 64, r[0], r[1]);
-          tmem_wait_ld();
-          if (h2 == 1) {
-            // chunk fully read: hand the TMEM buffer back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
-              else mbar_arrive(smem_u32(&bars->tempty[buf]));
+          for (int i = 0; i < 4; ++i) sa[i] = sl->sa[q * 32 + 8 * i + (lane >> 2)];
+          const float* sbw = &sl->sb[half * 128 + 2 * (lane & 3)];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {  // 64-column halves of the warp's 128 columns
+            uint32_t r[2][32];
+            tmem_ld16x64(taddr + h2 * 64, r[0]);                      // quarter lanes 0-15
+            tmem_ld16x64(taddr + (16u << 16) + h2 * 64, r[1]);        // quarter lanes 16-31
+            tmem_wait_ld();
+            if (h2 == 1) {
+              // chunk fully read: hand the TMEM buffer back to the MMA warp
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
+                else mbar_arrive(smem_u32(&bars->tempty[buf]));
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int g = h2 * 8 + j;
+              const float2 b2 = *reinterpret_cast<const float2*>(sbw + 8 * g);
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                  const int i = 2 * u + v;
+                  const float2 sc = fmul2(make_float2(sa[i], sa[i]), b2);
+                  acc[16 * i + g] = ffma2(make_float2(__uint_as_float(r[u][4 * j + 2 * v]),
+                                                      __uint_as_float(r[u][4 * j + 2 * v + 1])),
+                                          sc, acc[16 * i + g]);
+                }
+              }
             }
           }
+        } else {
+          const float sa = sl->sa[q * 32 + lane];
+          // Two rounds of two 32-column loads: one wait per 64 columns keeps
+          // the staging at 64 registers next to the 128 accumulators.
 #pragma unroll
-          for (int p2 = 0; p2 < 2; ++p2) {
-            const int p = h2 * 2 + p2;
-            if (KIND == FP8BW_WGRAD) {
-              const float2 sa2 = make_float2(sa, sa);
-              const float4* sb4 = reinterpret_cast<const float4*>(&sl->sb[half * 128 + p * 32]);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 b4 = sb4[j];  // one broadcast load serves four columns
-                const float2 sc0 = fmul2(sa2, make_float2(b4.x, b4.y));
-                const float2 sc1 = fmul2(sa2, make_float2(b4.z, b4.w));
-                acc[p * 16 + 2 * j] = ffma2(make_float2(__uint_as_float(r[p2][4 * j]), __uint_as_float(r[p2][4 * j + 1])),
-                                            sc0, acc[p * 16 + 2 * j]);
-                acc[p * 16 + 2 * j + 1] = ffma2(make_float2(__uint_as_float(r[p2][4 * j + 2]), __uint_as_float(r[p2][4 * j + 3])),
-                                                sc1, acc[p * 16 + 2 * j + 1]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t r[2][32];
+            tmem_ld64(taddr + h2 * 64, r[0], r[1]);
+            tmem_wait_ld();
+            if (h2 == 1) {
+              // chunk fully read: hand the TMEM buffer back to the MMA warp
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
+                else mbar_arrive(smem_u32(&bars->tempty[buf]));
               }
-            } else {
-              const float s = sa * sl->sb[half];
-              const float2 s2 = make_float2(s, s);
+            }
+            const float s = sa * sl->sb[half];
+            const float2 s2 = make_float2(s, s);
+#pragma unroll
+            for (int p2 = 0; p2 < 2; ++p2) {
+              const int p = h2 * 2 + p2;
 #pragma unroll
               for (int j = 0; j < 16; ++j)
                 acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1])),
@@ -447,15 +478,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
         }
         __syncwarp();
-        // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
+        if (KIND == FP8BW_WGRAD) {
+          // rows 8i + lane/4, columns 8c + 2(lane%4) + {0, 1} of the piece:
+          // one bf16 pair per store; the 64-byte swizzle keeps the 32 lanes
+          // of each store on 32 distinct banks
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 o;
-          o.x = pack_bf16x2(acc[p * 16 + 4 * c + 0].x, acc[p * 16 + 4 * c + 0].y);
-          o.y = pack_bf16x2(acc[p * 16 + 4 * c + 1].x, acc[p * 16 + 4 * c + 1].y);
-          o.z = pack_bf16x2(acc[p * 16 + 4 * c + 2].x, acc[p * 16 + 4 * c + 2].y);
-          o.w = pack_bf16x2(acc[p * 16 + 4 * c + 3].x, acc[p * 16 + 4 * c + 3].y);
-          *reinterpret_cast<uint4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = o;
+          for (int i = 0; i < 4; ++i) {
+            const int row = 8 * i + (lane >> 2);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 v2 = acc[16 * i + 4 * p + c];
+              *reinterpret_cast<uint32_t*>(epi + row * 64 + 16 * (c ^ ((row >> 1) & 3)) + 4 * (lane & 3)) =
+                  pack_bf16x2(v2.x, v2.y);
+            }
+          }
+        } else {
+          // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[p * 16 + 4 * c + 0].x, acc[p * 16 + 4 * c + 0].y);
+            o.y = pack_bf16x2(acc[p * 16 + 4 * c + 1].x, acc[p * 16 + 4 * c + 1].y);
+            o.z = pack_bf16x2(acc[p * 16 + 4 * c + 2].x, acc[p * 16 + 4 * c + 2].y);
+            o.w = pack_bf16x2(acc[p * 16 + 4 * c + 3].x, acc[p * 16 + 4 * c + 3].y);
+            *reinterpret_cast<uint4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = o;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
