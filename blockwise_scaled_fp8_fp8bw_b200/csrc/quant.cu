@@ -6,27 +6,27 @@
 // Durchbruch" (E4M3, 128x128 weight blocks, 1x128 activation blocks) and
 // "Leistungsgewinne in der Praxis" (scales recalibrated after every step).
 //
-// Design: one CTA of 256 threads per 128x128 bf16 tile (32 KB).  Each thread
-// loads eight 16-byte vectors (a half-warp covers one 256-byte row segment),
-// keeps them in registers for the row-wise pass and parks them in shared
-// memory for the column-wise pass.
+// Design: activations go through persistent CTAs of 256 threads that walk
+// 128x128 bf16 tiles, TMA-loaded (two 64-column boxes, 128-byte swizzle) two
+// tiles ahead into a double buffer; weights take one CTA per 128x128 block.
 //  * amax: bf16 magnitudes compared as packed unsigned 16-bit integers
 //    (sign bit cleared; the bit order of non-negative bf16 values is their
 //    numeric order), two elements per instruction.
 //  * x / s: the block's divisor is fixed, so its IEEE reciprocal y = RN(1/s)
 //    is taken once per block and every element uses one Markstein correction
 //    step (P. Markstein, "Computation of elementary functions on the IBM
-//    RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
-//        q0 = RN(x*y);  r = fma(-q0, s, x) (exact);  q = fma(r, y, q0)
-//    on packed f32x2 lanes, and the sign of x is copied onto q.  An
-//    exhaustive check over every bf16 block amax >= 2^-80 and every bf16
-//    |x| <= amax shows q equals RN(x/s) wherever |x/s| >= 2^-12; below that
-//    both give a signed-zero code (tests/test_division_scheme.py).  Blocks
-//    with a smaller amax use IEEE division.  In power-of-2 mode 1/s is exact
-//    and x*(1/s) is the correctly rounded x/s.
-//  * codes leave as coalesced stores: row-wise codes as 8-byte stores (a
-//    half-warp writes a 128-byte row); column-wise codes are staged in a
-//    swizzled 16 KB shared tile and written as full 128-byte rows.
+//    RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990), in the
+//    sign-symmetric form
+//        q0 = RN(x*y);  r = fma(q0, s, -x) (exact);  q = fma(r, -y, q0)
+//    on packed f32x2 lanes.  An exhaustive check over every bf16 block amax
+//    >= 2^-80 and every bf16 |x| <= amax shows q equals RN(x/s) wherever
+//    |x/s| >= 2^-12 and that the signs always agree, signed zeros included
+//    (tests/test_division_scheme.py).  Blocks with a smaller amax use IEEE
+//    division.  In power-of-2 mode 1/s is exact and x*(1/s) is the
+//    correctly rounded x/s.
+//  * activation codes leave as 32-byte stores (whole sectors) straight from
+//    registers: a thread holds 64 consecutive row codes of one row, or 32
+//    consecutive tokens of two columns for the column-wise copy.
 
 #include "common.cuh"
 #include "tmap.cuh"
@@ -85,28 +85,25 @@ __device__ __forceinline__ Divisor make_divisor(float amax) {
   return d;
 }
 
-__device__ __forceinline__ float copysign_bits(float q, float x) {
-  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
-}
-
 // RN(x / s) for a pair of values with per-lane divisors (s0,y0), (s1,y1):
 // power-of-2 mode multiplies by the exact reciprocal, FP32 mode takes one
-// Markstein step.  Blocks that need IEEE division take the slow path below.
+// Markstein step in its sign-symmetric form (the remainder is taken as
+// q0*s - x and applied with -y), which gives -0 for x = -0 without a
+// separate sign copy.  Blocks that need IEEE division take the slow path.
 template <int MODE>
 __device__ __forceinline__ float2 div2(float2 x, float2 s, float2 y) {
   if (MODE == FP8BW_SCALE_POW2) return fmul2(x, y);
   const float2 q0 = fmul2(x, y);
-  const float2 r = ffma2(q0, make_float2(-s.x, -s.y), x);
-  const float2 q = ffma2(r, y, q0);
-  return make_float2(copysign_bits(q.x, x.x), copysign_bits(q.y, x.y));
+  const float2 r = ffma2(q0, s, make_float2(-x.x, -x.y));
+  return ffma2(r, make_float2(-y.x, -y.y), q0);
 }
 
 // Scalar RN(x / s) in FP32 mode, IEEE division for a block that needs it.
 __device__ __forceinline__ float div1(float x, const Divisor& d) {
   if (d.exact) return __fdiv_rn(x, d.s);
   const float q0 = __fmul_rn(x, d.y);
-  const float r = __fmaf_rn(-q0, d.s, x);
-  return copysign_bits(__fmaf_rn(r, d.y, q0), x);
+  const float r = __fmaf_rn(q0, d.s, -x);
+  return __fmaf_rn(r, -d.y, q0);
 }
 
 template <int MODE>
@@ -140,17 +137,18 @@ __device__ __forceinline__ uint2 quant8(uint4 v, const Divisor& d) {
 struct ColCodes {
   uint32_t c0[8], c1[8];
 };
+struct ColWords {
+  uint32_t w[32];
+};
 
-// Slow path of the column pass: re-reads the thread's 32 words.
-__device__ __noinline__ ColCodes column_codes_exact(const uint32_t (*tile)[64], int wc, int rg,
-                                                   Divisor d0, Divisor d1) {
+// Slow path of the column pass (a column block with amax < 2^-80).
+__device__ __noinline__ ColCodes column_codes_exact(ColWords v, Divisor d0, Divisor d1) {
   ColCodes c;
   for (int i = 0; i < 8; ++i) {
     float a[4], b[4];
     for (int u = 0; u < 4; ++u) {
-      const uint32_t w = tile[rg * 32 + 4 * i + u][wc];
-      a[u] = div1(bf16lo(w), d0);
-      b[u] = div1(bf16hi(w), d1);
+      a[u] = div1(bf16lo(v.w[4 * i + u]), d0);
+      b[u] = div1(bf16hi(v.w[4 * i + u]), d1);
     }
     c.c0[i] = cvt_e4m3x2(a[0], a[1]) | (cvt_e4m3x2(a[2], a[3]) << 16);
     c.c1[i] = cvt_e4m3x2(b[0], b[1]) | (cvt_e4m3x2(b[2], b[3]) << 16);
@@ -158,93 +156,39 @@ __device__ __noinline__ ColCodes column_codes_exact(const uint32_t (*tile)[64], 
   return c;
 }
 
-// Swizzled byte tile: row r (128 bytes = 8 chunks of 16 B); logical chunk j
-// lives at physical chunk j ^ ((r >> 1) & 7).
-__device__ __forceinline__ uint4* code_chunk(uint32_t* codes, int r, int j) {
-  return reinterpret_cast<uint4*>(codes + r * 32 + 4 * (j ^ ((r >> 1) & 7)));
-}
-
-// Writes the 128x128 transposed code tile to dst (row stride ld bytes) as
-// full 128-byte rows: thread t copies chunk t%8 of rows t/8 + 32i.
-__device__ __forceinline__ void store_code_tile(uint32_t (*tile)[64], uint8_t* dst, int64_t ld) {
-  uint32_t* codes = &tile[0][0];
-  const int t = threadIdx.x, j = t & 7;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = (t >> 3) + 32 * i;
-    *reinterpret_cast<uint4*>(dst + (int64_t)r * ld + 16 * j) = *code_chunk(codes, r, j);
-  }
-}
-
 // ---------------------------------------------------------- activations ---
-// Column pass: thread (wc, rg) owns columns 2wc, 2wc+1 and rows 32rg..+31 of
-// the shared bf16 tile; quantizes them with the column blocks' scales into
-// the swizzled code tile (row = column index, bytes = token index).
-template <int MODE, typename S>
-__device__ __forceinline__ void act_column_pass(S& sm, uint32_t (*tile)[64], float* s_col) {
-  const int tid = threadIdx.x;
-  const int wc = tid & 63, rg = tid >> 6;
-  uint32_t wv[32];
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    wv[i] = tile[rg * 32 + i][wc];
-    m = umax2(m, wv[i] & kAbsMask);
-  }
-  sm.colmax[rg][wc] = m;
-  __syncthreads();
-  m = umax2(umax2(sm.colmax[0][wc], sm.colmax[1][wc]), umax2(sm.colmax[2][wc], sm.colmax[3][wc]));
-  const Divisor d0 = make_divisor<MODE>(__uint_as_float((m & 0xFFFFu) << 16));
-  const Divisor d1 = make_divisor<MODE>(__uint_as_float(m & 0xFFFF0000u));
-  if (rg == 0) *reinterpret_cast<float2*>(s_col + 2 * wc) = make_float2(d0.s, d1.s);
-  const float2 s2 = make_float2(d0.s, d1.s), y2 = make_float2(d0.y, d1.y);
-  uint32_t c0[8], c1[8];
-  if (MODE == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d0.exact || d1.exact)) {
-    const ColCodes c = column_codes_exact(tile, wc, rg, d0, d1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c0[i] = c.c0[i];
-      c1[i] = c.c1[i];
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float2 q[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t w = wv[4 * i + u];
-        q[u] = div2<MODE>(make_float2(bf16lo(w), bf16hi(w)), s2, y2);
-      }
-      c0[i] = cvt_e4m3x2(q[0].x, q[1].x) | (cvt_e4m3x2(q[2].x, q[3].x) << 16);
-      c1[i] = cvt_e4m3x2(q[0].y, q[1].y) | (cvt_e4m3x2(q[2].y, q[3].y) << 16);
-    }
-  }
-  __syncthreads();  // every thread is done with the bf16 tile; reuse it for codes
-  uint32_t* codes = &tile[0][0];
-  *code_chunk(codes, 2 * wc, 2 * rg) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
-  *code_chunk(codes, 2 * wc, 2 * rg + 1) = make_uint4(c0[4], c0[5], c0[6], c0[7]);
-  *code_chunk(codes, 2 * wc + 1, 2 * rg) = make_uint4(c1[0], c1[1], c1[2], c1[3]);
-  *code_chunk(codes, 2 * wc + 1, 2 * rg + 1) = make_uint4(c1[4], c1[5], c1[6], c1[7]);
-}
-
-// Persistent activation quantizer: each CTA walks tiles t = blockIdx.x +
-// i*gridDim.x (column tile fastest).  One thread TMA-loads tile i+1 into the
-// other half of a double buffer while all threads work on tile i, so every
-// SM keeps about 32 KB of loads in flight per resident CTA.
+// A 128x128 bf16 tile sits in shared memory as two boxes of 64 columns
+// (128 rows x 128 bytes each) with the TMA's 128-byte swizzle: 16-byte chunk
+// j of row r is stored at chunk j ^ (r & 7).
 struct ActSmem {
-  uint32_t buf[2][128][64];  // bf16 tiles (256-byte rows); a finished tile's
-                             // buffer then holds its transposed codes
-  uint32_t colmax[4][64];
-  float srow[128];
+  uint8_t buf[2][2][128 * 128];  // [buffer][box][row * 128 + byte], 1024-aligned
+  uint32_t colmax[2][4][64];     // partial column maxima, by tile parity
   uint64_t full[2];
 };
 
-__device__ __forceinline__ void issue_tile(ActSmem& sm, const CUtensorMap* tm, int t, int nK, int b) {
-  const uint32_t bar = smem_u32(&sm.full[b]);
-  mbar_arrive_expect_tx(bar, 128 * 256);
-  tma_load_2d(smem_u32(&sm.buf[b][0][0]), tm, bar, (t % nK) * 128, (t / nK) * 128);
+__device__ __forceinline__ uint32_t act_off(int box, int r, int chunk) {
+  return (uint32_t)(box * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4));
 }
 
+__device__ __forceinline__ void issue_tile(ActSmem& sm, const CUtensorMap* tm, int t, int nK, int b) {
+  const uint32_t bar = smem_u32(&sm.full[b]);
+  const int k0 = (t % nK) * 128, m0 = (t / nK) * 128;
+  mbar_arrive_expect_tx(bar, 128 * 256);
+  tma_load_2d(smem_u32(&sm.buf[b][0][0]), tm, bar, k0, m0);
+  tma_load_2d(smem_u32(&sm.buf[b][1][0]), tm, bar, k0 + 64, m0);
+}
+
+// Persistent activation quantizer: CTA c walks tiles t = c + i*gridDim.x
+// (column tile fastest), with tiles i+1 and i+2 in flight while tile i is
+// processed.  Per tile and thread:
+//   row pass     thread (row rr, half hh) reads its 64 columns (8 conflict-
+//                free 16-byte loads), takes the row amax with its partner
+//                lane (lane ^ 8 holds the other half), and writes 64 codes
+//                and, for hh = 0, the row scale;
+//   column pass  thread (column pair wc, row group rg) reads 32 rows of its
+//                two columns, posts the partial maxima; after the tile's one
+//                barrier it combines the four row groups, quantizes and
+//                writes 2 x 32 codes and, for rg = 0, the column scales.
 template <int MODE, bool COL>
 __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUtensorMap tmX,
                                                      int64_t M, int64_t K,
@@ -253,11 +197,12 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
                                                      uint8_t* __restrict__ q_col,
                                                      float* __restrict__ s_col) {
   extern __shared__ uint8_t smem_raw[];
-  ActSmem& sm = *reinterpret_cast<ActSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                            ~uintptr_t(127));
+  ActSmem& sm = *reinterpret_cast<ActSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
   const int tid = threadIdx.x;
-  const int r16 = tid >> 4, vec = tid & 15;
-  const int lane = tid & 31, half_base = lane & 16;
+  const int rr = (tid & 7) + 8 * (tid >> 4), hh = (tid >> 3) & 1;  // row pass
+  const int wc = tid & 63, rg = tid >> 6;                            // column pass
+  const int cbox = wc >> 5, cchunk = (wc & 31) >> 2, cword = wc & 3;
   const int nK = (int)(K / 128);
   const int tiles = nK * (int)(M / 128);
   if (tid == 0) {
@@ -267,58 +212,87 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
     prefetch_tmap(&tmX);
   }
   __syncthreads();
-  if (tid == 0 && (int)blockIdx.x < tiles) issue_tile(sm, &tmX, blockIdx.x, nK, 0);
+  if (tid == 0) {
+    if ((int)blockIdx.x < tiles) issue_tile(sm, &tmX, blockIdx.x, nK, 0);
+    if ((int)(blockIdx.x + gridDim.x) < tiles) issue_tile(sm, &tmX, blockIdx.x + gridDim.x, nK, 1);
+  }
   int i = 0;
   for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
     const int cur = i & 1;
     const int64_t k0 = (int64_t)(t % nK) * 128, m0 = (int64_t)(t / nK) * 128;
-    if (tid == 0 && t + (int)gridDim.x < tiles) {
-      fence_proxy_async_smem();  // generic accesses to the other buffer are done
-      issue_tile(sm, &tmX, t + gridDim.x, nK, cur ^ 1);
-    }
     if (!mbar_wait(smem_u32(&sm.full[cur]), (i >> 1) & 1)) return;  // bounded: never expected
-    uint32_t (*tile)[64] = sm.buf[cur];
-    uint4 v[8];
+    const uint8_t* tb = &sm.buf[cur][0][0];
+
+    // ---- row pass
+    {
+      uint4 v[8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) v[p] = *reinterpret_cast<const uint4*>(&tile[p * 16 + r16][vec * 4]);
-    // Row amaxes of the 8 rows this half-warp touches (reduced over 16 lanes).
-    uint32_t m[8];
+      for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(tb + act_off(hh, rr, j));
+      uint32_t m = absmax8(v[0]);
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      m[p] = absmax8(v[p]);
-      m[p] = umax2(m[p], __shfl_xor_sync(0xffffffffu, m[p], 8));
-      m[p] = umax2(m[p], __shfl_xor_sync(0xffffffffu, m[p], 4));
-      m[p] = umax2(m[p], __shfl_xor_sync(0xffffffffu, m[p], 2));
-      m[p] = umax2(m[p], __shfl_xor_sync(0xffffffffu, m[p], 1));
+      for (int j = 1; j < 8; ++j) m = umax2(m, absmax8(v[j]));
+      m = umax2(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      const Divisor d = make_divisor<MODE>(halves_max(m));
+      if (hh == 0) s_row[(k0 / 128) * M + m0 + rr] = d.s;
+      uint8_t* qr = q_row + (m0 + rr) * K + k0 + hh * 64;
+#pragma unroll
+      for (int j = 0; j < 8; j += 4) {
+        const uint2 c0 = quant8<MODE>(v[j], d), c1 = quant8<MODE>(v[j + 1], d);
+        const uint2 c2 = quant8<MODE>(v[j + 2], d), c3 = quant8<MODE>(v[j + 3], d);
+        st_global_v8(qr + 8 * j, make_uint4(c0.x, c0.y, c1.x, c1.y), make_uint4(c2.x, c2.y, c3.x, c3.y));
+      }
     }
-    // One divisor per lane instead of one per row per lane: lane L of each
-    // half-warp prepares the divisor of pass L & 7; the others fetch it by
-    // shuffle.
-    uint32_t mine = m[0];
-#pragma unroll
-    for (int p = 1; p < 8; ++p) mine = ((lane & 7) == p) ? m[p] : mine;
-    const Divisor dl = make_divisor<MODE>(halves_max(mine));
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      const int row = p * 16 + r16;
-      Divisor d;
-      d.s = __shfl_sync(0xffffffffu, dl.s, half_base + p);
-      d.y = __shfl_sync(0xffffffffu, dl.y, half_base + p);
-      d.exact = MODE == FP8BW_SCALE_FP32 && !(halves_max(m[p]) >= 0x1p-80f);
-      *reinterpret_cast<uint2*>(q_row + (m0 + row) * K + k0 + vec * 8) = quant8<MODE>(v[p], d);
-      if (vec == 0) sm.srow[row] = d.s;
-    }
+
+    // ---- column pass, part 1: the words and the partial maxima
+    ColWords cw;
     if (COL) {
-      // the row pass only read the tile: no barrier needed before the column pass
-      act_column_pass<MODE>(sm, tile, s_col + (m0 / 128) * K + k0);
+      uint32_t m = 0;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        cw.w[r] = *reinterpret_cast<const uint32_t*>(tb + act_off(cbox, rg * 32 + r, cchunk) + 4 * cword);
+        m = umax2(m, cw.w[r] & kAbsMask);
+      }
+      sm.colmax[cur][rg][wc] = m;
     }
+    // Partial maxima complete; every thread is done reading this buffer, so
+    // it may take the tile after next.
     __syncthreads();
-    if (tid < 32)
-      *reinterpret_cast<float4*>(s_row + (k0 / 128) * M + m0 + 4 * tid) =
-          *reinterpret_cast<const float4*>(&sm.srow[4 * tid]);
-    if (COL) store_code_tile(tile, q_col + k0 * M + m0, M);
-    fence_proxy_async_smem();
-    __syncthreads();  // this buffer may now be refilled by the next TMA load
+    if (tid == 0 && t + 2 * (int)gridDim.x < tiles) issue_tile(sm, &tmX, t + 2 * gridDim.x, nK, cur);
+
+    // ---- column pass, part 2
+    if (COL) {
+      const uint32_t m = umax2(umax2(sm.colmax[cur][0][wc], sm.colmax[cur][1][wc]),
+                               umax2(sm.colmax[cur][2][wc], sm.colmax[cur][3][wc]));
+      const Divisor d0 = make_divisor<MODE>(__uint_as_float((m & 0xFFFFu) << 16));
+      const Divisor d1 = make_divisor<MODE>(__uint_as_float(m & 0xFFFF0000u));
+      if (rg == 0)
+        *reinterpret_cast<float2*>(s_col + (m0 / 128) * K + k0 + 2 * wc) = make_float2(d0.s, d1.s);
+      uint32_t c0[8], c1[8];
+      if (MODE == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d0.exact || d1.exact)) {
+        const ColCodes c = column_codes_exact(cw, d0, d1);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c0[j] = c.c0[j];
+          c1[j] = c.c1[j];
+        }
+      } else {
+        const float2 s2 = make_float2(d0.s, d1.s), y2 = make_float2(d0.y, d1.y);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float2 q[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t w = cw.w[4 * j + u];
+            q[u] = div2<MODE>(make_float2(bf16lo(w), bf16hi(w)), s2, y2);
+          }
+          c0[j] = cvt_e4m3x2(q[0].x, q[1].x) | (cvt_e4m3x2(q[2].x, q[3].x) << 16);
+          c1[j] = cvt_e4m3x2(q[0].y, q[1].y) | (cvt_e4m3x2(q[2].y, q[3].y) << 16);
+        }
+      }
+      uint8_t* qc = q_col + (k0 + 2 * wc) * M + m0 + rg * 32;
+      st_global_v8(qc, make_uint4(c0[0], c0[1], c0[2], c0[3]), make_uint4(c0[4], c0[5], c0[6], c0[7]));
+      st_global_v8(qc + M, make_uint4(c1[0], c1[1], c1[2], c1[3]), make_uint4(c1[4], c1[5], c1[6], c1[7]));
+    }
   }
 }
 
@@ -434,12 +408,12 @@ cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, i
                              int num_sms, cudaStream_t st) {
   CUtensorMap tm;
   if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)K, (uint64_t)M,
-                (uint64_t)ldx, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                (uint64_t)ldx, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int64_t tiles = (K / 128) * (M / 128);
   const int per_sm = 3;
   const unsigned grid = (unsigned)(tiles < (int64_t)num_sms * per_sm ? tiles : (int64_t)num_sms * per_sm);
-  const size_t smem = sizeof(ActSmem) + 128;
+  const size_t smem = sizeof(ActSmem) + 1024;
   const bool col = q_col != nullptr;
   cudaError_t e = cudaSuccess;
 #define FP8BW_QA(MD, CL)                                                                      \

@@ -5,9 +5,10 @@
  * s = RN(amax / 448).  The quantizer needs RN(x / s) for every bf16 x of the
  * block (|x| <= amax).  Instead of one division per element it takes the
  * reciprocal y = RN(1 / s) once and applies one Markstein correction step
- * (P. Markstein, IBM J. Res. Dev. 34(1), 1990):
- *     q0 = RN(x * y);  r = fma(-q0, s, x);  q = fma(r, y, q0)
- * then copies the sign of x onto q.  Blocks with amax < 2^-80 divide.
+ * (P. Markstein, IBM J. Res. Dev. 34(1), 1990) in its sign-symmetric form:
+ *     q0 = RN(x * y);  r = fma(q0, s, -x);  q = fma(r, -y, q0)
+ * (the same arithmetic as r = x - q0*s, q = q0 + r*y, up to the sign of an
+ * exact zero, so that x = -0 gives q = -0).  Blocks with amax < 2^-80 divide.
  *
  * Claim checked here, over every positive finite bf16 amax >= 2^-80 and every
  * bf16 x (both signs) with |x| <= amax:
@@ -38,9 +39,8 @@ int main(void) {
         const float x = from_bf16(xb | (neg ? 0x8000u : 0u));
         const float ref = x / s;
         const float q0 = x * y;
-        const float r = fmaf(-q0, s, x);
-        float q = fmaf(r, y, q0);
-        q = copysignf(q, x);
+        const float r = fmaf(q0, s, -x);
+        const float q = fmaf(r, -y, q0);
         ++pairs;
         if (bits(q) != bits(ref) && (fabsf(ref) >= 0x1p-12f || fabsf(q) >= 0x1p-12f)) ++bad;
         if ((bits(q) ^ bits(ref)) & 0x80000000u) ++badsign;
