@@ -459,49 +459,68 @@ def main():
         d2h = sum(a.numel() * 2 + b.numel() * 2 + c.numel() * 2 for a, b, c in host_out)
 
         # Copies overlap the compute: host->device on one stream, device->host
-        # on another, the layers in order on the compute stream; a step's
-        # uploads start once the previous step's compute has finished.
+        # on another, the layers in order on the compute stream.  The device
+        # inputs and outputs are double-buffered across steps, so that step
+        # k+1's uploads run while step k computes and step k's downloads run
+        # while step k+1 computes.
         comp = torch.cuda.current_stream()
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        bufs = [[(l.X, l.W, l.dY, l.Y, l.dX, l.dW) for l in layers],
+                [tuple(torch.empty_like(t) for t in (l.X, l.W, l.dY, l.Y, l.dX, l.dW)) for l in layers]]
+        in_free = [None, None]   # compute of the step that last read this input set is done
+        out_free = [None, None]  # downloads of the step that last wrote this output set are done
 
-        def e2e_step():
-            s_in.wait_stream(comp)
+        def e2e_step(k):
+            b = k & 1
+            dev_set = bufs[b]
+            if in_free[b] is not None:
+                s_in.wait_event(in_free[b])
             with torch.cuda.stream(s_in):
-                for l, (x, w, d) in zip(layers, host_in):
-                    l.W.copy_(w, non_blocking=True)
+                for (x, w, d), (X, W, dY, _, _, _) in zip(host_in, dev_set):
+                    W.copy_(w, non_blocking=True)
                 ev_w = torch.cuda.Event()
                 ev_w.record(s_in)
                 ev_in = []
-                for l, (x, w, d) in zip(layers, host_in):
-                    l.X.copy_(x, non_blocking=True)
-                    l.dY.copy_(d, non_blocking=True)
+                for (x, w, d), (X, W, dY, _, _, _) in zip(host_in, dev_set):
+                    X.copy_(x, non_blocking=True)
+                    dY.copy_(d, non_blocking=True)
                     ev_in.append(torch.cuda.Event())
                     ev_in[-1].record(s_in)
             comp.wait_event(ev_w)
-            fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT) for l in layers], mode)
-            for i, l in enumerate(layers):
+            fb.fp8bw_requant_weights([(W, l.qw, l.sw, l.qwT) for l, (_, W, _, _, _, _) in zip(layers, dev_set)],
+                                     mode)
+            if out_free[b] is not None:
+                comp.wait_event(out_free[b])
+            for i, (l, (X, W, dY, Y, dX, dW)) in enumerate(zip(layers, dev_set)):
                 comp.wait_event(ev_in[i])
-                fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)
-                fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode)
-                fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)
-                fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode)
-                fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode)
+                fb.fp8bw_quant_act_1x128(X, mode, l.qx, l.sx, l.qxc, l.sxc)
+                fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, Y, mode)
+                fb.fp8bw_quant_act_1x128(dY, mode, l.qd, l.sd, l.qdc, l.sdc)
+                fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, dX, mode)
+                fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, dW, mode)
                 ev = torch.cuda.Event()
                 ev.record(comp)
                 s_out.wait_event(ev)
                 with torch.cuda.stream(s_out):
-                    a, b, c = host_out[i]
-                    a.copy_(l.Y, non_blocking=True)
-                    b.copy_(l.dX, non_blocking=True)
-                    c.copy_(l.dW, non_blocking=True)
-            comp.wait_stream(s_out)
-        e2e_step()
+                    a, bb, c = host_out[i]
+                    a.copy_(Y, non_blocking=True)
+                    bb.copy_(dX, non_blocking=True)
+                    c.copy_(dW, non_blocking=True)
+            in_free[b] = torch.cuda.Event()
+            in_free[b].record(comp)
+            out_free[b] = torch.cuda.Event()
+            out_free[b].record(s_out)
+
+        e2e_step(0)
+        e2e_step(1)
         torch.cuda.synchronize()
         barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        s_in.wait_stream(comp)
+        for k in range(args.e2e_steps):
+            e2e_step(k)
+        comp.wait_stream(s_out)
         e.record()
         torch.cuda.synchronize()
         e_ms = s.elapsed_time(e)
