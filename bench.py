@@ -49,8 +49,12 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--case", default=None,
                    help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
-                        "requant|bf16_fprop, on --layer")
+                        "requant|bf16_fprop on --layer at --tokens, requant_sweep (32 layers), or "
+                        "moe_fprop|moe_dgrad|moe_wgrad "
+                        "on the MoE expert layer --layer gate_up|down")
     p.add_argument("--layer", default="gate_up", choices=[n for n, _, _ in workloads.LLAMA8B_LAYERS])
+    p.add_argument("--tokens", type=int, default=workloads.LLAMA8B_TOKENS,
+                   help="tokens of the --case layer (32768 = the packed long-sequence batch)")
     return p.parse_args()
 
 
@@ -302,6 +306,39 @@ def reference_arm(args):
 
 
 # ---------------------------------------------------------- one case -----
+MOE_LAYERS = {"gate_up": (workloads.MOE_HIDDEN, 2 * workloads.MOE_INTER),
+              "down": (workloads.MOE_INTER, workloads.MOE_HIDDEN)}
+
+
+def moe_calls(fb, mode, layer):
+    """Grouped GEMMs of one Qwen3-30B-A3B-like expert layer (128 experts,
+    top-8 of 16384 tokens, Zipf(1.1) routing, segments padded to 128).
+    FLOPs count the routed tokens (16384 * 8), not the padding rows."""
+    dev = torch.device("cuda", 0)
+    K, N = MOE_LAYERS[layer]
+    r = workloads.moe_routing(0)
+    G, Mt = len(r.counts), r.m_total_pad
+    X = workloads.moe_permuted(r, K, 1.0, 11, dev)
+    dY = workloads.moe_permuted(r, N, 1e-3, 12, dev)
+    W = workloads.moe_experts(G, N, K, 13, dev)
+    u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+    e = lambda *sh, dt=u8: torch.empty(sh, dtype=dt, device=dev)  # noqa: E731
+    qx, sx, qxc, sxc = e(Mt, K), e(K // 128, Mt, dt=f32), e(K, Mt), e(Mt // 128, K, dt=f32)
+    qd, sd, qdc, sdc = e(Mt, N), e(N // 128, Mt, dt=f32), e(N, Mt), e(Mt // 128, N, dt=f32)
+    qw, sw, qwT = e(G, N, K), e(G, N // 128, K // 128, dt=f32), e(G, K, N)
+    fb.fp8bw_quant_act_1x128(X, mode, qx, sx, qxc, sxc)
+    fb.fp8bw_quant_act_1x128(dY, mode, qd, sd, qdc, sdc)
+    fb.fp8bw_requant_weights([(W[g], qw[g], sw[g], qwT[g]) for g in range(G)], mode)
+    off = torch.tensor(r.offsets, dtype=torch.int32, device=dev)
+    Y, dX, dW = e(Mt, N, dt=bf), e(Mt, K, dt=bf), e(G, N, K, dt=bf)
+    flops = 2 * workloads.MOE_TOKENS * workloads.MOE_TOPK * N * K
+    return {
+        "moe_fprop": (lambda: fb.fp8bw_grouped_gemm(fb.FP8BW_FPROP, off, qx, sx, qw, sw, Y, mode), flops, "TFLOP/s"),
+        "moe_dgrad": (lambda: fb.fp8bw_grouped_gemm(fb.FP8BW_DGRAD, off, qd, sd, qwT, sw, dX, mode), flops, "TFLOP/s"),
+        "moe_wgrad": (lambda: fb.fp8bw_grouped_gemm(fb.FP8BW_WGRAD, off, qdc, sdc, qxc, sxc, dW, mode), flops, "TFLOP/s"),
+    }
+
+
 def run_case(args):
     """Times a single call of one layer (used for ncu captures and sweeps)."""
     import blockwise_scaled_fp8_fp8bw_b200 as fb
@@ -309,8 +346,25 @@ def run_case(args):
     fb.fp8bw_init(0)
     mode = fb.FP8BW_SCALE_POW2 if args.mode == "pow2" else fb.FP8BW_SCALE_FP32
     name = args.layer
+    if args.case.startswith("moe_"):
+        fn, work, unit = moe_calls(fb, mode, name)[args.case]
+        time_call(fb, args, name, mode, fn, work, unit)
+        return
+    if args.case == "requant_sweep":
+        # the per-step requant of 32 layers x 4 weights (about 7B parameters)
+        dev = torch.device("cuda", 0)
+        items, nbytes = [], 0
+        for layer in range(32):
+            for (n, K, N) in workloads.LLAMA8B_LAYERS:
+                w = workloads.llama_weight(n, layer, device=dev)
+                items.append((w, torch.empty((N, K), dtype=torch.uint8, device=dev),
+                              torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev),
+                              torch.empty((K, N), dtype=torch.uint8, device=dev)))
+                nbytes += N * K * 4 + 4 * (N // 128) * (K // 128)
+        time_call(fb, args, "all", mode, lambda: fb.fp8bw_requant_weights(items, mode), nbytes, "GB/s")
+        return
     K, N = [(k, n) for nm, k, n in workloads.LLAMA8B_LAYERS if nm == name][0]
-    l = Layer(name, K, N, workloads.LLAMA8B_TOKENS, torch.device("cuda", 0))
+    l = Layer(name, K, N, args.tokens, torch.device("cuda", 0))
     fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode)
     fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)
     fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)
@@ -324,6 +378,10 @@ def run_case(args):
         "bf16_fprop": (lambda: fb.fp8bw_gemm_bf16(l.X, l.W, l.Y), l.flops / 3, "TFLOP/s"),
     }
     fn, work, unit = calls[args.case]
+    time_call(fb, args, name, mode, fn, work, unit)
+
+
+def time_call(fb, args, name, mode, fn, work, unit):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -336,7 +394,8 @@ def run_case(args):
     assert fb.fp8bw_last_device_error() == 0
     ms = s.elapsed_time(e) / max(args.steps, 1)
     rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
-    print(json.dumps({"case": args.case, "layer": name, "mode": args.mode, "ms": ms, unit: rate}), flush=True)
+    print(json.dumps({"case": args.case, "layer": name, "tokens": args.tokens, "mode": args.mode, "ms": ms,
+                      unit: rate}), flush=True)
 
 
 # --------------------------------------------------------------- main -----
