@@ -398,6 +398,23 @@ def time_call(fb, args, name, mode, fn, work, unit):
                       unit: rate}), flush=True)
 
 
+# ------------------------------------------------------------ ranks -------
+def max_over_ranks(x: float, dist, device) -> float:
+    """The job's time is its slowest rank's: the maximum of x over all ranks
+    (x itself when there is one rank)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed
+    `units_per_rank` units, the slowest of them in `ms` milliseconds."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # --------------------------------------------------------------- main -----
 def main():
     args = parse()
@@ -458,13 +475,10 @@ def main():
     st = fb.fp8bw_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error: {fb.status_string(st)}")
-    if dist:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
     step_flops = sum(l.flops for l in layers)
-    value = step_flops * args.steps * world / (ms_total * 1e-3) / 1e12
+    value = job_rate(step_flops * args.steps, world, ms_total) / 1e12
 
     def kind_ms(k):
         return sum(s.elapsed_time(e) for s, e in ev[k])
@@ -494,14 +508,11 @@ def main():
         p1.record()
         torch.cuda.synchronize()
         p_ms = p0.elapsed_time(p1)
-        if dist:
-            t = torch.tensor([p_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            p_ms = float(t.item())
+        p_ms = max_over_ranks(p_ms, dist, dev)
         st = fb.fp8bw_last_device_error()
         if st != 0:
             raise RuntimeError(f"device error (pow2): {fb.status_string(st)}")
-        pow2 = {"value": step_flops * args.steps * world / (p_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        pow2 = {"value": job_rate(step_flops * args.steps, world, p_ms) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": p_ms / args.steps,
                 "note": "same step with power-of-2 scales (GEMMs on the block-scaled MMA)"}
 
@@ -583,11 +594,8 @@ def main():
         e.record()
         torch.cuda.synchronize()
         e_ms = s.elapsed_time(e)
-        if dist:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": step_flops * args.e2e_steps * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, dist, dev)
+        e2e = {"value": job_rate(step_flops * args.e2e_steps, world, e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms / args.e2e_steps}
 
