@@ -49,7 +49,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--case", default=None,
                    help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
-                        "requant|bf16_fprop on --layer at --tokens, requant_sweep (32 layers), or "
+                        "requant|bf16_fprop|wgrad_acc on --layer at --tokens, requant_sweep (32 layers), or "
                         "moe_fprop|moe_dgrad|moe_wgrad "
                         "on the MoE expert layer --layer gate_up|down")
     p.add_argument("--layer", default="gate_up", choices=[n for n, _, _ in workloads.LLAMA8B_LAYERS])
@@ -377,6 +377,10 @@ def run_case(args):
         "requant": (lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode), l.weight_bytes, "GB/s"),
         "bf16_fprop": (lambda: fb.fp8bw_gemm_bf16(l.X, l.W, l.Y), l.flops / 3, "TFLOP/s"),
     }
+    if args.case == "wgrad_acc":   # wgrad added into an fp32 main gradient
+        main_grad = torch.zeros((N, K), dtype=torch.float32, device=l.X.device)
+        calls["wgrad_acc"] = (lambda: fb.fp8bw_gemm_f32(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, main_grad,
+                                                        accumulate=True, mode=mode), l.flops / 3, "TFLOP/s")
     fn, work, unit = calls[args.case]
     time_call(fb, args, name, mode, fn, work, unit)
 

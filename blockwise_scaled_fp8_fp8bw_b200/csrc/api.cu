@@ -17,7 +17,7 @@ cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cuda
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M,
                             int64_t N, int64_t K, const uint8_t* A, const float* sA,
                             const uint8_t* B, const float* sB, void* D, int64_t ldd, int mode,
-                            int num_sms, cudaStream_t st);
+                            int num_sms, cudaStream_t st, int out_mode);
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
@@ -176,7 +176,30 @@ FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, in
   if (M == 0 || N == 0) return FP8BW_OK;
   if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
   return from_cuda(fp8bw::launch_gemm_fp8(kind, false, 0, nullptr, M, N, K, A, sA, B, sB, D, ldd,
-                                          mode, sms, reinterpret_cast<cudaStream_t>(stream)));
+                                          mode, sms, reinterpret_cast<cudaStream_t>(stream), 0));
+}
+
+FP8BW_API fp8bw_status fp8bw_gemm_f32(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                            const uint8_t* A, const float* sA, const uint8_t* B,
+                            const float* sB, float* D, int64_t ldd, int32_t accumulate,
+                            fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  if (kind != FP8BW_FPROP && kind != FP8BW_DGRAD && kind != FP8BW_WGRAD) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return FP8BW_ERR_INVALID_ARG;
+  if (!A || !sA || !B || !sB || !D) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(N) || !mult128(K) || (ldd & 3) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sA) || !aligned16(sB))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (M == 0 || N == 0) return FP8BW_OK;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return accumulate ? FP8BW_OK : from_cuda(cudaMemset2DAsync(D, ldd * 4, 0, N * 4, M, cs));
+  return from_cuda(fp8bw::launch_gemm_fp8(kind, false, 0, nullptr, M, N, K, A, sA, B, sB, D, ldd,
+                                          mode, sms, cs, accumulate ? 2 : 1));
 }
 
 FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
@@ -202,12 +225,12 @@ FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const
     // GEMM sizes: rows = N (out), cols = K (in), contraction = tokens.
     if (N == 0 || K == 0) return FP8BW_OK;
     return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, N, K, M_total_pad, A, sA, B,
-                                            sB, D, K, mode, sms, cs));
+                                            sB, D, K, mode, sms, cs, 0));
   }
   if (M_total_pad == 0 || N == 0) return FP8BW_OK;
   if (K == 0) return FP8BW_ERR_INVALID_ARG;
   return from_cuda(fp8bw::launch_gemm_fp8(kind, true, G, d_offsets, M_total_pad, N, K, A, sA, B,
-                                          sB, D, N, mode, sms, cs));
+                                          sB, D, N, mode, sms, cs, 0));
 }
 
 FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,

@@ -51,7 +51,10 @@ constexpr int kScaleStages = 8;
 constexpr uint32_t kATile = BM * BK;  // 16 KB: one CTA's A rows
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = FP8BW_MAX_EXPERTS;
-constexpr uint32_t kEpiPiece = 2048;  // 32 rows x 32 bf16: one TMA store
+constexpr uint32_t kEpiPiece = 2048;  // 32 rows x 32 bf16 (or 16 fp32): one TMA store
+
+// Output of the FP8 GEMMs: bf16 (the default), fp32, or fp32 added to D.
+enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F32_ADD = 2 };
 
 template <bool PAIR>
 struct Cfg {
@@ -93,6 +96,7 @@ struct GemmArgs {
   int G;
   uint16_t* D;         // BF16 kernel only (the FP8 kernel stores through a tensor map)
   int64_t ldd;
+  int out_mode;        // OutMode of the FP8 kernels' epilogue
   int stall_chunk;     // testing: CTA 0's producer never fills this chunk (-1: off)
 };
 
@@ -149,6 +153,38 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
     }
   }
   return ti;
+}
+
+// fp32 output pieces are 32 rows x 16 columns (64-byte rows, 64-byte
+// swizzle: 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)).
+// Row-per-lane accumulators (32x32b TMEM shape): a[j] = columns 2j, 2j+1.
+__device__ __forceinline__ void stage_rows_f32(uint8_t* epi, int lane, const float2* a) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<float4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) =
+        make_float4(a[2 * c].x, a[2 * c].y, a[2 * c + 1].x, a[2 * c + 1].y);
+}
+
+// Accumulators of the 16x256b shape (wgrad promotion): acc[16 i + g] holds
+// row 8i + lane/4 and columns 8g + 2(lane%4) + {0, 1}; piece pp covers the
+// column groups g = 2pp, 2pp + 1.
+__device__ __forceinline__ void stage_quad_f32(uint8_t* epi, int lane, const float2* acc, int pp) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 8 * i + (lane >> 2);
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int chunk = 2 * gg + ((lane & 3) >> 1);
+      *reinterpret_cast<float2*>(epi + row * 64 + 16 * (chunk ^ ((row >> 1) & 3)) + 8 * (lane & 1)) =
+          acc[16 * i + 2 * pp + gg];
+    }
+  }
+}
+
+// Writes (or adds) one staged fp32 piece.
+__device__ __forceinline__ void emit_f32(const CUtensorMap* tmD, uint32_t src, int x, int y, int out_mode) {
+  if (out_mode == OUT_F32_ADD) tma_reduce_add_2d(tmD, src, x, y);
+  else tma_store_2d(tmD, src, x, y);
 }
 
 __device__ __forceinline__ void raise_timeout(Bars* bars) {
@@ -470,6 +506,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pieces (rows / columns outside the output are clipped by the TMA).
       const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
       // (a pair's second CTA past the last row of M computed nothing real)
+      if (a.out_mode != OUT_BF16) {
+        // fp32 output: eight 32x16 pieces per warp, stored or added to D
+#pragma unroll
+        for (int pp = 0; pp < 8 && row0 < a.M; ++pp) {
+          uint8_t* epi = epi0 + (pp % C::kEpiBufs) * kEpiPiece;
+          if (lane == 0) {
+            if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
+          }
+          __syncwarp();
+          if (KIND == FP8BW_WGRAD) stage_quad_f32(epi, lane, acc, pp);
+          else stage_rows_f32(epi, lane, &acc[8 * pp]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            emit_f32(&tmD, smem_u32(epi), col0 + 16 * pp, drow, a.out_mode);
+            bulk_commit();
+          }
+        }
+        if (bars->abort) break;
+        continue;
+      }
 #pragma unroll
       for (int p = 0; p < 4 && row0 < a.M; ++p) {
         uint8_t* epi = epi0 + (p % C::kEpiBufs) * kEpiPiece;
@@ -931,6 +988,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tphase ^= 1;
       }
       const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
+      if (a.out_mode != OUT_BF16) {
+#pragma unroll
+        for (int pp = 0; pp < 8 && row0 < a.M; ++pp) {
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          stage_rows_f32(epi, lane, &acc[8 * pp]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            emit_f32(&tmD, smem_u32(epi), col0 + 16 * pp, drow, a.out_mode);
+            bulk_commit();
+          }
+        }
+        if (bars->abort) break;
+        continue;
+      }
 #pragma unroll
       for (int p = 0; p < 4 && row0 < a.M; ++p) {
         if (lane == 0) bulk_wait_read0();
@@ -1184,7 +1257,7 @@ int gemm_stall_chunk = -1;  // testing hook, consumed by the next FP8 GEMM launc
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
                             const float* sB, void* D, int64_t ldd, int mode, int num_sms,
-                            cudaStream_t st) {
+                            cudaStream_t st, int out_mode) {
   // CTA pairs everywhere except grouped fprop/dgrad (128-row expert segments)
   const bool pair = !(grouped && kind != FP8BW_WGRAD);
   GemmArgs a = {};
@@ -1199,6 +1272,7 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   a.offsets = d_off;
   a.G = G;
   a.stall_chunk = gemm_stall_chunk;
+  a.out_mode = out_mode;
   gemm_stall_chunk = -1;
   if (grouped && kind == FP8BW_WGRAD) a.tiles = G * a.m_tiles * a.n_tiles;
   else a.tiles = a.m_tiles * a.n_tiles;
@@ -1211,8 +1285,9 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
                 CU_TENSOR_MAP_SWIZZLE_128B, b3 ? (uint64_t)G : 0))
     return cudaErrorInvalidValue;
   const uint64_t drows = (grouped && kind == FP8BW_WGRAD) ? (uint64_t)G * M : (uint64_t)M;
-  if (!make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, drows, ldd, 32, 32,
-                CU_TENSOR_MAP_SWIZZLE_64B))
+  const bool f32 = out_mode != OUT_BF16;
+  if (!make_map(&td, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                f32 ? 4 : 2, D, N, drows, ldd, f32 ? 16 : 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   int grid;
   cudaError_t e;

@@ -162,6 +162,23 @@ FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, in
                         const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                         void* D, int64_t ldd, fp8bw_scale_mode mode, fp8bw_stream_t stream);
 
+/* The same GEMM with an fp32 output, for the weight gradient's fp32 main
+ * gradient of mixed-precision training (the optimizer step after which the
+ * weights are requantized, "Leistungsgewinne in der Praxis", keeps fp32
+ * master state):
+ *   accumulate = 0:  D[m][n]  = sum_kb sA(m,kb) sB(n,kb) sum_k A[m][k] B[n][k]
+ *   accumulate = 1:  D[m][n] += the same sum (one fp32 rounding of the add,
+ *                    done in L2; no bf16 rounding anywhere)
+ * Operands, kinds and scale layouts as in fp8bw_gemm.  D [M][ldd] fp32,
+ * 16-byte aligned, ldd >= N and a multiple of 4 (16-byte rows).  The
+ * result is within |D - ref| <= 1e-2 * sum_k |a_k b_k| + 2^-22 |ref| of the
+ * fp64 reference (plus the prior D when accumulating).  Calls on one stream
+ * accumulate in order; no two calls may write the same D concurrently. */
+FP8BW_API fp8bw_status fp8bw_gemm_f32(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                            const uint8_t* A, const float* sA, const uint8_t* B,
+                            const float* sB, float* D, int64_t ldd, int32_t accumulate,
+                            fp8bw_scale_mode mode, fp8bw_stream_t stream);
+
 /* Grouped GEMM for mixture-of-experts layers ("Leistungsgewinne in der
  * Praxis": the recipe also trains the Qwen3-30B MoE model).  Tokens are
  * grouped by expert: expert g owns rows [off[g], off[g+1]) of the permuted

@@ -227,3 +227,21 @@ def check_tol(y_bits, yref, yabs, rel=REL_TOL):
     worst = np.zeros(1, np.float64)
     bad = lib().orc_check_tol(_p(y), _p(yref), _p(yabs), y.size, rel, _p(worst))
     return int(bad), float(worst[0])
+
+
+# fp32-output acceptance: the GEMM gate with the bf16 output ulp replaced by
+# 2^-22 |y_ref| (two fp32 roundings: the result and, when accumulating, the add)
+F32_ABS_REL = 2.0 ** -22
+
+
+def check_tol_f32(y, yref, yabs, rel=REL_TOL):
+    """|y - y_ref| <= rel * yabs + 2^-22 |y_ref| elementwise (NaN fails).
+    Returns (violations, worst error/allowance ratio)."""
+    y = np.asarray(y, np.float64).ravel()
+    yref = np.asarray(yref, np.float64).ravel()
+    lim = rel * np.asarray(yabs, np.float64).ravel() + F32_ABS_REL * np.abs(yref)
+    err = np.abs(y - yref)
+    ok = err <= lim
+    ratio = np.where(lim > 0, err / np.where(lim > 0, lim, 1.0), np.where(err > 0, np.inf, 0.0))
+    worst = float(np.max(np.where(np.isnan(ratio), np.inf, ratio))) if ratio.size else 0.0
+    return int(np.count_nonzero(~ok)), worst

@@ -159,3 +159,37 @@ def test_requant_sweep(fb, orc):
         torch.cuda.synchronize()
         assert torch.equal(q, outs[i][0]) and torch.equal(qT, outs[i][2])
         assert torch.equal(s.view(torch.int32), outs[i][1].view(torch.int32))
+
+
+def test_wgrad_accumulates_into_fp32_main_grad(fb, orc):
+    """Gradient accumulation over two micro-batches of the down layer
+    (8192 tokens each, 14336 -> 4096): dW of each is added to an fp32 main
+    gradient by fp8bw_gemm_f32(accumulate); sampled 32x32 tiles are checked
+    against main_grad0 + the fp64 references of both micro-batches."""
+    name, K, N = workloads.LLAMA8B_LAYERS[3]
+    M = workloads.LLAMA8B_TOKENS
+    rng = np.random.default_rng(77)
+    main = torch.randn((N, K), generator=torch.Generator(device=DEV).manual_seed(5), device=DEV) * 1e-2
+    main0 = main.cpu().numpy().astype(np.float64)
+    ops = []
+    for mb in range(2):
+        X, _, dY = workloads.llama_layer(name, seed=10 + mb, device=DEV, M=M)
+        qx, sx, qxc, sxc = act_buffers(M, K, DEV)
+        qd, sd, qdc, sdc = act_buffers(M, N, DEV)
+        fb.fp8bw_quant_act_1x128(X, 0, qx, sx, qxc, sxc)
+        fb.fp8bw_quant_act_1x128(dY, 0, qd, sd, qdc, sdc)
+        fb.fp8bw_gemm_f32(2, qdc, sdc, qxc, sxc, main, accumulate=True)
+        ops.append((qdc, sdc, qxc, sxc))
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    got = main.cpu().numpy()
+    host = [tuple(np_u8(t) if t.dtype == torch.uint8 else t.cpu().numpy() for t in o) for o in ops]
+    for (m0, n0) in gemm_points(rng, N, K, 8):
+        ref = main0[m0:m0 + 32, n0:n0 + 32].copy()
+        yabs = np.zeros((32, 32))
+        for A, sA, B, sB in host:
+            y, ya = orc.gemm_ref_tile(2, A, sA, B, sB, m0, m0 + 32, n0, n0 + 32)
+            ref += y
+            yabs += ya
+        bad, worst = orc.check_tol_f32(got[m0:m0 + 32, n0:n0 + 32], ref, yabs)
+        assert bad == 0, (m0, n0, worst)

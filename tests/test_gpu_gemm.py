@@ -187,3 +187,42 @@ def test_pow2_mode_rejects_other_scales(fb, orc):
     D = torch.zeros((128, 256), dtype=torch.bfloat16, device=DEV)
     fb.fp8bw_gemm(0, dev(A), dev(sA), dev(B), dev(sB), D, 1)
     assert fb.fp8bw_last_device_error() == 6
+
+
+def pow2_scales(ops):
+    """The same operands with every scale rounded to a power of two."""
+    A, sA, B, sB = ops
+    r = lambda s: (2.0 ** np.round(np.log2(s))).astype(np.float32)  # noqa: E731
+    return A, r(sA), B, r(sB)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_gemm_f32_store_and_accumulate(fb, orc, kind, mode):
+    """fp32 output (fp8bw_gemm_f32): a plain store into a strided buffer
+    (columns past N untouched), then two accumulations onto a prior D, as for
+    two micro-batches into an fp32 main gradient.  384 x 640 x 384: pair tiles
+    with a ragged 128-row tail and a 128-column tail."""
+    rng = np.random.default_rng(100 + 3 * kind + mode)
+    M, N, K = 384, 640, 384
+    ops = rand_ops(rng, M, N, K, kind)
+    if mode == 1:
+        ops = pow2_scales(ops)
+    yr, ya = orc.gemm_ref_tile(kind, *ops, 0, M, 0, N)
+    A, sA, B, sB = (dev(x) for x in ops)
+    Dbig = torch.full((M, N + 64), float("nan"), dtype=torch.float32, device=DEV)
+    D = Dbig[:, :N]
+    fb.fp8bw_gemm_f32(kind, A, sA, B, sB, D, accumulate=False, mode=mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    bad, worst = orc.check_tol_f32(D.cpu().numpy(), yr, ya)
+    assert bad == 0, worst
+    assert torch.isnan(Dbig[:, N:]).all()
+    D0 = (rng.standard_normal((M, N)) * np.abs(yr).mean()).astype(np.float32)
+    Dacc = dev(D0)
+    for _ in range(2):
+        fb.fp8bw_gemm_f32(kind, A, sA, B, sB, Dacc, accumulate=True, mode=mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    bad, worst = orc.check_tol_f32(Dacc.cpu().numpy(), D0.astype(np.float64) + 2 * yr, 2 * ya)
+    assert bad == 0, worst

@@ -311,3 +311,17 @@ def test_check_tol_and_mimic(orc):
     qx2[:, 128:256] = 0
     y2, _ = orc.gemm_ref_tile(0, qx2, sx, qw, sw, 0, 128, 0, 128)
     assert orc.check_tol(to_bits(y2), y, ya)[0] > 100
+
+
+def test_check_tol_f32(orc):
+    """The fp32-output gate: exact values and errors up to the allowance pass,
+    anything beyond it (or NaN) fails."""
+    yref = np.array([1.0, -3.0, 0.0, 1e-3])
+    yabs = np.array([2.0, 3.0, 0.0, 1e-3])
+    lim = orc.REL_TOL * yabs + orc.F32_ABS_REL * np.abs(yref)
+    assert orc.check_tol_f32(yref, yref, yabs)[0] == 0
+    assert orc.check_tol_f32(yref + 0.99 * lim, yref, yabs)[0] == 0
+    bad, worst = orc.check_tol_f32(yref + 1.01 * lim * np.array([1, 0, 0, 1]), yref, yabs)
+    assert bad == 2 and worst > 1.0
+    assert orc.check_tol_f32(np.array([np.nan, -3.0, 0.0, 1e-3]), yref, yabs)[0] == 1
+    assert orc.check_tol_f32(np.array([1.0, -3.0, 1e-30, 1e-3]), yref, yabs)[0] == 1  # zero allowance
