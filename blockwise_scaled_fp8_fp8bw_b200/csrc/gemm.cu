@@ -104,31 +104,61 @@ template <bool PAIR>
 constexpr size_t smem_fp8() {
   return 1024 + size_t(Cfg<PAIR>::kStages) * Cfg<PAIR>::kStageBytes +
          size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * Cfg<PAIR>::kEpiBytes + sizeof(Bars) +
-         sizeof(int32_t) * (kMaxGroups + 1);
+         2 * sizeof(int32_t) * (kMaxGroups + 1);
 }
 static_assert(smem_fp8<true>() <= 232448 && smem_fp8<false>() <= 232448, "shared memory budget");
 
 struct TileInfo {
   int mt, nt, g, kb0, kb1;
+  int m0;    // first row of the tile (of the pair's 256 rows for a pair)
+  int mend;  // rows at or past mend are not part of the result
   bool skip;
 };
 
-// Tile t -> (m tile, n tile, expert, K-chunk range).  M tiles are 256 rows
+// Tile t -> (rows, n tile, expert, K-chunk range).  M tiles are 256 rows
 // for a pair, 128 otherwise; dense tiles go in bands of `band` M tiles so
-// that the CTAs running at once share A and B panels in L2.
-template <int KIND, bool GROUPED>
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off) {
+// that the CTAs running at once share A and B panels in L2.  Grouped
+// fprop/dgrad tiles are pair tiles inside one expert: expert g's rows
+// [off[g], off[g+1]) form ceil(rows/256) of them (pp[g] = those of the
+// experts before g); in the last one the second CTA's 128 rows may lie past
+// the segment, and that CTA then writes nothing.
+template <int KIND, bool GROUPED, bool PAIR>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off,
+                                                const int32_t* pp) {
   TileInfo ti;
   ti.g = 0;
   ti.skip = false;
+  ti.mend = a.M;
   if (GROUPED && KIND == FP8BW_WGRAD) {
     const int per = a.m_tiles * a.n_tiles;
     ti.g = t / per;
     const int r = t - ti.g * per;
     ti.mt = r % a.m_tiles;
     ti.nt = r / a.m_tiles;
+    ti.m0 = ti.mt * (PAIR ? 2 * BM : BM);
     ti.kb0 = off[ti.g] >> 7;
     ti.kb1 = off[ti.g + 1] >> 7;
+    return ti;
+  }
+  ti.kb0 = 0;
+  ti.kb1 = a.K / BK;
+  if (GROUPED && PAIR) {
+    const int pt = t / a.n_tiles;
+    ti.nt = t - pt * a.n_tiles;
+    ti.mt = pt;
+    if (pt >= pp[a.G]) {
+      ti.skip = true;
+      ti.m0 = 0;
+      return ti;
+    }
+    int lo = 0, hi = a.G - 1;  // last g with pp[g] <= pt (an expert that owns pt)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pp[mid] <= pt) lo = mid; else hi = mid - 1;
+    }
+    ti.g = lo;
+    ti.m0 = off[lo] + (pt - pp[lo]) * (2 * BM);
+    ti.mend = off[lo + 1];
     return ti;
   }
   const int band_tiles = a.band * a.n_tiles;
@@ -137,8 +167,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
   const int rows = min(a.band, a.m_tiles - band * a.band);
   ti.mt = band * a.band + r % rows;
   ti.nt = r / rows;
-  ti.kb0 = 0;
-  ti.kb1 = a.K / BK;
+  ti.m0 = ti.mt * (PAIR ? 2 * BM : BM);
   if (GROUPED) {
     const int row0 = ti.mt * BM;
     if (row0 >= off[a.G]) {
@@ -150,9 +179,33 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
         if (off[mid] <= row0) lo = mid; else hi = mid - 1;
       }
       ti.g = lo;
+      ti.mend = off[lo + 1];
     }
   }
   return ti;
+}
+
+// Pair tiles per expert for grouped fprop/dgrad: pp[g+1] = pp[g] +
+// ceil((off[g+1] - off[g]) / 256), scanned by warp 0 (32 experts a round).
+// Every thread of the CTA must call it.
+__device__ __forceinline__ void pair_prefix(const int32_t* off, int32_t* pp, int G) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int v = g < G ? (off[g + 1] - off[g] + 2 * BM - 1) / (2 * BM) : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += u;
+      }
+      if (g < G) pp[g + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) pp[0] = 0;
+  }
+  __syncthreads();
 }
 
 // fp32 output pieces are 32 rows x 16 columns (64-byte rows, 64-byte
@@ -198,7 +251,7 @@ __device__ __forceinline__ void raise_timeout_mx(B* bars) {
   atomicExch(&bars->abort, 1);
 }
 
-template <int KIND, bool GROUPED, bool PAIR>
+template <int KIND, bool GROUPED, bool PAIR, bool F32OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
@@ -211,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(epi_base + 8 * C::kEpiBytes);
   Bars* bars = reinterpret_cast<Bars*>(slots + kScaleStages);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
+  int32_t* s_pp = s_off + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0;
@@ -272,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return;
     }
+    if (KIND != FP8BW_WGRAD && PAIR) pair_prefix(s_off, s_pp, a.G);
   }
   const uint32_t tmem = bars->tmem_base;
   // Barriers the MMA waits on live in the first CTA of a pair.
@@ -289,9 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
         if (ti.skip) continue;
-        const int arow = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++chunk) {
           if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
@@ -304,7 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (PAIR) {
               if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[stage]), 2 * C::kStageBytes);
               tma_load_2d_pair(sa, &tmA, full, kb * BK, arow);
-              tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
+              if (GROUPED && KIND != FP8BW_WGRAD)
+                tma_load_3d_pair(sa + kATile, &tmB, full, kb * BK, brow, ti.g);
+              else
+                tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
             } else {
               mbar_arrive_expect_tx(full, C::kStageBytes);
               tma_load_2d(sa, &tmA, full, kb * BK, arow);
@@ -325,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
-          const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
           if (ti.skip) continue;
           for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
             if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1) ||
@@ -361,9 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sphase = 0;
       const int nKb = a.K / BK, nNb = a.N / 128;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
         if (ti.skip) continue;
-        const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const bool rows_ok = row0 < a.M;
         const float* sBg = a.sB;
         if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
@@ -407,9 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
       if (ti.skip) continue;
-      const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+      const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
       float2 acc[64];
 #pragma unroll
@@ -505,11 +563,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: bf16 rows through shared memory, TMA stores of 32x32
       // pieces (rows / columns outside the output are clipped by the TMA).
       const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
-      // (a pair's second CTA past the last row of M computed nothing real)
-      if (a.out_mode != OUT_BF16) {
+      // (a pair's second CTA past the last row of M, or of the expert's
+      // segment, computed nothing real)
+      if (row0 >= ti.mend) {
+        // nothing of this CTA's rows is part of the result
+      } else if (F32OUT) {
         // fp32 output: eight 32x16 pieces per warp, stored or added to D
 #pragma unroll
-        for (int pp = 0; pp < 8 && row0 < a.M; ++pp) {
+        for (int pp = 0; pp < 8; ++pp) {
           uint8_t* epi = epi0 + (pp % C::kEpiBufs) * kEpiPiece;
           if (lane == 0) {
             if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
@@ -524,11 +585,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit();
           }
         }
-        if (bars->abort) break;
-        continue;
-      }
+      } else {
 #pragma unroll
-      for (int p = 0; p < 4 && row0 < a.M; ++p) {
+      for (int p = 0; p < 4; ++p) {
         uint8_t* epi = epi0 + (p % C::kEpiBufs) * kEpiPiece;
         // the store that last used this staging piece has read it
         if (lane == 0) {
@@ -567,6 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_2d(&tmD, smem_u32(epi), col0 + p * 32, drow);
           bulk_commit();
         }
+      }
       }
       if (bars->abort) break;
     }
@@ -617,7 +677,7 @@ constexpr int kMxMaxStages = 6;
 template <bool PAIR>
 struct MxCfg {
   static constexpr uint32_t kStageBytes = kATile + (PAIR ? (BN / 2) * BK : BN * BK);
-  static constexpr int kStages = PAIR ? 5 : 4;
+  static constexpr int kStages = PAIR ? 5 : 3;  // (single-CTA tiles: not launched)
   static constexpr uint32_t kIdescM = PAIR ? 2 * BM : BM;
 };
 
@@ -638,7 +698,7 @@ template <bool PAIR>
 constexpr size_t smem_mx() {
   return 1024 + size_t(MxCfg<PAIR>::kStages) * MxCfg<PAIR>::kStageBytes + 8 * kEpiPiece +
          size_t(kMxRaw) * sizeof(ScaleSlot) + size_t(kSfSlots) * sizeof(SfSlot) +
-         sizeof(MxBars) + sizeof(int32_t) * (kMaxGroups + 1);
+         sizeof(MxBars) + 2 * sizeof(int32_t) * (kMaxGroups + 1);
 }
 static_assert(smem_mx<true>() <= 232448 && smem_mx<false>() <= 232448, "shared memory budget (MX)");
 
@@ -683,7 +743,7 @@ __device__ __forceinline__ void sf_convert(const ScaleSlot* const* r, int n, SfS
   *reinterpret_cast<uint4*>(&o->b[1][lane][0]) = make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
 }
 
-template <int KIND, bool GROUPED, bool PAIR>
+template <int KIND, bool GROUPED, bool PAIR, bool F32OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
@@ -697,6 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   SfSlot* sf = reinterpret_cast<SfSlot*>(raw + kMxRaw);
   MxBars* bars = reinterpret_cast<MxBars*>(sf + kSfSlots);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
+  int32_t* s_pp = s_off + (kMaxGroups + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0;
   const bool leader = rank == 0;
@@ -752,6 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return;
     }
+    if (KIND != FP8BW_WGRAD && PAIR) pair_prefix(s_off, s_pp, a.G);
   }
   const uint32_t tmem = bars->tmem_base;
   // Barriers the MMA waits on live in the first CTA of a pair.
@@ -770,9 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
         if (ti.skip) continue;
-        const int arow = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++chunk) {
           if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
@@ -785,7 +847,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (PAIR) {
               if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[stage]), 2 * C::kStageBytes);
               tma_load_2d_pair(sa, &tmA, full, kb * BK, arow);
-              tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
+              if (GROUPED && KIND != FP8BW_WGRAD)
+                tma_load_3d_pair(sa + kATile, &tmB, full, kb * BK, brow, ti.g);
+              else
+                tma_load_2d_pair(sa + kATile, &tmB, full, kb * BK, brow);
             } else {
               mbar_arrive_expect_tx(full, C::kStageBytes);
               tma_load_2d(sa, &tmA, full, kb * BK, arow);
@@ -806,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, gslot = 0;
         uint32_t phase = 0, tphase = 0, gphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
-          const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
           if (ti.skip || ti.kb0 == ti.kb1) continue;
           if (!mbar_wait(smem_u32(&bars->tempty), tphase ^ 1)) {
             raise_timeout_mx(bars);
@@ -879,10 +944,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool have = t < a.tiles;
         TileInfo ti = {};
         if (have) {
-          ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+          ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
           if (ti.skip) continue;
         }
-        const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+        const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const float* sBg = a.sB;
         if (GROUPED && KIND != FP8BW_WGRAD) sBg += (size_t)ti.g * nNb * nKb;
         for (int kg = ti.kb0; have ? kg < ti.kb1 : pend; kg += kSfGroup) {
@@ -952,9 +1017,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* epi = epi_base + (warp - 4) * kEpiPiece;
     uint32_t tphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED>(a, t, s_off);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
       if (ti.skip) continue;
-      const int row0 = PAIR ? (ti.mt * 2 + (int)rank) * BM : ti.mt * BM;
+      const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
       float2 acc[64];
       if (ti.kb0 == ti.kb1) {
@@ -988,9 +1053,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tphase ^= 1;
       }
       const int drow = (GROUPED && KIND == FP8BW_WGRAD ? ti.g * a.M : 0) + row0 + q * 32;
-      if (a.out_mode != OUT_BF16) {
+      if (F32OUT) {
 #pragma unroll
-        for (int pp = 0; pp < 8 && row0 < a.M; ++pp) {
+        for (int pp = 0; pp < 8 && row0 < ti.mend; ++pp) {
           if (lane == 0) bulk_wait_read0();
           __syncwarp();
           stage_rows_f32(epi, lane, &acc[8 * pp]);
@@ -1005,7 +1070,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 #pragma unroll
-      for (int p = 0; p < 4 && row0 < a.M; ++p) {
+      for (int p = 0; p < 4 && row0 < ti.mend; ++p) {
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
 #pragma unroll
@@ -1086,7 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false>(a, t, nullptr);
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr);
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
           raise_timeout(bars);
@@ -1142,7 +1207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false>(a, t, nullptr);
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr);
       if (!mbar_wait(smem_u32(&bars->tfull[buf]), bphase)) {
         raise_timeout(bars);
         goto done;
@@ -1201,10 +1266,10 @@ cudaError_t prepare(K kernel, size_t smem, bool check_regs) {
   return cudaSuccess;
 }
 
-template <int KIND, bool GROUPED, bool PAIR>
+template <int KIND, bool GROUPED, bool PAIR, bool F32OUT = false>
 cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                        const GemmArgs& a, int grid, cudaStream_t st) {
-  auto kern = k_gemm_fp8<KIND, GROUPED, PAIR>;
+  auto kern = k_gemm_fp8<KIND, GROUPED, PAIR, F32OUT>;
   const size_t smem = smem_fp8<PAIR>();
   cudaError_t e = prepare(kern, smem, true);
   if (e != cudaSuccess) return e;
@@ -1225,10 +1290,10 @@ cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
 }
 
-template <int KIND, bool GROUPED, bool PAIR>
+template <int KIND, bool GROUPED, bool PAIR, bool F32OUT = false>
 cudaError_t launch_mx(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                       const GemmArgs& a, int grid, cudaStream_t st) {
-  auto kern = k_gemm_mx<KIND, GROUPED, PAIR>;
+  auto kern = k_gemm_mx<KIND, GROUPED, PAIR, F32OUT>;
   const size_t smem = smem_mx<PAIR>();
   cudaError_t e = prepare(kern, smem, true);
   if (e != cudaSuccess) return e;
@@ -1258,13 +1323,16 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
                             const float* sB, void* D, int64_t ldd, int mode, int num_sms,
                             cudaStream_t st, int out_mode) {
-  // CTA pairs everywhere except grouped fprop/dgrad (128-row expert segments)
-  const bool pair = !(grouped && kind != FP8BW_WGRAD);
+  // CTA pairs everywhere; grouped fprop/dgrad pair tiles stay inside one
+  // expert, so their number is only bounded here (sum of ceil(rows_g/256)
+  // <= (M/128 + G)/2) and the kernel skips the tiles past the real count.
+  const bool pair = true;
   GemmArgs a = {};
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
-  a.m_tiles = (int)(pair ? (M + 2 * BM - 1) / (2 * BM) : M / BM);
+  if (grouped && kind != FP8BW_WGRAD) a.m_tiles = (int)((M / BM + G + 1) / 2);
+  else a.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
   a.n_tiles = (int)((N + BN - 1) / BN);
   a.band = pair ? (gemm_band_rows + 1) / 2 : gemm_band_rows;
   a.sA = sA;
@@ -1297,14 +1365,28 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   } else {
     grid = a.tiles < num_sms ? a.tiles : num_sms;
   }
+  if (f32) {  // fp32 output: dense GEMMs only
+    if (grouped) return cudaErrorInvalidValue;
+    if (mode == FP8BW_SCALE_POW2) {
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false, true, true>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false, true, true>(ta, tb, td, a, grid, st);
+      else e = launch_mx<FP8BW_WGRAD, false, true, true>(ta, tb, td, a, grid, st);
+    } else {
+      if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true, true>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true, true>(ta, tb, td, a, grid, st);
+      else e = launch_one<FP8BW_WGRAD, false, true, true>(ta, tb, td, a, grid, st);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (mode == FP8BW_SCALE_POW2) {
     if (!grouped) {
       if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false, true>(ta, tb, td, a, grid, st);
       else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false, true>(ta, tb, td, a, grid, st);
       else e = launch_mx<FP8BW_WGRAD, false, true>(ta, tb, td, a, grid, st);
     } else {
-      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, true, false>(ta, tb, td, a, grid, st);
-      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, true, false>(ta, tb, td, a, grid, st);
+      if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, true, true>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, true, true>(ta, tb, td, a, grid, st);
       else e = launch_mx<FP8BW_WGRAD, true, true>(ta, tb, td, a, grid, st);
     }
     if (e != cudaSuccess) return e;
@@ -1315,8 +1397,8 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
     else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true>(ta, tb, td, a, grid, st);
     else e = launch_one<FP8BW_WGRAD, false, true>(ta, tb, td, a, grid, st);
   } else {
-    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, true, false>(ta, tb, td, a, grid, st);
-    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, true, false>(ta, tb, td, a, grid, st);
+    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, true, true>(ta, tb, td, a, grid, st);
+    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, true, true>(ta, tb, td, a, grid, st);
     else e = launch_one<FP8BW_WGRAD, true, true>(ta, tb, td, a, grid, st);
   }
   if (e != cudaSuccess) return e;
