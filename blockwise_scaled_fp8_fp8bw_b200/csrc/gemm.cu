@@ -10,8 +10,8 @@
 // FP8 kernel (persistent, 384 threads per CTA, one CTA per SM).  Output tile
 // 256x256 per CTA pair (PAIR: a 2-CTA cluster, tcgen05 cta_group::2, M=256
 // split over the two SMs, each SM holding its own 128 A rows and half of the
-// 256 B rows) or 128x256 per CTA (grouped fprop/dgrad, whose 128-row expert
-// segments cannot share a 256-row tile).  Roles per CTA:
+// 256 B rows); grouped fprop/dgrad pair tiles stay inside one expert (see
+// decode_tile).  Roles per CTA:
 //   warp 0      TMA producer: per 128-wide K chunk, the CTA's 128x128 A tile
 //               and its B tile (128 or 256 rows) into a shared-memory ring
 //               (E4M3, 128-byte swizzle).  In a pair both CTAs count their
@@ -649,8 +649,7 @@ done:
 // (tcgen05.mma.kind::mxf8f6f4.block_scale): each 128-wide scale block is one
 // UE8M0 byte replicated over its four 32-element MMA blocks, and the whole K
 // loop accumulates in one TMEM accumulator with no promotion.
-// Tiles as in the promotion kernel: 256x256 per CTA pair (cta_group::2) for
-// dense GEMMs and grouped wgrad, 128x256 per CTA for grouped fprop/dgrad.
+// Tiles as in the promotion kernel: 256x256 per CTA pair (cta_group::2).
 // 384 threads per CTA:
 //   warp 0      TMA producer
 //   warp 1      MMA issuer (first CTA of a pair): per chunk, tcgen05.cp of
