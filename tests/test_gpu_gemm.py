@@ -128,6 +128,26 @@ def test_ldd(fb, orc):
     assert torch.all(Dbig[:, :128] == 0) and torch.all(Dbig[:, 384:] == 0)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_ldd_16_byte_rows(fb, orc, kind, mode):
+    """Rows of D only 16-byte aligned (ldd = N + 8) and a 128-column tail
+    (N = 384 is not a multiple of the 256-wide tile): nothing outside the
+    N columns is written."""
+    rng = np.random.default_rng(40 + kind + 3 * mode)
+    M, N, K = 256, 384, 256
+    ops = rand_ops(rng, M, N, K, kind)
+    if mode == 1:
+        ops = pow2_scales(ops)
+    Dbig = torch.full((M, N + 8), float("nan"), dtype=torch.bfloat16, device=DEV)
+    D = Dbig[:, :N]
+    fb.fp8bw_gemm(kind, *(dev(x) for x in ops), D, mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    check(orc, bits(D), kind, *ops)
+    assert torch.isnan(Dbig[:, N:].float()).all()
+
+
 @pytest.mark.parametrize("MNK", [(256, 512, 512), (128, 384, 256)])
 def test_bf16_gemm(fb, orc, MNK):
     M, N, K = MNK
