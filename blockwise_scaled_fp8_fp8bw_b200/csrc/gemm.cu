@@ -124,7 +124,7 @@ struct TileInfo {
 // the segment, and that CTA then writes nothing.
 template <int KIND, bool GROUPED, bool PAIR>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off,
-                                                const int32_t* pp) {
+                                                const int32_t* pp, int& hint) {
   TileInfo ti;
   ti.g = 0;
   ti.skip = false;
@@ -151,14 +151,16 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
       ti.m0 = 0;
       return ti;
     }
-    int lo = 0, hi = a.G - 1;  // last g with pp[g] <= pt (an expert that owns pt)
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pp[mid] <= pt) lo = mid; else hi = mid - 1;
-    }
-    ti.g = lo;
-    ti.m0 = off[lo] + (pt - pp[lo]) * (2 * BM);
-    ti.mend = off[lo + 1];
+    // The expert that owns pt: the last g with pp[g] <= pt.  A role visits
+    // its tiles in increasing order, so the search walks forward from the
+    // expert of its previous tile (`hint`): one or two dependent shared
+    // loads per tile instead of a full binary search.
+    int g = hint;
+    while (g + 1 < a.G && pp[g + 1] <= pt) ++g;
+    hint = g;
+    ti.g = g;
+    ti.m0 = off[g] + (pt - pp[g]) * (2 * BM);
+    ti.mend = off[g + 1];
     return ti;
   }
   const int band_tiles = a.band * a.n_tiles;
@@ -271,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int cta_slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile-loop index
   const int cta_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  int ghint = 0;  // expert of this thread's previous tile (grouped fprop/dgrad)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -344,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
-          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
           if (ti.skip) continue;
           for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
             if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1) ||
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sphase = 0;
       const int nKb = a.K / BK, nNb = a.N / 128;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const bool rows_ok = row0 < a.M;
@@ -465,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
       if (ti.skip) continue;
       const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
@@ -762,6 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int cta_slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int cta_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  int ghint = 0;  // expert of this thread's previous tile (grouped fprop/dgrad)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -831,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
@@ -870,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, gslot = 0;
         uint32_t phase = 0, tphase = 0, gphase = 0;
         for (int t = cta_slot; t < a.tiles; t += cta_step) {
-          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+          const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
           if (ti.skip || ti.kb0 == ti.kb1) continue;
           if (!mbar_wait(smem_u32(&bars->tempty), tphase ^ 1)) {
             raise_timeout_mx(bars);
@@ -943,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool have = t < a.tiles;
         TileInfo ti = {};
         if (have) {
-          ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+          ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
           if (ti.skip) continue;
         }
         const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
@@ -1016,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* epi = epi_base + (warp - 4) * kEpiPiece;
     uint32_t tphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
       if (ti.skip) continue;
       const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
@@ -1120,6 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int ghint = 0;  // unused by dense tiles
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
@@ -1150,7 +1155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr);
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr, ghint);
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
           raise_timeout(bars);
@@ -1206,7 +1211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr);
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr, ghint);
       if (!mbar_wait(smem_u32(&bars->tfull[buf]), bphase)) {
         raise_timeout(bars);
         goto done;
