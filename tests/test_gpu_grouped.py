@@ -151,3 +151,60 @@ def test_grouped_moe_full_size_sampled(fb, orc):
         y, ya = orc.grouped_gemm_ref_tile(2, offs, A, sA, B, sB, e, nb, nb + 32, kb, kb + 32)
         bad, worst = orc.check_tol(np.ascontiguousarray(bits(dW[e])[nb:nb + 32, kb:kb + 32]), y, ya)
         assert bad == 0, (e, worst)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_grouped_max_experts(fb, orc, mode):
+    """FP8BW_MAX_EXPERTS (512) experts, most of them empty or a single
+    128-row block (the per-expert pair-tile prefix spans 16 rounds of the
+    device scan; odd block counts leave the second CTA of a pair idle)."""
+    rng = np.random.default_rng(17 + mode)
+    G = 512
+    lens = [int(x) for x in rng.choice([0, 0, 1, 100, 130, 300], G)]
+    K, N = 128, 256
+    c = moe_case(orc, 23 + mode, lens, K, N, mode)
+    off, Mtot = c["off"], c["Mtot"]
+    for kind, Nout in [(0, N), (1, K)]:
+        D, ops = run_grouped(fb, kind, c, mode, (Mtot, Nout))
+        y, ya = orc.grouped_gemm_ref_tile(kind, off, *ops, 0, 0, int(off[-1]), 0, Nout)
+        bad, worst = orc.check_tol(bits(D)[:int(off[-1])], y, ya)
+        assert bad == 0, (kind, worst)
+        assert torch.isnan(D[int(off[-1]):].float()).all()
+    D, ops = run_grouped(fb, 2, c, mode, (G, N, K))
+    Dh = bits(D)
+    for e in rng.choice(G, 24, replace=False):
+        y, ya = orc.grouped_gemm_ref_tile(2, off, *ops, int(e), 0, N, 0, K)
+        bad, worst = orc.check_tol(Dh[e], y, ya)
+        assert bad == 0, (int(e), worst)
+        if lens[e] == 0:
+            assert torch.all(D[e] == 0)
+
+
+def test_degenerate_sizes(fb, orc):
+    """K = 0 gives exact zeros (bf16 and fp32 stores) and leaves an fp32
+    accumulator unchanged; M = 0 or N = 0 is a no-op."""
+    p = torch.zeros(128 * 128, dtype=torch.uint8, device=DEV)
+    s = torch.ones(128 * 128, dtype=torch.float32, device=DEV)
+    r = fb.raw
+    D = torch.full((128, 256), 5.0, dtype=torch.bfloat16, device=DEV)
+    assert r.fp8bw_gemm(0, 128, 256, 0, p.data_ptr(), s.data_ptr(), p.data_ptr(), s.data_ptr(),
+                        D.data_ptr(), 256, 0, None) == 0
+    torch.cuda.synchronize()
+    assert torch.all(D == 0)
+    F = torch.full((128, 256), 5.0, dtype=torch.float32, device=DEV)
+    assert r.fp8bw_gemm_f32(2, 128, 256, 0, p.data_ptr(), s.data_ptr(), p.data_ptr(), s.data_ptr(),
+                            F.data_ptr(), 256, 1, 0, None) == 0
+    torch.cuda.synchronize()
+    assert torch.all(F == 5.0)
+    assert r.fp8bw_gemm_f32(2, 128, 256, 0, p.data_ptr(), s.data_ptr(), p.data_ptr(), s.data_ptr(),
+                            F.data_ptr(), 256, 0, 0, None) == 0
+    torch.cuda.synchronize()
+    assert torch.all(F == 0)
+    D.fill_(5.0)
+    assert r.fp8bw_gemm(0, 0, 256, 128, p.data_ptr(), s.data_ptr(), p.data_ptr(), s.data_ptr(),
+                        D.data_ptr(), 256, 0, None) == 0
+    assert r.fp8bw_quant_act_1x128(D.data_ptr(), 0, 128, 128, 0, p.data_ptr(), s.data_ptr(),
+                                   None, None, None) == 0
+    torch.cuda.synchronize()
+    assert torch.all(D == 5.0)
+    assert fb.fp8bw_last_device_error() == 0
