@@ -57,11 +57,13 @@ def _load():
     L.fp8bw_gemm.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, vp, i64, i32, vp]
     L.fp8bw_gemm_f32.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, vp, i64, ctypes.c_int32, i32, vp]
     L.fp8bw_grouped_gemm.argtypes = [i32, ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
+    L.fp8bw_grouped_wgrad_f32.argtypes = [ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp,
+                                          ctypes.c_int32, i32, vp]
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm",
               "fp8bw_quant_act_1x128",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
-              "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_gemm_bf16"):
+              "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16"):
         getattr(L, f).restype = i32
     return L
 
@@ -178,6 +180,16 @@ def fp8bw_grouped_gemm(kind, offsets, A, sA, B, sB, D, mode=FP8BW_SCALE_FP32, st
     _check("fp8bw_grouped_gemm", load().fp8bw_grouped_gemm(
         int(kind), G, _ptr(offsets), Mtot, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(D),
         int(mode), _stream(stream)))
+
+
+def fp8bw_grouped_wgrad_f32(offsets, A, sA, B, sB, D, accumulate=False, mode=FP8BW_SCALE_FP32, stream=None):
+    """offsets device int32 [G+1]; A [N,Mtot], B [K,Mtot]; D [G,N,K] fp32."""
+    G = offsets.numel() - 1
+    N, Mtot = A.shape
+    K = B.shape[0]
+    _check("fp8bw_grouped_wgrad_f32", load().fp8bw_grouped_wgrad_f32(
+        G, _ptr(offsets), Mtot, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(D),
+        int(bool(accumulate)), int(mode), _stream(stream)))
 
 
 def fp8bw_gemm_bf16(A, B, D, stream=None):

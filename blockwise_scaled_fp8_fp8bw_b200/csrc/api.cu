@@ -233,6 +233,32 @@ FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const
                                           sB, D, N, mode, sms, cs, 0));
 }
 
+FP8BW_API fp8bw_status fp8bw_grouped_wgrad_f32(int32_t G, const int32_t* d_offsets,
+                                     int64_t M_total_pad, int64_t N, int64_t K,
+                                     const uint8_t* A, const float* sA, const uint8_t* B,
+                                     const float* sB, float* D, int32_t accumulate,
+                                     fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return FP8BW_ERR_INVALID_ARG;
+  if (!d_offsets || !A || !sA || !B || !sB || !D) return FP8BW_ERR_INVALID_ARG;
+  if (G < 1 || M_total_pad < 0 || N < 0 || K < 0) return FP8BW_ERR_INVALID_ARG;
+  if (G > FP8BW_MAX_EXPERTS) return FP8BW_ERR_TOO_LARGE;
+  if (M_total_pad > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M_total_pad) || !mult128(N) || !mult128(K)) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sA) || !aligned16(sB) ||
+      (reinterpret_cast<uintptr_t>(d_offsets) & 3u))
+    return FP8BW_ERR_ALIGNMENT;
+  if ((int64_t)G * N * K > (int64_t(1) << 40)) return FP8BW_ERR_TOO_LARGE;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (N == 0 || K == 0) return FP8BW_OK;
+  // GEMM sizes: rows = N (out), cols = K (in), contraction = tokens.
+  return from_cuda(fp8bw::launch_gemm_fp8(FP8BW_WGRAD, true, G, d_offsets, N, K, M_total_pad, A, sA,
+                                          B, sB, D, K, mode, sms, reinterpret_cast<cudaStream_t>(stream),
+                                          accumulate ? 2 : 1));
+}
+
 FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,
                              int64_t ldd, fp8bw_stream_t stream) {
   if (!A || !B || !D) return FP8BW_ERR_INVALID_ARG;

@@ -1369,9 +1369,12 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   } else {
     grid = a.tiles < num_sms ? a.tiles : num_sms;
   }
-  if (f32) {  // fp32 output: dense GEMMs only
-    if (grouped) return cudaErrorInvalidValue;
-    if (mode == FP8BW_SCALE_POW2) {
+  if (f32) {  // fp32 output: dense GEMMs and grouped wgrad
+    if (grouped && kind != FP8BW_WGRAD) return cudaErrorInvalidValue;
+    if (grouped) {
+      if (mode == FP8BW_SCALE_POW2) e = launch_mx<FP8BW_WGRAD, true, true, true>(ta, tb, td, a, grid, st);
+      else e = launch_one<FP8BW_WGRAD, true, true, true>(ta, tb, td, a, grid, st);
+    } else if (mode == FP8BW_SCALE_POW2) {
       if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false, true, true>(ta, tb, td, a, grid, st);
       else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false, true, true>(ta, tb, td, a, grid, st);
       else e = launch_mx<FP8BW_WGRAD, false, true, true>(ta, tb, td, a, grid, st);

@@ -202,6 +202,17 @@ FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const
                                 const float* sB, void* D, fp8bw_scale_mode mode,
                                 fp8bw_stream_t stream);
 
+/* Grouped weight gradient with an fp32 output, for mixture-of-experts
+ * layers' fp32 main gradients: operands, offsets and checks as in
+ * fp8bw_grouped_gemm with kind FP8BW_WGRAD; D [G][N][K] fp32 (16-byte
+ * aligned), accumulate as in fp8bw_gemm_f32 (an expert with no tokens adds
+ * zeros, or stores zeros when accumulate = 0). */
+FP8BW_API fp8bw_status fp8bw_grouped_wgrad_f32(int32_t G, const int32_t* d_offsets,
+                                     int64_t M_total_pad, int64_t N, int64_t K,
+                                     const uint8_t* A, const float* sA, const uint8_t* B,
+                                     const float* sB, float* D, int32_t accumulate,
+                                     fp8bw_scale_mode mode, fp8bw_stream_t stream);
+
 /* BF16 GEMM, the comparison path of "Der technische Durchbruch" (FP8 linear
  * layers have twice the BF16 peak): D[m][n] = bf16( sum_k A[m][k] B[n][k] )
  * with FP32 accumulation.  A [M][K], B [N][K] bf16, K-major (dense rows);

@@ -208,3 +208,37 @@ def test_degenerate_sizes(fb, orc):
     torch.cuda.synchronize()
     assert torch.all(D == 5.0)
     assert fb.fp8bw_last_device_error() == 0
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_grouped_wgrad_f32_accumulate(fb, orc, mode):
+    """fp8bw_grouped_wgrad_f32: each expert's weight gradient stored in fp32,
+    then added twice onto a prior fp32 main gradient [G][N][K] (empty experts
+    add zeros)."""
+    lens = [300, 0, 128, 1, 517, 0, 256, 77]
+    K, N = 256, 384
+    c = moe_case(orc, 31 + mode, lens, K, N, mode)
+    off, G = c["off"], c["G"]
+    A, sA, B, sB = c["qdc"], c["sdc"], c["qxc"], c["sxc"]
+    offd = dev(off)
+    Ad, sAd, Bd, sBd = dev(A), dev(sA), dev(B), dev(sB)
+    D = torch.full((G, N, K), float("nan"), dtype=torch.float32, device=DEV)
+    fb.fp8bw_grouped_wgrad_f32(offd, Ad, sAd, Bd, sBd, D, accumulate=False, mode=mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    rng = np.random.default_rng(8)
+    D0 = (rng.standard_normal((G, N, K)) * 1e-3).astype(np.float32)
+    Dacc = dev(D0)
+    for _ in range(2):
+        fb.fp8bw_grouped_wgrad_f32(offd, Ad, sAd, Bd, sBd, Dacc, accumulate=True, mode=mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    Dh, Dacch = D.cpu().numpy(), Dacc.cpu().numpy()
+    for e in range(G):
+        y, ya = orc.grouped_gemm_ref_tile(2, off, A, sA, B, sB, e, 0, N, 0, K)
+        bad, worst = orc.check_tol_f32(Dh[e], y, ya)
+        assert bad == 0, (e, worst)
+        bad, worst = orc.check_tol_f32(Dacch[e], D0[e].astype(np.float64) + 2 * y, 2 * ya)
+        assert bad == 0, (e, worst)
+        if lens[e] == 0:
+            assert np.all(Dh[e] == 0) and np.array_equal(Dacch[e], D0[e])
