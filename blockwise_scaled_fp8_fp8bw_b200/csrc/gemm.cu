@@ -61,7 +61,7 @@ struct Cfg {
   static constexpr uint32_t kBTile = PAIR ? (BN / 2) * BK : BN * BK;  // this CTA's B rows
   static constexpr uint32_t kStageBytes = kATile + kBTile;
   static constexpr int kStages = PAIR ? 5 : 4;
-  static constexpr int kEpiBufs = PAIR ? 2 : 1;  // staging pieces per promotion warp
+  static constexpr int kEpiBufs = PAIR ? 3 : 1;  // staging pieces per promotion warp
   static constexpr uint32_t kEpiBytes = kEpiBufs * kEpiPiece;
   static constexpr uint32_t kIdesc = idesc_make(0, 0, PAIR ? 2 * BM : BM, BN);  // E4M3 -> F32
   static constexpr uint32_t kTemptyCount = PAIR ? 16 : 8;
@@ -576,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int pp = 0; pp < 8; ++pp) {
           uint8_t* epi = epi0 + (pp % C::kEpiBufs) * kEpiPiece;
           if (lane == 0) {
-            if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
+            bulk_wait_read<C::kEpiBufs - 1>();
           }
           __syncwarp();
           if (KIND == FP8BW_WGRAD) stage_quad_f32(epi, lane, acc, pp);
@@ -594,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* epi = epi0 + (p % C::kEpiBufs) * kEpiPiece;
         // the store that last used this staging piece has read it
         if (lane == 0) {
-          if (C::kEpiBufs == 2) bulk_wait_read1(); else bulk_wait_read0();
+          bulk_wait_read<C::kEpiBufs - 1>();
         }
         __syncwarp();
         if (KIND == FP8BW_WGRAD) {
@@ -675,6 +675,7 @@ constexpr int kMxRaw = kSfGroup * kSfSlots;     // raw fp32 chunk slots
 constexpr uint32_t kSfCol0 = 256;               // TMEM: accumulator [0,256), scales after
 constexpr uint32_t kSfCols = 12;                // per group: A 4 columns + B 8 columns
 constexpr int kMxMaxStages = 6;
+constexpr int kMxEpiBufs = 2;                   // staging pieces per epilogue warp
 
 template <bool PAIR>
 struct MxCfg {
@@ -698,7 +699,7 @@ struct SfSlot {
 
 template <bool PAIR>
 constexpr size_t smem_mx() {
-  return 1024 + size_t(MxCfg<PAIR>::kStages) * MxCfg<PAIR>::kStageBytes + 8 * kEpiPiece +
+  return 1024 + size_t(MxCfg<PAIR>::kStages) * MxCfg<PAIR>::kStageBytes + 8 * kMxEpiBufs * kEpiPiece +
          size_t(kMxRaw) * sizeof(ScaleSlot) + size_t(kSfSlots) * sizeof(SfSlot) +
          sizeof(MxBars) + 2 * sizeof(int32_t) * (kMaxGroups + 1);
 }
@@ -755,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + C::kStages * C::kStageBytes;
-  ScaleSlot* raw = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kEpiPiece);
+  ScaleSlot* raw = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kMxEpiBufs * kEpiPiece);
   SfSlot* sf = reinterpret_cast<SfSlot*>(raw + kMxRaw);
   MxBars* bars = reinterpret_cast<MxBars*>(sf + kSfSlots);
   int32_t* s_off = reinterpret_cast<int32_t*>(bars + 1);
@@ -1017,7 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<kRegsHigh>();
     // -------------------------------------------------------- epilogue ---
     const int q = warp & 3, half = (warp - 4) >> 2;
-    uint8_t* epi = epi_base + (warp - 4) * kEpiPiece;
+    uint8_t* epi0 = epi_base + (warp - 4) * kMxEpiBufs * kEpiPiece;
     uint32_t tphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
       const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
@@ -1059,7 +1060,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (F32OUT) {
 #pragma unroll
         for (int pp = 0; pp < 8 && row0 < ti.mend; ++pp) {
-          if (lane == 0) bulk_wait_read0();
+          uint8_t* epi = epi0 + (pp % kMxEpiBufs) * kEpiPiece;
+          if (lane == 0) bulk_wait_read<kMxEpiBufs - 1>();
           __syncwarp();
           stage_rows_f32(epi, lane, &acc[8 * pp]);
           fence_proxy_async_smem();
@@ -1074,7 +1076,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int p = 0; p < 4 && row0 < ti.mend; ++p) {
-        if (lane == 0) bulk_wait_read0();
+        uint8_t* epi = epi0 + (p % kMxEpiBufs) * kEpiPiece;
+        if (lane == 0) bulk_wait_read<kMxEpiBufs - 1>();
         __syncwarp();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
