@@ -18,7 +18,7 @@
 //       precisie": E4M3 has 4 exponent bits, 3 mantissa bits and values up to
 //       +-448.
 //
-// Readings taken where the pages are silent (each is listed in the design doc):
+// Readings taken where the pages are silent:
 //  * block scale s = fp32(amax / 448) (current scaling), s = 1 for an
 //    all-zero block;
 //  * power-of-2 mode: s = 2^e with e the smallest integer such that
