@@ -23,15 +23,19 @@
 //   warp 2      scale loader: the chunk's 128 A-row scales and the B scales
 //               (2 block scales, or 256 column scales for wgrad) into an
 //               8-slot shared ring with cp.async.
-//   warps 4-11  promotion: each thread owns one accumulator row and 128
-//               columns; per chunk it reads the chunk product from TMEM,
-//               multiplies by sA*sB in fp32 and adds it to its registers
-//               (packed f32x2 FMAs), releasing the TMEM buffer as soon as it
-//               is read so the MMA of the next chunk overlaps.  At the end
-//               of a tile the rows are rounded to bf16, staged in shared
-//               memory (64-byte swizzle) and written by TMA stores.
-// Registers: warpgroup 0 drops to 40 per thread, the promotion warpgroups
-// rise to 232 (128 accumulators + 64 staging); 40*128 + 232*256 = 64512 =
+//   warps 4-11  promotion: each warp owns a 32-row quarter of TMEM lanes and
+//               128 columns (fprop/dgrad: a thread per row, 32x32b loads;
+//               wgrad: 4 rows x 32 columns per thread, 16x256b loads, so the
+//               per-column scales need few shared loads); per chunk it reads
+//               the chunk product from TMEM, multiplies by sA*sB in fp32 and
+//               adds it to its registers (packed f32x2 FMAs), releasing the
+//               TMEM buffer as soon as it is read so the MMA of the next
+//               chunk overlaps.  At the end of a tile the results are
+//               rounded to bf16 (or kept fp32), staged in shared memory
+//               (64-byte swizzle, three pieces per warp) and written by TMA
+//               stores (or TMA reduce-adds).
+// Registers: warpgroup 0 drops to 56 per thread, the promotion warpgroups
+// rise to 224 (128 accumulators + 64 staging); 56*128 + 224*256 = 64512 =
 // 384 * 168, the launch allocation (checked on the host before launch).
 // Every wait is bounded; on a timeout the kernel latches an error bit and
 // leaves its loops.
