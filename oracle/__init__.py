@@ -54,6 +54,16 @@ def lib():
         L.orc_e4m3_encode.restype = ctypes.c_uint8
         L.orc_block_scale.argtypes = [flt, i32]
         L.orc_block_scale.restype = flt
+        L.orc_e5m2_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e5m2_decode.restype = dbl
+        L.orc_e5m2_encode.argtypes = [flt]
+        L.orc_e5m2_encode.restype = ctypes.c_uint8
+        L.orc_e5m2_encode_array.argtypes = [vp, i64, vp]
+        L.orc_block_scale_fmt.argtypes = [flt, i32, i32]
+        L.orc_block_scale_fmt.restype = flt
+        L.orc_quant_act_1x128_fmt.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+        L.orc_gemm_ref_tile_fmt.argtypes = [i32, i32, i32, i64, i64, i64, vp, vp, vp, vp,
+                                            i64, i64, i64, i64, vp, vp]
         L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_float.restype = flt
         L.orc_float_to_bf16.argtypes = [flt]
@@ -117,12 +127,37 @@ def block_scale(amax: float, mode: int) -> float:
     return lib().orc_block_scale(float(amax), int(mode))
 
 
+# Element formats: E4M3 (the method's) and E5M2 (the gradient format of the
+# per-tensor recipe, "FP8 Trainingsinfrastructuur", "Het landschap van
+# numerieke precisie").
+FMT_E4M3, FMT_E5M2 = 0, 1
+
+
+def e5m2_decode(code: int) -> float:
+    return lib().orc_e5m2_decode(int(code))
+
+
+def e5m2_encode(v: float) -> int:
+    return int(lib().orc_e5m2_encode(float(v)))
+
+
+def e5m2_encode_array(v: np.ndarray) -> np.ndarray:
+    v = _f32(v)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e5m2_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def block_scale_fmt(amax: float, mode: int, fmt: int) -> float:
+    return lib().orc_block_scale_fmt(float(amax), int(mode), int(fmt))
+
+
 def bf16_ulp(v: float) -> float:
     return lib().orc_bf16_ulp(float(v))
 
 
 # -------------------------------------------------------------- quantizers --
-def quant_act_1x128(x_bits: np.ndarray, mode: int, colwise: bool = True):
+def quant_act_1x128(x_bits: np.ndarray, mode: int, colwise: bool = True, fmt: int = FMT_E4M3):
     """x_bits: uint16 [M, K].  Returns (q_row, s_row, q_col, s_col)."""
     x = _u16(x_bits)
     M, K = x.shape
@@ -130,9 +165,9 @@ def quant_act_1x128(x_bits: np.ndarray, mode: int, colwise: bool = True):
     s_row = np.empty((K // 128, M), np.float32)
     q_col = np.empty((K, M), np.uint8) if colwise else None
     s_col = np.empty((M // 128, K), np.float32) if colwise else None
-    lib().orc_quant_act_1x128(_p(x), M, K, K, mode, _p(q_row), _p(s_row),
-                              _p(q_col) if colwise else None,
-                              _p(s_col) if colwise else None)
+    lib().orc_quant_act_1x128_fmt(_p(x), M, K, K, mode, fmt, _p(q_row), _p(s_row),
+                                  _p(q_col) if colwise else None,
+                                  _p(s_col) if colwise else None)
     return q_row, s_row, q_col, s_col
 
 
@@ -149,15 +184,16 @@ def quant_weight_128x128(w_bits: np.ndarray, mode: int, transposed: bool = True)
 
 
 # ------------------------------------------------------------------- GEMMs --
-def gemm_ref_tile(kind, A, sA, B, sB, m0, m1, n0, n1):
-    """fp64 reference of rows [m0,m1) x cols [n0,n1).  Returns (y, yabs)."""
+def gemm_ref_tile(kind, A, sA, B, sB, m0, m1, n0, n1, fa=FMT_E4M3, fb=FMT_E4M3):
+    """fp64 reference of rows [m0,m1) x cols [n0,n1); fa/fb the element
+    formats of the A and B codes.  Returns (y, yabs)."""
     A, B, sA, sB = _u8(A), _u8(B), _f32(sA), _f32(sB)
     M, K = A.shape
     N = B.shape[0]
     y = np.empty((m1 - m0, n1 - n0), np.float64)
     ya = np.empty_like(y)
-    lib().orc_gemm_ref_tile(kind, M, N, K, _p(A), _p(sA), _p(B), _p(sB),
-                            m0, m1, n0, n1, _p(y), _p(ya))
+    lib().orc_gemm_ref_tile_fmt(kind, fa, fb, M, N, K, _p(A), _p(sA), _p(B), _p(sB),
+                                m0, m1, n0, n1, _p(y), _p(ya))
     return y, ya
 
 

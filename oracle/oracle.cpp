@@ -110,24 +110,80 @@ uint8_t e4m3_encode(float v) {
   return static_cast<uint8_t>(sign | code);
 }
 
+// ---------------------------------------------------------------- E5M2 ----
+// E5M2 ([P2] "Het landschap van numerieke precisie": the gradient format of
+// the per-tensor recipe): sign bit, 5 exponent bits (bias 15), 2 mantissa
+// bits; exponent field 31 holds +-inf (mantissa 0) and NaN; the largest
+// finite value is 1.75 * 2^15 = 57344.
+//   field e in 1..30: (1 + m/4) * 2^(e-15)
+//   field e == 0    : (m/4) * 2^(1-15) = m * 2^-16   (subnormals)
+double e5m2_decode(uint8_t code) {
+  int sign = (code >> 7) & 1;
+  int e = (code >> 2) & 0x1F;
+  int m = code & 0x3;
+  double mag;
+  if (e == 31) {
+    if (m != 0) return std::nan("");
+    mag = INFINITY;
+  } else if (e == 0) {
+    mag = std::ldexp(static_cast<double>(m), -16);
+  } else {
+    mag = std::ldexp(1.0 + m / 4.0, e - 15);
+  }
+  return sign ? -mag : mag;
+}
+
+// Round a finite fp32 value to the E5M2 grid, ties to even, saturating to
+// +-57344 (as the E4M3 encoder: the spacing in [2^E, 2^(E+1)) is 2^(E-2)
+// for E >= -14 and 2^-16 below, and the parity of v / spacing is the parity
+// of the mantissa field).  NaN keeps its sign with code 0x7F.
+uint8_t e5m2_encode(float v) {
+  uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  if (std::isnan(v)) return static_cast<uint8_t>(sign | 0x7F);
+  double a = std::fabs(static_cast<double>(v));
+  if (a >= 57344.0) return static_cast<uint8_t>(sign | 0x7B);  // saturate
+  if (a == 0.0) return sign;
+  int E;
+  std::frexp(a, &E);
+  E -= 1;                          // a in [2^E, 2^(E+1))
+  int spacing_exp = (E < -14) ? -16 : E - 2;
+  double k = std::ldexp(a, -spacing_exp);
+  double r = std::nearbyint(k);    // ties to even
+  //  subnormal range: r * 2^-16, r in 0..4 (r == 4 is 2^-14 = code 4);
+  //  normal range: (r/4) * 2^E, r in 4..8, code (E + 15) * 4 + (r - 4).
+  long r_int = static_cast<long>(r);
+  if (r_int == 0) return sign;
+  long code = (E < -14) ? r_int : (E + 15) * 4 + (r_int - 4);
+  return static_cast<uint8_t>(sign | code);
+}
+
+// Element formats: 0 = E4M3 (largest value 448), 1 = E5M2 (57344).
+constexpr int FMT_E4M3 = 0;
+constexpr int FMT_E5M2 = 1;
+
+double fmt_max(int fmt) { return fmt == FMT_E5M2 ? 57344.0 : 448.0; }
+double decode(uint8_t code, int fmt) { return fmt == FMT_E5M2 ? e5m2_decode(code) : e4m3_decode(code); }
+uint8_t encode(float v, int fmt) { return fmt == FMT_E5M2 ? e5m2_encode(v) : e4m3_encode(v); }
+
 // ------------------------------------------------------------ block scale --
 constexpr int MODE_FP32 = 0;
 constexpr int MODE_POW2 = 1;
 
-float block_scale(float amax, int mode) {
+float block_scale(float amax, int mode, int fmt = FMT_E4M3) {
   if (amax == 0.0f) return 1.0f;
-  if (mode == MODE_FP32) return amax / 448.0f;  // IEEE fp32 division
-  // Power of two: the smallest e with amax <= 448 * 2^e (found by search,
+  const float qmax = static_cast<float>(fmt_max(fmt));
+  if (mode == MODE_FP32) return amax / qmax;  // IEEE fp32 division
+  // Power of two: the smallest e with amax <= qmax * 2^e (found by search,
   // which is the definition), clamped to the UE8M0-representable [-127,127].
   int e = -127;
-  while (e < 127 && static_cast<double>(amax) > std::ldexp(448.0, e)) ++e;
+  while (e < 127 && static_cast<double>(amax) > std::ldexp(static_cast<double>(qmax), e)) ++e;
   return static_cast<float>(std::ldexp(1.0, e));
 }
 
-uint8_t quant_one(uint16_t xb, float s) {
+uint8_t quant_one(uint16_t xb, float s, int fmt = FMT_E4M3) {
   float x = bf16_bits_to_float(xb);
   float t = x / s;  // IEEE fp32 division, round to nearest even
-  return e4m3_encode(t);
+  return encode(t, fmt);
 }
 
 }  // namespace
@@ -136,12 +192,19 @@ extern "C" {
 
 double orc_e4m3_decode(uint8_t code) { return e4m3_decode(code); }
 uint8_t orc_e4m3_encode(float v) { return e4m3_encode(v); }
+double orc_e5m2_decode(uint8_t code) { return e5m2_decode(code); }
+uint8_t orc_e5m2_encode(float v) { return e5m2_encode(v); }
 float orc_block_scale(float amax, int mode) { return block_scale(amax, mode); }
+float orc_block_scale_fmt(float amax, int mode, int fmt) { return block_scale(amax, mode, fmt); }
 float orc_bf16_to_float(uint16_t b) { return bf16_bits_to_float(b); }
 uint16_t orc_float_to_bf16(float f) { return float_to_bf16_bits(f); }
 
 void orc_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(v[i]);
+}
+
+void orc_e5m2_encode_array(const float* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e5m2_encode(v[i]);
 }
 
 // Activation quantization, 1x128 blocks [P1 "Der technische Durchbruch"].
@@ -151,9 +214,10 @@ void orc_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
 //            consecutive rows of one column; s_col : [M/128][K].
 //   The column-wise copy is quantized from x itself, not from q_row.
 //   q_col/s_col may be null (row-wise only).
-void orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
-                         int mode, uint8_t* q_row, float* s_row,
-                         uint8_t* q_col, float* s_col) {
+//   fmt: element format of the codes (0 = E4M3, 1 = E5M2).
+void orc_quant_act_1x128_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                             int mode, int fmt, uint8_t* q_row, float* s_row,
+                             uint8_t* q_col, float* s_col) {
   const int64_t nK = K / 128;
 #pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
@@ -163,10 +227,10 @@ void orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
         float a = std::fabs(bf16_bits_to_float(x[m * ldx + kb * 128 + j]));
         if (a > amax) amax = a;
       }
-      float s = block_scale(amax, mode);
+      float s = block_scale(amax, mode, fmt);
       s_row[kb * M + m] = s;
       for (int64_t j = 0; j < 128; ++j)
-        q_row[m * K + kb * 128 + j] = quant_one(x[m * ldx + kb * 128 + j], s);
+        q_row[m * K + kb * 128 + j] = quant_one(x[m * ldx + kb * 128 + j], s, fmt);
     }
   }
   if (!q_col) return;
@@ -179,12 +243,18 @@ void orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
         float a = std::fabs(bf16_bits_to_float(x[(mb * 128 + i) * ldx + k]));
         if (a > amax) amax = a;
       }
-      float s = block_scale(amax, mode);
+      float s = block_scale(amax, mode, fmt);
       s_col[mb * K + k] = s;
       for (int64_t i = 0; i < 128; ++i)
-        q_col[k * M + mb * 128 + i] = quant_one(x[(mb * 128 + i) * ldx + k], s);
+        q_col[k * M + mb * 128 + i] = quant_one(x[(mb * 128 + i) * ldx + k], s, fmt);
     }
   }
+}
+
+void orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                         int mode, uint8_t* q_row, float* s_row,
+                         uint8_t* q_col, float* s_col) {
+  orc_quant_act_1x128_fmt(x, M, K, ldx, mode, FMT_E4M3, q_row, s_row, q_col, s_col);
 }
 
 // Weight quantization, 128x128 blocks [P1 "Der technische Durchbruch"].
@@ -231,18 +301,20 @@ static double b_scale(int kind, const float* sB, int64_t N, int64_t K,
 // One output element of the GEMM reference over K-chunks [kb0, kb1):
 // sum_k (qA[m][k] * sA[k/128][m]) * (qB[n][k] * sB(n, k/128)) in fp64 from
 // the dequantized operands, and sum_k |a * b|.
+// fa / fb: element formats of the A and B codes (0 = E4M3, 1 = E5M2).
 static void ref_element(int kind, int64_t M, int64_t N, int64_t K,
                         const uint8_t* A, const float* sA, const uint8_t* B,
                         const float* sB, int64_t kb0, int64_t kb1, int64_t m,
-                        int64_t n, double* y, double* yabs) {
+                        int64_t n, double* y, double* yabs, int fa = FMT_E4M3,
+                        int fb = FMT_E4M3) {
   double acc = 0.0, aacc = 0.0;
   for (int64_t kb = kb0; kb < kb1; ++kb) {
     double sa = sA[kb * M + m];
     double sb = b_scale(kind, sB, N, K, n, kb);
     for (int64_t j = 0; j < 128; ++j) {
       int64_t k = kb * 128 + j;
-      double a = e4m3_decode(A[m * K + k]) * sa;
-      double b = e4m3_decode(B[n * K + k]) * sb;
+      double a = decode(A[m * K + k], fa) * sa;
+      double b = decode(B[n * K + k], fb) * sb;
       acc += a * b;
       aacc += std::fabs(a * b);
     }
@@ -255,16 +327,23 @@ static void ref_element(int kind, int64_t M, int64_t N, int64_t K,
 // over rows [m0,m1) x cols [n0,n1); y/yabs laid out [m1-m0][n1-n0].
 //   A : [M][K] codes (K-major), sA : [K/128][M]
 //   B : [N][K] codes (K-major), sB : per kind (see b_scale)
-void orc_gemm_ref_tile(int kind, int64_t M, int64_t N, int64_t K,
-                       const uint8_t* A, const float* sA, const uint8_t* B,
-                       const float* sB, int64_t m0, int64_t m1, int64_t n0,
-                       int64_t n1, double* y, double* yabs) {
+void orc_gemm_ref_tile_fmt(int kind, int fa, int fb, int64_t M, int64_t N, int64_t K,
+                           const uint8_t* A, const float* sA, const uint8_t* B,
+                           const float* sB, int64_t m0, int64_t m1, int64_t n0,
+                           int64_t n1, double* y, double* yabs) {
   const int64_t W = n1 - n0;
 #pragma omp parallel for schedule(static)
   for (int64_t m = m0; m < m1; ++m)
     for (int64_t n = n0; n < n1; ++n)
       ref_element(kind, M, N, K, A, sA, B, sB, 0, K / 128, m, n,
-                  &y[(m - m0) * W + (n - n0)], &yabs[(m - m0) * W + (n - n0)]);
+                  &y[(m - m0) * W + (n - n0)], &yabs[(m - m0) * W + (n - n0)], fa, fb);
+}
+
+void orc_gemm_ref_tile(int kind, int64_t M, int64_t N, int64_t K,
+                       const uint8_t* A, const float* sA, const uint8_t* B,
+                       const float* sB, int64_t m0, int64_t m1, int64_t n0,
+                       int64_t n1, double* y, double* yabs) {
+  orc_gemm_ref_tile_fmt(kind, FMT_E4M3, FMT_E4M3, M, N, K, A, sA, B, sB, m0, m1, n0, n1, y, yabs);
 }
 
 // Grouped (MoE expert) GEMM reference [P1 "Leistungsgewinne in der Praxis":
