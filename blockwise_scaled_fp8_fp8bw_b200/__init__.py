@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libfp8bw.so")
 FP8BW_OK = 0
 FP8BW_SCALE_FP32, FP8BW_SCALE_POW2 = 0, 1
 FP8BW_FPROP, FP8BW_DGRAD, FP8BW_WGRAD = 0, 1, 2
+FP8BW_FMT_E4M3, FP8BW_FMT_E5M2 = 0, 1
 FP8BW_REQUANT_MAX_PER_LAUNCH = 256
 FP8BW_MAX_EXPERTS = 512
 STATUS = {0: "FP8BW_OK", 1: "FP8BW_ERR_INVALID_ARG", 2: "FP8BW_ERR_ALIGNMENT",
@@ -55,13 +56,15 @@ def _load():
     L.fp8bw_quant_weight_128x128.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp]
     L.fp8bw_requant_weights.argtypes = [ctypes.POINTER(fp8bw_weight_desc), ctypes.c_int32, i32, vp]
     L.fp8bw_gemm.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, vp, i64, i32, vp]
+    L.fp8bw_quant_act_1x128_fmt.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp]
+    L.fp8bw_gemm_fmt.argtypes = [i32, i64, i64, i64, vp, vp, i32, vp, vp, i32, vp, i64, i32, vp]
     L.fp8bw_gemm_f32.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, vp, i64, ctypes.c_int32, i32, vp]
     L.fp8bw_grouped_gemm.argtypes = [i32, ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
     L.fp8bw_grouped_wgrad_f32.argtypes = [ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp,
                                           ctypes.c_int32, i32, vp]
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm",
-              "fp8bw_quant_act_1x128",
+              "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
               "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16"):
         getattr(L, f).restype = i32
@@ -133,6 +136,14 @@ def fp8bw_quant_act_1x128(x, mode, q_row, s_row, q_col=None, s_col=None, stream=
         _stream(stream)))
 
 
+def fp8bw_quant_act_1x128_fmt(x, mode, fmt, q_row, s_row, q_col=None, s_col=None, stream=None):
+    """fp8bw_quant_act_1x128 with the element format (FP8BW_FMT_E4M3 / _E5M2)."""
+    M, K = x.shape
+    _check("fp8bw_quant_act_1x128_fmt", load().fp8bw_quant_act_1x128_fmt(
+        _ptr(x), M, K, x.stride(0), int(mode), int(fmt), _ptr(q_row), _ptr(s_row), _ptr(q_col),
+        _ptr(s_col), _stream(stream)))
+
+
 def fp8bw_quant_weight_128x128(w, mode, q, s, qT=None, stream=None):
     """w [N, ldw] bf16; q [N,K] u8; s [N/128,K/128] f32; qT [K,N] u8 or None."""
     N, K = w.shape
@@ -156,6 +167,15 @@ def fp8bw_gemm(kind, A, sA, B, sB, D, mode=FP8BW_SCALE_FP32, stream=None):
     N = B.shape[0]
     _check("fp8bw_gemm", load().fp8bw_gemm(int(kind), M, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
                                         _ptr(D), D.stride(0), int(mode), _stream(stream)))
+
+
+def fp8bw_gemm_fmt(kind, A, sA, a_fmt, B, sB, b_fmt, D, mode=FP8BW_SCALE_FP32, stream=None):
+    """fp8bw_gemm with the element formats of A and B given."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check("fp8bw_gemm_fmt", load().fp8bw_gemm_fmt(int(kind), M, N, K, _ptr(A), _ptr(sA), int(a_fmt),
+                                                _ptr(B), _ptr(sB), int(b_fmt), _ptr(D), D.stride(0),
+                                                int(mode), _stream(stream)))
 
 
 def fp8bw_gemm_f32(kind, A, sA, B, sB, D, accumulate=False, mode=FP8BW_SCALE_FP32, stream=None):

@@ -10,14 +10,14 @@
 namespace fp8bw {
 cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
                              uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
-                             int num_sms, cudaStream_t st);
+                             int num_sms, cudaStream_t st, int fmt = 0);
 cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, int mode,
                                 uint8_t* q, float* s, uint8_t* qT, cudaStream_t st);
 cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cudaStream_t st);
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M,
                             int64_t N, int64_t K, const uint8_t* A, const float* sA,
                             const uint8_t* B, const float* sB, void* D, int64_t ldd, int mode,
-                            int num_sms, cudaStream_t st, int out_mode);
+                            int num_sms, cudaStream_t st, int out_mode, int a_fmt = 0, int b_fmt = 0);
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
@@ -108,6 +108,15 @@ FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {
 FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx,
                                    fp8bw_scale_mode mode, uint8_t* q_row, float* s_row,
                                    uint8_t* q_col, float* s_col, fp8bw_stream_t stream) {
+  return fp8bw_quant_act_1x128_fmt(x, M, K, ldx, mode, FP8BW_FMT_E4M3, q_row, s_row, q_col, s_col,
+                                   stream);
+}
+
+FP8BW_API fp8bw_status fp8bw_quant_act_1x128_fmt(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                       fp8bw_scale_mode mode, fp8bw_format fmt,
+                                       uint8_t* q_row, float* s_row, uint8_t* q_col,
+                                       float* s_col, fp8bw_stream_t stream) {
+  if (fmt != FP8BW_FMT_E4M3 && fmt != FP8BW_FMT_E5M2) return FP8BW_ERR_INVALID_ARG;
   if (!x || !q_row || !s_row) return FP8BW_ERR_INVALID_ARG;
   if ((q_col == nullptr) != (s_col == nullptr)) return FP8BW_ERR_INVALID_ARG;
   if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
@@ -122,7 +131,7 @@ FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K
   if (s != FP8BW_OK) return s;
   if (M == 0 || K == 0) return FP8BW_OK;
   return from_cuda(fp8bw::launch_quant_act(x, M, K, ldx, mode, q_row, s_row, q_col, s_col, sms,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+                                           reinterpret_cast<cudaStream_t>(stream), fmt));
 }
 
 FP8BW_API fp8bw_status fp8bw_quant_weight_128x128(const void* w, int64_t N, int64_t K, int64_t ldw,
@@ -162,7 +171,19 @@ FP8BW_API fp8bw_status fp8bw_requant_weights(const fp8bw_weight_desc* descs, int
 FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K, const uint8_t* A,
                         const float* sA, const uint8_t* B, const float* sB, void* D, int64_t ldd,
                         fp8bw_scale_mode mode, fp8bw_stream_t stream) {
+  return fp8bw_gemm_fmt(kind, M, N, K, A, sA, FP8BW_FMT_E4M3, B, sB, FP8BW_FMT_E4M3, D, ldd, mode,
+                        stream);
+}
+
+FP8BW_API fp8bw_status fp8bw_gemm_fmt(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                            const uint8_t* A, const float* sA, fp8bw_format a_fmt,
+                            const uint8_t* B, const float* sB, fp8bw_format b_fmt,
+                            void* D, int64_t ldd, fp8bw_scale_mode mode,
+                            fp8bw_stream_t stream) {
   if (kind != FP8BW_FPROP && kind != FP8BW_DGRAD && kind != FP8BW_WGRAD) return FP8BW_ERR_INVALID_ARG;
+  if ((a_fmt != FP8BW_FMT_E4M3 && a_fmt != FP8BW_FMT_E5M2) ||
+      (b_fmt != FP8BW_FMT_E4M3 && b_fmt != FP8BW_FMT_E5M2))
+    return FP8BW_ERR_INVALID_ARG;
   if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
   if (!A || !sA || !B || !sB || !D) return FP8BW_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || ldd < N) return FP8BW_ERR_INVALID_ARG;
@@ -176,7 +197,8 @@ FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, in
   if (M == 0 || N == 0) return FP8BW_OK;
   if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
   return from_cuda(fp8bw::launch_gemm_fp8(kind, false, 0, nullptr, M, N, K, A, sA, B, sB, D, ldd,
-                                          mode, sms, reinterpret_cast<cudaStream_t>(stream), 0));
+                                          mode, sms, reinterpret_cast<cudaStream_t>(stream), 0,
+                                          a_fmt, b_fmt));
 }
 
 FP8BW_API fp8bw_status fp8bw_gemm_f32(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,

@@ -30,21 +30,36 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Block scale: FP32 mode s = fp32(amax/448); POW2 mode s = 2^e with e the
-// smallest integer such that amax <= 448*2^e, clamped to [-127, 127];
-// s = 1 for an all-zero block.
-template <int MODE>
+// Two fp32 values to E5M2 codes (round to nearest even, saturating to 57344).
+__device__ __forceinline__ uint32_t cvt_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Codes of the element format FMT (FP8BW_FMT_E4M3 or FP8BW_FMT_E5M2).
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi) {
+  return FMT == FP8BW_FMT_E5M2 ? cvt_e5m2x2(lo, hi) : cvt_e4m3x2(lo, hi);
+}
+
+// Block scale: FP32 mode s = fp32(amax/Q); POW2 mode s = 2^e with e the
+// smallest integer such that amax <= Q*2^e, clamped to [-127, 127];
+// s = 1 for an all-zero block.  Q is the format's largest value, 448 =
+// 1.75 * 2^8 (E4M3) or 57344 = 1.75 * 2^15 (E5M2).
+template <int MODE, int FMT = FP8BW_FMT_E4M3>
 __device__ __forceinline__ float block_scale(float amax) {
+  constexpr int kQexp = FMT == FP8BW_FMT_E5M2 ? 15 : 8;
   if (amax == 0.0f) return 1.0f;
-  if (MODE == FP8BW_SCALE_FP32) return __fdiv_rn(amax, 448.0f);
+  if (MODE == FP8BW_SCALE_FP32) return __fdiv_rn(amax, FMT == FP8BW_FMT_E5M2 ? 57344.0f : 448.0f);
   const uint32_t b = __float_as_uint(amax);
   const int ef = (int)(b >> 23);          // biased exponent (amax > 0)
   int e;
   if (ef == 0) {
     e = -127;                             // subnormal amax: below the clamp
   } else {
-    // amax = (1 + f) * 2^(ef-127); 448*2^e = 1.75 * 2^(8+e)
-    e = ef - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    // amax = (1 + f) * 2^(ef-127); Q*2^e = 1.75 * 2^(kQexp+e)
+    e = ef - 127 - kQexp + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
     e = e < -127 ? -127 : (e > 127 ? 127 : e);
   }
   return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
@@ -469,6 +484,12 @@ __device__ __forceinline__ void bulk_wait0() {
 // [23] (1 = UE8M0), M>>4 at [24,29), A scale-factor id [29,31).
 __host__ __device__ constexpr uint32_t idesc_mx(uint32_t M, uint32_t N, uint32_t sf_id) {
   return (sf_id << 4) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) | (sf_id << 29);
+}
+
+// Operand-format fields of both instruction descriptors (A at bits [7,10),
+// B at [10,13)): 0 = E4M3, 1 = E5M2.
+__host__ __device__ constexpr uint32_t idesc_fmt_bits(uint32_t a_fmt, uint32_t b_fmt) {
+  return (a_fmt << 7) | (b_fmt << 10);
 }
 
 // ----------------------------------------------------------- setmaxnreg ---

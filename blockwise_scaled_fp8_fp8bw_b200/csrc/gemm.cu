@@ -101,6 +101,7 @@ struct GemmArgs {
   uint16_t* D;         // BF16 kernel only (the FP8 kernel stores through a tensor map)
   int64_t ldd;
   int out_mode;        // OutMode of the FP8 kernels' epilogue
+  uint32_t fmt_bits;   // operand formats in the MMA instruction descriptor (0: both E4M3)
   int stall_chunk;     // testing: CTA 0's producer never fills this chunk (-1: off)
 };
 
@@ -404,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d = tmem + buf * BN;
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk) {  // +32 bytes = +2 in the >>4 address field
-              if (PAIR) umma_f8f6f4_pair(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
-              else umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, C::kIdesc, kk > 0 ? 1u : 0u);
+              if (PAIR) umma_f8f6f4_pair(d, da + 2 * kk, db + 2 * kk, C::kIdesc | a.fmt_bits, kk > 0 ? 1u : 0u);
+              else umma_f8f6f4(d, da + 2 * kk, db + 2 * kk, C::kIdesc | a.fmt_bits, kk > 0 ? 1u : 0u);
             }
             if (PAIR) {
               umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
@@ -919,9 +920,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BK / 32; ++kk) {
               const uint32_t acc = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
               if (PAIR)
-                umma_mx_pair(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j), tsf, tsf + 4, acc);
+                umma_mx_pair(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j) | a.fmt_bits, tsf, tsf + 4, acc);
               else
-                umma_mx(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j), tsf, tsf + 4, acc);
+                umma_mx(tmem, da + 2 * kk, db + 2 * kk, idesc_mx(C::kIdescM, BN, j) | a.fmt_bits, tsf, tsf + 4, acc);
             }
             if (PAIR) umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
             else umma_commit(smem_u32(&bars->empty[stage]));
@@ -1333,7 +1334,7 @@ int gemm_stall_chunk = -1;  // testing hook, consumed by the next FP8 GEMM launc
 cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off, int64_t M, int64_t N,
                             int64_t K, const uint8_t* A, const float* sA, const uint8_t* B,
                             const float* sB, void* D, int64_t ldd, int mode, int num_sms,
-                            cudaStream_t st, int out_mode) {
+                            cudaStream_t st, int out_mode, int a_fmt, int b_fmt) {
   // CTA pairs everywhere; grouped fprop/dgrad pair tiles stay inside one
   // expert, so their number is only bounded here (sum of ceil(rows_g/256)
   // <= (M/128 + G)/2) and the kernel skips the tiles past the real count.
@@ -1352,6 +1353,7 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   a.G = G;
   a.stall_chunk = gemm_stall_chunk;
   a.out_mode = out_mode;
+  a.fmt_bits = idesc_fmt_bits((uint32_t)a_fmt, (uint32_t)b_fmt);
   gemm_stall_chunk = -1;
   if (grouped && kind == FP8BW_WGRAD) a.tiles = G * a.m_tiles * a.n_tiles;
   else a.tiles = a.m_tiles * a.n_tiles;

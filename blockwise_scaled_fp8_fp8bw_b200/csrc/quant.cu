@@ -71,10 +71,10 @@ struct Divisor {
   bool exact;
 };
 
-template <int MODE>
+template <int MODE, int FMT = FP8BW_FMT_E4M3>
 __device__ __forceinline__ Divisor make_divisor(float amax) {
   Divisor d;
-  d.s = block_scale<MODE>(amax);
+  d.s = block_scale<MODE, FMT>(amax);
   if (MODE == FP8BW_SCALE_POW2) {
     d.y = rcp_rn(d.s);  // exact: s is a power of two in [2^-127, 2^127]
     d.exact = false;
@@ -106,32 +106,33 @@ __device__ __forceinline__ float div1(float x, const Divisor& d) {
   return __fmaf_rn(r, -d.y, q0);
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __device__ __forceinline__ uint2 quant8_fast(uint4 v, float s, float y) {
   const float2 s2 = make_float2(s, s), y2 = make_float2(y, y);
   const float2 a = div2<MODE>(make_float2(bf16lo(v.x), bf16hi(v.x)), s2, y2);
   const float2 b = div2<MODE>(make_float2(bf16lo(v.y), bf16hi(v.y)), s2, y2);
   const float2 c = div2<MODE>(make_float2(bf16lo(v.z), bf16hi(v.z)), s2, y2);
   const float2 e = div2<MODE>(make_float2(bf16lo(v.w), bf16hi(v.w)), s2, y2);
-  return make_uint2(cvt_e4m3x2(a.x, a.y) | (cvt_e4m3x2(b.x, b.y) << 16),
-                    cvt_e4m3x2(c.x, c.y) | (cvt_e4m3x2(e.x, e.y) << 16));
+  return make_uint2(cvt_fp8x2<FMT>(a.x, a.y) | (cvt_fp8x2<FMT>(b.x, b.y) << 16),
+                    cvt_fp8x2<FMT>(c.x, c.y) | (cvt_fp8x2<FMT>(e.x, e.y) << 16));
 }
 
 // Slow path (kept out of line so the fast path carries no division code).
+template <int FMT>
 __device__ __noinline__ uint2 quant8_exact(uint4 v, Divisor d) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[2];
   for (int i = 0; i < 2; ++i)
-    o[i] = cvt_e4m3x2(div1(bf16lo(w[2 * i]), d), div1(bf16hi(w[2 * i]), d)) |
-           (cvt_e4m3x2(div1(bf16lo(w[2 * i + 1]), d), div1(bf16hi(w[2 * i + 1]), d)) << 16);
+    o[i] = cvt_fp8x2<FMT>(div1(bf16lo(w[2 * i]), d), div1(bf16hi(w[2 * i]), d)) |
+           (cvt_fp8x2<FMT>(div1(bf16lo(w[2 * i + 1]), d), div1(bf16hi(w[2 * i + 1]), d)) << 16);
   return make_uint2(o[0], o[1]);
 }
 
 // 8 codes of one 16-byte vector with one divisor (uniform branch per warp).
-template <int MODE>
+template <int MODE, int FMT = FP8BW_FMT_E4M3>
 __device__ __forceinline__ uint2 quant8(uint4 v, const Divisor& d) {
-  if (MODE == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d.exact)) return quant8_exact(v, d);
-  return quant8_fast<MODE>(v, d.s, d.y);
+  if (MODE == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d.exact)) return quant8_exact<FMT>(v, d);
+  return quant8_fast<MODE, FMT>(v, d.s, d.y);
 }
 
 struct ColCodes {
@@ -142,6 +143,7 @@ struct ColWords {
 };
 
 // Slow path of the column pass (a column block with amax < 2^-80).
+template <int FMT>
 __device__ __noinline__ ColCodes column_codes_exact(ColWords v, Divisor d0, Divisor d1) {
   ColCodes c;
   for (int i = 0; i < 8; ++i) {
@@ -150,8 +152,8 @@ __device__ __noinline__ ColCodes column_codes_exact(ColWords v, Divisor d0, Divi
       a[u] = div1(bf16lo(v.w[4 * i + u]), d0);
       b[u] = div1(bf16hi(v.w[4 * i + u]), d1);
     }
-    c.c0[i] = cvt_e4m3x2(a[0], a[1]) | (cvt_e4m3x2(a[2], a[3]) << 16);
-    c.c1[i] = cvt_e4m3x2(b[0], b[1]) | (cvt_e4m3x2(b[2], b[3]) << 16);
+    c.c0[i] = cvt_fp8x2<FMT>(a[0], a[1]) | (cvt_fp8x2<FMT>(a[2], a[3]) << 16);
+    c.c1[i] = cvt_fp8x2<FMT>(b[0], b[1]) | (cvt_fp8x2<FMT>(b[2], b[3]) << 16);
   }
   return c;
 }
@@ -189,7 +191,7 @@ __device__ __forceinline__ void issue_tile(ActSmem& sm, const CUtensorMap* tm, i
 //                two columns, posts the partial maxima; after the tile's one
 //                barrier it combines the four row groups, quantizes and
 //                writes 2 x 32 codes and, for rg = 0, the column scales.
-template <int MODE, bool COL>
+template <int MODE, bool COL, int FMT>
 __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUtensorMap tmX,
                                                      int64_t M, int64_t K,
                                                      uint8_t* __restrict__ q_row,
@@ -232,13 +234,13 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
 #pragma unroll
       for (int j = 1; j < 8; ++j) m = umax2(m, absmax8(v[j]));
       m = umax2(m, __shfl_xor_sync(0xffffffffu, m, 8));
-      const Divisor d = make_divisor<MODE>(halves_max(m));
+      const Divisor d = make_divisor<MODE, FMT>(halves_max(m));
       if (hh == 0) s_row[(k0 / 128) * M + m0 + rr] = d.s;
       uint8_t* qr = q_row + (m0 + rr) * K + k0 + hh * 64;
 #pragma unroll
       for (int j = 0; j < 8; j += 4) {
-        const uint2 c0 = quant8<MODE>(v[j], d), c1 = quant8<MODE>(v[j + 1], d);
-        const uint2 c2 = quant8<MODE>(v[j + 2], d), c3 = quant8<MODE>(v[j + 3], d);
+        const uint2 c0 = quant8<MODE, FMT>(v[j], d), c1 = quant8<MODE, FMT>(v[j + 1], d);
+        const uint2 c2 = quant8<MODE, FMT>(v[j + 2], d), c3 = quant8<MODE, FMT>(v[j + 3], d);
         st_global_v8(qr + 8 * j, make_uint4(c0.x, c0.y, c1.x, c1.y), make_uint4(c2.x, c2.y, c3.x, c3.y));
       }
     }
@@ -263,13 +265,13 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
     if (COL) {
       const uint32_t m = umax2(umax2(sm.colmax[cur][0][wc], sm.colmax[cur][1][wc]),
                                umax2(sm.colmax[cur][2][wc], sm.colmax[cur][3][wc]));
-      const Divisor d0 = make_divisor<MODE>(__uint_as_float((m & 0xFFFFu) << 16));
-      const Divisor d1 = make_divisor<MODE>(__uint_as_float(m & 0xFFFF0000u));
+      const Divisor d0 = make_divisor<MODE, FMT>(__uint_as_float((m & 0xFFFFu) << 16));
+      const Divisor d1 = make_divisor<MODE, FMT>(__uint_as_float(m & 0xFFFF0000u));
       if (rg == 0)
         *reinterpret_cast<float2*>(s_col + (m0 / 128) * K + k0 + 2 * wc) = make_float2(d0.s, d1.s);
       uint32_t c0[8], c1[8];
       if (MODE == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d0.exact || d1.exact)) {
-        const ColCodes c = column_codes_exact(cw, d0, d1);
+        const ColCodes c = column_codes_exact<FMT>(cw, d0, d1);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           c0[j] = c.c0[j];
@@ -285,8 +287,8 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
             const uint32_t w = cw.w[4 * j + u];
             q[u] = div2<MODE>(make_float2(bf16lo(w), bf16hi(w)), s2, y2);
           }
-          c0[j] = cvt_e4m3x2(q[0].x, q[1].x) | (cvt_e4m3x2(q[2].x, q[3].x) << 16);
-          c1[j] = cvt_e4m3x2(q[0].y, q[1].y) | (cvt_e4m3x2(q[2].y, q[3].y) << 16);
+          c0[j] = cvt_fp8x2<FMT>(q[0].x, q[1].x) | (cvt_fp8x2<FMT>(q[2].x, q[3].x) << 16);
+          c1[j] = cvt_fp8x2<FMT>(q[0].y, q[1].y) | (cvt_fp8x2<FMT>(q[2].y, q[3].y) << 16);
         }
       }
       uint8_t* qc = q_col + (k0 + 2 * wc) * M + m0 + rg * 32;
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(QT) k_requant(const __grid_constant__ RequantT
 // ------------------------------------------------------------ launchers ---
 cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
                              uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
-                             int num_sms, cudaStream_t st) {
+                             int num_sms, cudaStream_t st, int fmt) {
   CUtensorMap tm;
   if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)K, (uint64_t)M,
                 (uint64_t)ldx, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -416,16 +418,23 @@ cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, i
   const size_t smem = sizeof(ActSmem) + 1024;
   const bool col = q_col != nullptr;
   cudaError_t e = cudaSuccess;
-#define FP8BW_QA(MD, CL)                                                                      \
-  do {                                                                                        \
-    e = cudaFuncSetAttribute(k_quant_act<MD, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             (int)smem);                                                      \
-    if (e == cudaSuccess) k_quant_act<MD, CL><<<grid, QT, smem, st>>>(tm, M, K, q_row, s_row, q_col, s_col); \
+#define FP8BW_QA(MD, CL, FM)                                                                      \
+  do {                                                                                            \
+    e = cudaFuncSetAttribute(k_quant_act<MD, CL, FM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)smem);                                                          \
+    if (e == cudaSuccess)                                                                         \
+      k_quant_act<MD, CL, FM><<<grid, QT, smem, st>>>(tm, M, K, q_row, s_row, q_col, s_col);      \
   } while (0)
-  if (mode == FP8BW_SCALE_FP32) {
-    if (col) FP8BW_QA(0, true); else FP8BW_QA(0, false);
+  if (fmt == FP8BW_FMT_E5M2) {
+    if (mode == FP8BW_SCALE_FP32) {
+      if (col) FP8BW_QA(0, true, 1); else FP8BW_QA(0, false, 1);
+    } else {
+      if (col) FP8BW_QA(1, true, 1); else FP8BW_QA(1, false, 1);
+    }
+  } else if (mode == FP8BW_SCALE_FP32) {
+    if (col) FP8BW_QA(0, true, 0); else FP8BW_QA(0, false, 0);
   } else {
-    if (col) FP8BW_QA(1, true); else FP8BW_QA(1, false);
+    if (col) FP8BW_QA(1, true, 0); else FP8BW_QA(1, false, 0);
   }
 #undef FP8BW_QA
   if (e != cudaSuccess) return e;

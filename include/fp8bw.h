@@ -65,6 +65,15 @@ typedef enum { FP8BW_SCALE_FP32 = 0, FP8BW_SCALE_POW2 = 1 } fp8bw_scale_mode;
 
 typedef enum { FP8BW_FPROP = 0, FP8BW_DGRAD = 1, FP8BW_WGRAD = 2 } fp8bw_gemm_kind;
 
+/* Element format of the FP8 codes.  E4M3 is the method's; E5M2 (5 exponent
+ * bits, 2 mantissa bits, bias 15, largest finite value 57344; page "FP8
+ * Trainingsinfrastructuur", section "Het landschap van numerieke precisie":
+ * the gradient format of the per-tensor recipe) is offered for activation
+ * gradients as a comparison point.  Block scales then use 57344 in place of
+ * 448 (FP32: s = fp32(amax / 57344); POW2: the smallest 2^e with
+ * amax <= 57344 * 2^e). */
+typedef enum { FP8BW_FMT_E4M3 = 0, FP8BW_FMT_E5M2 = 1 } fp8bw_format;
+
 /* Checks that `device` is an sm_100 part and caches its SM count.  Called
  * implicitly by every entry point for the current device; calling it
  * explicitly first keeps that one-time query out of timed regions. */
@@ -161,6 +170,24 @@ FP8BW_API fp8bw_status fp8bw_requant_weights(const fp8bw_weight_desc* descs, int
 FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
                         const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                         void* D, int64_t ldd, fp8bw_scale_mode mode, fp8bw_stream_t stream);
+
+/* fp8bw_quant_act_1x128 with the element format chosen: FP8BW_FMT_E4M3
+ * gives exactly fp8bw_quant_act_1x128's result; FP8BW_FMT_E5M2 encodes E5M2
+ * codes (round to nearest even, saturating to 57344) with the E5M2 scale
+ * rule above.  Arguments, layouts and errors as in fp8bw_quant_act_1x128. */
+FP8BW_API fp8bw_status fp8bw_quant_act_1x128_fmt(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                       fp8bw_scale_mode mode, fp8bw_format fmt,
+                                       uint8_t* q_row, float* s_row, uint8_t* q_col,
+                                       float* s_col, fp8bw_stream_t stream);
+
+/* fp8bw_gemm with the element formats of A and B given (codes decoded as
+ * E4M3 or E5M2; e.g. dgrad/wgrad with E5M2 activation gradients against
+ * E4M3 weights or activations).  Everything else as in fp8bw_gemm. */
+FP8BW_API fp8bw_status fp8bw_gemm_fmt(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                            const uint8_t* A, const float* sA, fp8bw_format a_fmt,
+                            const uint8_t* B, const float* sB, fp8bw_format b_fmt,
+                            void* D, int64_t ldd, fp8bw_scale_mode mode,
+                            fp8bw_stream_t stream);
 
 /* The same GEMM with an fp32 output, for the weight gradient's fp32 main
  * gradient of mixed-precision training (the optimizer step after which the

@@ -66,6 +66,10 @@ def test_host_validation(lib):
     assert r.fp8bw_quant_act_1x128(p, 128, 200, 256, 0, p, p, N, N, N) == 2
     assert r.fp8bw_quant_act_1x128(p, 128, 128, 100, 0, p, p, N, N, N) == 1   # ldx < K
     assert r.fp8bw_gemm_bf16(128, 128, 100, p, p, p, 128, N) == 2
+    # element formats: only E4M3 (0) and E5M2 (1)
+    assert r.fp8bw_quant_act_1x128_fmt(p, 128, 128, 128, 0, 2, p, p, N, N, N) == 1
+    assert r.fp8bw_gemm_fmt(1, 128, 128, 128, p, p, 2, p, p, 0, p, 128, 0, N) == 1
+    assert r.fp8bw_gemm_fmt(1, 128, 128, 128, p, p, 1, p, p, 3, p, 128, 0, N) == 1
     # fp32 output: accumulate flag, 16-byte rows (ldd a multiple of 4), ldd >= N
     assert r.fp8bw_gemm_f32(2, 128, 128, 128, p, p, p, p, p, 128, 2, 0, N) == 1
     assert r.fp8bw_gemm_f32(2, 128, 128, 128, p, p, p, p, p, 130, 1, 0, N) == 2

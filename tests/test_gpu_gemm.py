@@ -246,3 +246,28 @@ def test_gemm_f32_store_and_accumulate(fb, orc, kind, mode):
     assert fb.fp8bw_last_device_error() == 0
     bad, worst = orc.check_tol_f32(Dacc.cpu().numpy(), D0.astype(np.float64) + 2 * yr, 2 * ya)
     assert bad == 0, worst
+
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("kind", [1, 2])
+def test_e5m2_gradient_gemms(fb, orc, kind, mode):
+    """dgrad / wgrad with E5M2 activation gradients (quantized by the oracle
+    with the E5M2 rule) against E4M3 weights / activations: fp8bw_gemm_fmt
+    within tolerance of the oracle's reference decoding A as E5M2."""
+    X, W, dY = workloads.tiny(3)
+    qx, sx, qxc, sxc = orc.quant_act_1x128(bits(X), mode)
+    qw, sw, qwT = orc.quant_weight_128x128(bits(W), mode)
+    qd, sd, qdc, sdc = orc.quant_act_1x128(bits(dY), mode, fmt=orc.FMT_E5M2)
+    A, sA, B, sB = (qd, sd, qwT, sw) if kind == 1 else (qdc, sdc, qxc, sxc)
+    M, N = A.shape[0], B.shape[0]
+    D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_gemm_fmt(kind, dev(A), dev(sA), fb.FP8BW_FMT_E5M2, dev(B), dev(sB), fb.FP8BW_FMT_E4M3, D, mode)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    yr, ya = orc.gemm_ref_tile(kind, A, sA, B, sB, 0, M, 0, N, fa=orc.FMT_E5M2)
+    bad, worst = orc.check_tol(bits(D), yr, ya)
+    assert bad == 0, worst
+    # read as E4M3 the same bytes give a different product: the format is used
+    yr4, _ = orc.gemm_ref_tile(kind, A, sA, B, sB, 0, M, 0, N)
+    assert not np.allclose(yr4, yr)

@@ -100,3 +100,30 @@ def test_requant_batch(fb, orc, mode):
         assert_bytes_equal(f32(s).view(np.uint32), os_.view(np.uint32), f"s[{i}]")
         if qT is not None:
             assert_bytes_equal(u8(qT), oqT, f"qT[{i}]")
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_act_e5m2(fb, orc, mode):
+    """E5M2 codes (the gradient format of the per-tensor recipe, "FP8
+    Trainingsinfrastructuur", "Het landschap van numerieke precisie") with
+    the 57344 scale rule: bit-exact against the oracle, including zero, -0,
+    subnormal and huge blocks."""
+    _, _, dY = workloads.tiny(0)
+    g = torch.Generator().manual_seed(12)
+    edge = torch.zeros((256, 384), dtype=torch.float32)
+    edge[:128, 128:256] = torch.randn((128, 128), generator=g) * 1e-39
+    edge[128:, 128:256] = torch.randn((128, 128), generator=g).clamp(-3, 3) * 1.1e38
+    edge[:, 256:] = torch.randn((256, 128), generator=g) * 1e-3
+    edge = edge.to(torch.bfloat16)
+    edge[128:, :128] = -0.0
+    for x_cpu in (dY, edge):
+        x = x_cpu.to(DEV)
+        M, K = x.shape
+        q_row, s_row, q_col, s_col = act_buffers(M, K, DEV)
+        fb.fp8bw_quant_act_1x128_fmt(x, mode, fb.FP8BW_FMT_E5M2, q_row, s_row, q_col, s_col)
+        torch.cuda.synchronize()
+        oq, os_, oqc, osc = orc.quant_act_1x128(bits(x_cpu), mode, fmt=orc.FMT_E5M2)
+        assert_bytes_equal(u8(q_row), oq, "q_row")
+        assert_bytes_equal(f32(s_row).view(np.uint32), os_.view(np.uint32), "s_row")
+        assert_bytes_equal(u8(q_col), oqc, "q_col")
+        assert_bytes_equal(f32(s_col).view(np.uint32), osc.view(np.uint32), "s_col")
