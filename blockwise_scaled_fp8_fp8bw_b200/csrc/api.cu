@@ -30,6 +30,8 @@ constexpr int kMaxDevices = 64;
 int g_sms[kMaxDevices];  // 0 = not initialised, -1 = unsupported
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// The activation quantizer writes its codes with 32-byte stores.
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 inline bool mult128(int64_t v) { return v >= 0 && (v & 127) == 0; }
 constexpr int64_t kMaxDim = int64_t(1) << 30;  // sizes index with 32-bit tile math
 
@@ -123,7 +125,7 @@ FP8BW_API fp8bw_status fp8bw_quant_act_1x128_fmt(const void* x, int64_t M, int64
   if (M < 0 || K < 0 || ldx < K) return FP8BW_ERR_INVALID_ARG;
   if (M > kMaxDim || K > kMaxDim || M / 128 > 65535) return FP8BW_ERR_TOO_LARGE;
   if (!mult128(M) || !mult128(K) || (ldx & 7) != 0) return FP8BW_ERR_ALIGNMENT;
-  if (!aligned16(x) || !aligned16(q_row) || !aligned16(s_row) || (q_col && !aligned16(q_col)) ||
+  if (!aligned16(x) || !aligned32(q_row) || !aligned16(s_row) || (q_col && !aligned32(q_col)) ||
       (s_col && !aligned16(s_col)))
     return FP8BW_ERR_ALIGNMENT;
   int sms = 0;

@@ -112,7 +112,8 @@ FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk);
  * For mixture-of-experts tokens grouped by expert, pad each expert's segment
  * to a multiple of 128 rows (zero rows): column blocks then never straddle
  * two experts and zero rows change no block's amax.
- * Requires M, K multiples of 128, ldx >= K, ldx a multiple of 8. */
+ * Requires M, K multiples of 128, ldx >= K, ldx a multiple of 8, and q_row,
+ * q_col 32-byte aligned (the codes leave in 32-byte stores). */
 FP8BW_API fp8bw_status fp8bw_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx,
                                    fp8bw_scale_mode mode, uint8_t* q_row, float* s_row,
                                    uint8_t* q_col, float* s_col, fp8bw_stream_t stream);

@@ -65,6 +65,11 @@ def test_host_validation(lib):
     assert r.fp8bw_gemm(0, 128, 256, 128, p, p, p, p, p, 128, 0, N) == 1   # ldd < N
     assert r.fp8bw_quant_act_1x128(p, 128, 200, 256, 0, p, p, N, N, N) == 2
     assert r.fp8bw_quant_act_1x128(p, 128, 128, 100, 0, p, p, N, N, N) == 1   # ldx < K
+    # activation codes leave in 32-byte stores: q_row / q_col 32-byte aligned
+    p16 = ctypes.c_void_p(0x10010)
+    assert r.fp8bw_quant_act_1x128(p, 128, 128, 128, 0, p16, p, N, N, N) == 2
+    assert r.fp8bw_quant_act_1x128(p, 128, 128, 128, 0, p, p, p16, p, N) == 2
+    assert r.fp8bw_quant_act_1x128_fmt(p, 128, 128, 128, 0, 1, p, p, p16, p, N) == 2
     assert r.fp8bw_gemm_bf16(128, 128, 100, p, p, p, 128, N) == 2
     # element formats: only E4M3 (0) and E5M2 (1)
     assert r.fp8bw_quant_act_1x128_fmt(p, 128, 128, 128, 0, 2, p, p, N, N, N) == 1
