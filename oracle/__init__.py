@@ -62,6 +62,8 @@ def lib():
         L.orc_block_scale_fmt.argtypes = [flt, i32, i32]
         L.orc_block_scale_fmt.restype = flt
         L.orc_quant_act_1x128_fmt.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+        L.orc_quant_tensor_delayed.argtypes = [vp, i64, i64, i64, i32, i32, vp, i32, vp, vp,
+                                               vp, vp]
         L.orc_gemm_ref_tile_fmt.argtypes = [i32, i32, i32, i64, i64, i64, vp, vp, vp, vp,
                                             i64, i64, i64, i64, vp, vp]
         L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
@@ -181,6 +183,24 @@ def quant_weight_128x128(w_bits: np.ndarray, mode: int, transposed: bool = True)
     lib().orc_quant_weight_128x128(_p(w), N, K, K, mode, _p(q), _p(s),
                                    _p(qT) if transposed else None)
     return q, s, qT
+
+
+def quant_tensor_delayed(x_bits: np.ndarray, hist: np.ndarray, mode: int,
+                         fmt: int = FMT_E4M3, transposed: bool = True):
+    """Per-tensor delayed scaling ("FP8 Trainingsinfrastructuur", sections
+    "Transformer Engine: de softwarebasis" and "Scaling-strategieën en
+    stabiliteit").  x_bits: uint16 [M, K]; hist: float32 [H], newest first
+    (not modified).  Returns (q, qT, scale, amax, new_hist)."""
+    x = _u16(x_bits)
+    M, K = x.shape
+    h = _f32(hist).copy()
+    q = np.empty((M, K), np.uint8)
+    qT = np.empty((K, M), np.uint8) if transposed else None
+    sc = np.zeros(1, np.float32)
+    am = np.zeros(1, np.float32)
+    lib().orc_quant_tensor_delayed(_p(x), M, K, K, mode, fmt, _p(h), h.size, _p(q),
+                                   _p(qT) if transposed else None, _p(sc), _p(am))
+    return q, qT, np.float32(sc[0]), np.float32(am[0]), h
 
 
 # ------------------------------------------------------------------- GEMMs --

@@ -287,6 +287,46 @@ void orc_quant_weight_128x128(const uint16_t* w, int64_t N, int64_t K,
     for (int64_t k = 0; k < K; ++k) qT[k * N + n] = q[n * K + k];
 }
 
+// Per-tensor delayed scaling [P2 "Transformer Engine: de softwarebasis" and
+// "Scaling-strategieën en stabiliteit"]: one scale for the whole tensor,
+// taken from the largest absolute values observed in earlier iterations
+// (the page's recipe keeps a history of 16 and takes its maximum, margin 0),
+// not from the tensor being quantized; this call's amax then enters the
+// history.  The scale rule applied to that maximum is the block rule above.
+//   x     : bf16 bits [M][ldx], first K columns
+//   hist  : [H] amax history, newest first, updated in place:
+//           hist'[0] = amax(x), hist'[i] = hist[i-1] for 0 < i < H
+//   q     : [M][K] codes, q = encode(fp32(x) / s); values beyond the
+//           format's largest saturate (the history may under-estimate)
+//   qT    : [K][M] the byte transpose of q (one scale: the column-wise copy
+//           is the transpose), may be null
+//   scale : s = block_scale(max(hist), mode, fmt)
+//   amax  : max |x| of this call
+// A NaN, in x or in hist, never wins a maximum (the comparisons below are
+// false for NaN).
+void orc_quant_tensor_delayed(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                              int mode, int fmt, float* hist, int32_t H, uint8_t* q,
+                              uint8_t* qT, float* scale, float* amax) {
+  float h = 0.0f;
+  for (int32_t i = 0; i < H; ++i)
+    if (hist[i] > h) h = hist[i];
+  const float s = block_scale(h, mode, fmt);
+  float a = 0.0f;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = std::fabs(bf16_bits_to_float(x[m * ldx + k]));
+      if (v > a) a = v;
+      q[m * K + k] = quant_one(x[m * ldx + k], s, fmt);
+    }
+  if (qT)
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t k = 0; k < K; ++k) qT[k * M + m] = q[m * K + k];
+  for (int32_t i = H - 1; i > 0; --i) hist[i] = hist[i - 1];
+  if (H > 0) hist[0] = a;
+  *scale = s;
+  *amax = a;
+}
+
 // Scale of operand B for output column n at K-chunk kb, per GEMM kind:
 //   kind 0 (fprop): 128x128 block grid [N/128][K/128]
 //   kind 1 (dgrad): the weight's own grid, read transposed: [K/128][N/128]
