@@ -49,7 +49,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--case", default=None,
                    help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
-                        "requant|bf16_fprop|wgrad_acc on --layer at --tokens, requant_sweep (32 layers), or "
+                        "requant|bf16_fprop|wgrad_acc|quant_delayed_dy|quant_delayed_x on --layer at "
+                        "--tokens, requant_sweep (32 layers), or "
                         "moe_fprop|moe_dgrad|moe_wgrad "
                         "on the MoE expert layer --layer gate_up|down")
     p.add_argument("--layer", default="gate_up", choices=[n for n, _, _ in workloads.LLAMA8B_LAYERS])
@@ -377,6 +378,16 @@ def run_case(args):
         "requant": (lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode), l.weight_bytes, "GB/s"),
         "bf16_fprop": (lambda: fb.fp8bw_gemm_bf16(l.X, l.W, l.Y), l.flops / 3, "TFLOP/s"),
     }
+    # per-tensor delayed scaling (history of 16, the comparison recipe):
+    # dY in E5M2 and X in E4M3, each with its byte-transposed copy; 2 bytes
+    # read and 2 written per element
+    hist, sc, am = (torch.zeros(16, dtype=torch.float32, device=l.X.device),
+                    torch.empty(1, dtype=torch.float32, device=l.X.device),
+                    torch.empty(1, dtype=torch.float32, device=l.X.device))
+    calls["quant_delayed_dy"] = (lambda: fb.fp8bw_quant_tensor_delayed(
+        l.dY, fb.FP8BW_FMT_E5M2, mode, hist, l.qd, l.qdc, sc, am), 4 * l.M * l.N, "GB/s")
+    calls["quant_delayed_x"] = (lambda: fb.fp8bw_quant_tensor_delayed(
+        l.X, fb.FP8BW_FMT_E4M3, mode, hist, l.qx, l.qxc, sc, am), 4 * l.M * l.K, "GB/s")
     if args.case == "wgrad_acc":   # wgrad added into an fp32 main gradient
         main_grad = torch.zeros((N, K), dtype=torch.float32, device=l.X.device)
         calls["wgrad_acc"] = (lambda: fb.fp8bw_gemm_f32(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, main_grad,

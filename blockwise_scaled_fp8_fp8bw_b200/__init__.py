@@ -25,6 +25,7 @@ FP8BW_FPROP, FP8BW_DGRAD, FP8BW_WGRAD = 0, 1, 2
 FP8BW_FMT_E4M3, FP8BW_FMT_E5M2 = 0, 1
 FP8BW_REQUANT_MAX_PER_LAUNCH = 256
 FP8BW_MAX_EXPERTS = 512
+FP8BW_MAX_HISTORY = 1024
 STATUS = {0: "FP8BW_OK", 1: "FP8BW_ERR_INVALID_ARG", 2: "FP8BW_ERR_ALIGNMENT",
           3: "FP8BW_ERR_UNSUPPORTED_ARCH", 4: "FP8BW_ERR_CUDA", 5: "FP8BW_ERR_TIMEOUT",
           6: "FP8BW_ERR_DEVICE_CHECK", 7: "FP8BW_ERR_TOO_LARGE"}
@@ -63,10 +64,13 @@ def _load():
     L.fp8bw_grouped_wgrad_f32.argtypes = [ctypes.c_int32, vp, i64, i64, i64, vp, vp, vp, vp, vp,
                                           ctypes.c_int32, i32, vp]
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
+    L.fp8bw_quant_tensor_delayed.argtypes = [vp, i64, i64, i64, i32, i32, vp, ctypes.c_int32, vp, vp,
+                                             vp, vp, vp, i64, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm",
               "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
-              "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16"):
+              "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16",
+              "fp8bw_quant_tensor_delayed"):
         getattr(L, f).restype = i32
     return L
 
@@ -142,6 +146,17 @@ def fp8bw_quant_act_1x128_fmt(x, mode, fmt, q_row, s_row, q_col=None, s_col=None
     _check("fp8bw_quant_act_1x128_fmt", load().fp8bw_quant_act_1x128_fmt(
         _ptr(x), M, K, x.stride(0), int(mode), int(fmt), _ptr(q_row), _ptr(s_row), _ptr(q_col),
         _ptr(s_col), _stream(stream)))
+
+
+def fp8bw_quant_tensor_delayed(x, fmt, mode, hist, q, qT, scale, amax, s_grid=None, stream=None):
+    """Per-tensor delayed scaling.  x [M, ldx] bf16; hist [H] f32 (updated);
+    q [M,K] u8; qT [K,M] u8 or None; scale, amax: 1-element f32 tensors;
+    s_grid: f32 tensor filled with the scale, or None."""
+    M, K = x.shape
+    n = s_grid.numel() if s_grid is not None else 0
+    _check("fp8bw_quant_tensor_delayed", load().fp8bw_quant_tensor_delayed(
+        _ptr(x), M, K, x.stride(0), int(fmt), int(mode), _ptr(hist), hist.numel(), _ptr(q),
+        _ptr(qT), _ptr(scale), _ptr(amax), _ptr(s_grid), n, _stream(stream)))
 
 
 def fp8bw_quant_weight_128x128(w, mode, q, s, qT=None, stream=None):

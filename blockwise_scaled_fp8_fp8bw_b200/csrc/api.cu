@@ -20,6 +20,10 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
                             int num_sms, cudaStream_t st, int out_mode, int a_fmt = 0, int b_fmt = 0);
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
+cudaError_t launch_quant_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
+                                int fmt, float* hist, int H, uint8_t* q, uint8_t* qT,
+                                float* scale, float* amax, float* s_grid, int64_t s_grid_len,
+                                int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
 extern int gemm_stall_chunk;
 }  // namespace fp8bw
@@ -32,6 +36,7 @@ int g_sms[kMaxDevices];  // 0 = not initialised, -1 = unsupported
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 // The activation quantizer writes its codes with 32-byte stores.
 inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 inline bool mult128(int64_t v) { return v >= 0 && (v & 127) == 0; }
 constexpr int64_t kMaxDim = int64_t(1) << 30;  // sizes index with 32-bit tile math
 
@@ -297,6 +302,31 @@ FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const vo
   if (K == 0) return from_cuda(cudaMemset2DAsync(D, ldd * 2, 0, N * 2, M, reinterpret_cast<cudaStream_t>(stream)));
   return from_cuda(fp8bw::launch_gemm_bf16(M, N, K, A, B, D, ldd, sms,
                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                        fp8bw_format fmt, fp8bw_scale_mode mode, float* hist,
+                                        int32_t H, uint8_t* q, uint8_t* qT, float* scale,
+                                        float* amax, float* s_grid, int64_t s_grid_len,
+                                        fp8bw_stream_t stream) {
+  if (fmt != FP8BW_FMT_E4M3 && fmt != FP8BW_FMT_E5M2) return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (!hist || !scale || !amax) return FP8BW_ERR_INVALID_ARG;
+  if (M != 0 && K != 0 && (!x || !q)) return FP8BW_ERR_INVALID_ARG;  // empty: nothing to touch
+  if (H < 1 || H > FP8BW_MAX_HISTORY) return FP8BW_ERR_INVALID_ARG;
+  if (s_grid_len < 0 || (s_grid_len > 0 && !s_grid)) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || K < 0 || ldx < K) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(K) || (ldx & 15) != 0) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned32(x) || !aligned32(q) || (qT && !aligned32(qT)) || !aligned4(hist) ||
+      !aligned4(scale) || !aligned4(amax) || (s_grid && !aligned4(s_grid)))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  return from_cuda(fp8bw::launch_quant_tensor(x, M, K, ldx, mode, fmt, hist, H, q, qT, scale, amax,
+                                              s_grid_len > 0 ? s_grid : nullptr, s_grid_len, sms,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

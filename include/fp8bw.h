@@ -248,6 +248,41 @@ FP8BW_API fp8bw_status fp8bw_grouped_wgrad_f32(int32_t G, const int32_t* d_offse
 FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, fp8bw_stream_t stream);
 
+/* Per-tensor delayed scaling, the comparison recipe of "FP8
+ * Trainingsinfrastructuur" (sections "Transformer Engine: de softwarebasis":
+ * a history of 16 amax values, the "max" rule, margin 0, E4M3 forward and
+ * E5M2 backward; "Scaling-strategieën en stabiliteit": one scale per tensor,
+ * chosen from earlier iterations so that no reduction over the current
+ * tensor precedes its quantization).
+ *   x        [M][ldx] bf16, row-major; the first K columns are quantized.
+ *   hist     [H] fp32 amax history, newest first, read and updated:
+ *            s = scale rule of `fmt` and `mode` applied to max(hist)
+ *            (s = 1 while the history holds no positive value); after the
+ *            tensor is quantized hist[i] = hist[i-1] for i = H-1 .. 1 and
+ *            hist[0] = amax.  Zero-initialise it before the first call.
+ *   q        [M][K] codes, q = encode(fp32(x) / s); a tensor that outgrew its
+ *            history saturates to the format's largest value.
+ *   qT       [K][M] the byte transpose of q (one scale: the column-wise copy
+ *            the weight gradient reads), or NULL.
+ *   scale    one fp32, the s this call used.
+ *   amax     one fp32, max |x| of this call (NaN elements are ignored).
+ *   s_grid   NULL, or s_grid_len fp32 values all set to s: a constant scale
+ *            grid, so that (q, s_grid) or (qT, s_grid) feed the blockwise
+ *            GEMMs (fp8bw_gemm, fp8bw_gemm_fmt) as an operand whose every
+ *            block carries s.  A grid of M*K/128 values serves both
+ *            activation layouts; a weight needs N*K/16384.
+ * All outputs are device memory; hist, scale, amax and s_grid must not
+ * overlap each other or the tensors.  An empty tensor (M or K zero; x, q,
+ * qT may then be NULL) still sets scale, amax = 0, s_grid and the history.  Requires M, K multiples of 128,
+ * ldx >= K and a multiple of 16, x, q and qT 32-byte aligned,
+ * 1 <= H <= FP8BW_MAX_HISTORY. */
+#define FP8BW_MAX_HISTORY 1024
+FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                        fp8bw_format fmt, fp8bw_scale_mode mode, float* hist,
+                                        int32_t H, uint8_t* q, uint8_t* qT, float* scale,
+                                        float* amax, float* s_grid, int64_t s_grid_len,
+                                        fp8bw_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,7 @@ def test_header_declares_the_calls():
     names = _declared()
     for n in ["fp8bw_quant_act_1x128", "fp8bw_quant_weight_128x128", "fp8bw_requant_weights",
               "fp8bw_gemm", "fp8bw_grouped_gemm", "fp8bw_gemm_bf16", "fp8bw_init",
-              "fp8bw_status_string", "fp8bw_last_device_error"]:
+              "fp8bw_status_string", "fp8bw_last_device_error", "fp8bw_quant_tensor_delayed"]:
         assert n in names
 
 
@@ -92,6 +92,23 @@ def test_host_validation(lib):
     d[1] = lib.fp8bw_weight_desc(0x10000, 128, 136, 136, 0x10000, 0x10000, None)
     assert r.fp8bw_requant_weights(d, 2, 0, N) == 2
     assert r.fp8bw_requant_weights(None, 1, 0, N) == 1
+    # per-tensor delayed scaling: formats, history length, 32-byte operands,
+    # ldx a multiple of 16, a grid length needs a grid
+    q32, p16 = ctypes.c_void_p(0x10020), ctypes.c_void_p(0x10010)
+    dl = r.fp8bw_quant_tensor_delayed
+    assert dl(N, 128, 128, 128, 0, 0, p, 16, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 2, 0, p, 16, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 0, 2, p, 16, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 0, 0, p, 0, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 0, 0, p, 1025, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 0, 0, N, 16, q32, N, p, p, N, 0, N) == 1
+    assert dl(p, 128, 128, 128, 0, 0, p, 16, q32, N, p, p, N, 64, N) == 1
+    assert dl(p, 130, 128, 128, 0, 0, p, 16, q32, N, p, p, N, 0, N) == 2
+    assert dl(p, 128, 128, 136, 0, 0, p, 16, q32, N, p, p, N, 0, N) == 2
+    assert dl(p16, 128, 128, 128, 0, 0, p, 16, q32, N, p, p, N, 0, N) == 2
+    assert dl(p, 128, 128, 128, 0, 0, p, 16, p16, N, p, p, N, 0, N) == 2
+    assert dl(p, 128, 128, 128, 0, 0, p, 16, q32, p16, p, p, N, 0, N) == 2
+    assert dl(p, 128, 128, 128, 0, 0, ctypes.c_void_p(0x10002), 16, q32, N, p, p, N, 0, N) == 2
     # testing hook: only chunk >= -1 is accepted; -1 cancels
     assert r.fp8bw_testing_stall_next_gemm(-2) == 1
     assert r.fp8bw_testing_stall_next_gemm(-1) == 0
