@@ -9,7 +9,8 @@
 // A call is three stream-ordered steps: a 4-byte memset of the amax output,
 // k_quant_tensor, and k_push_history.
 //
-// k_quant_tensor (256 threads; a grid-stride loop over 128x128 tiles of x):
+// k_quant_tensor (256 threads, 4 CTAs per SM; a grid-stride loop over
+// 128x128 tiles of x):
 //  * every CTA derives the scale itself from the H history entries, so no
 //    launch has to wait for another;
 //  * phase 1: a thread reads 32 consecutive bf16 of rows r and r+64 with two
@@ -147,6 +148,10 @@ cudaError_t launch_t(const void* x, int64_t M, int64_t K, int64_t ldx, float* hi
   int occ = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0);
   if (e != cudaSuccess) return e;
+  // Four resident CTAs per SM stream best on B200 (measured over 1-6 on the
+  // [8192, 28672] tensor: five or six CTAs per SM were 15-30 % slower, and
+  // prefetching the next tile into registers did not help either).
+  if (occ > 4) occ = 4;
   if (occ < 1) occ = 1;
   const int64_t tiles = (M / kTile) * (K / kTile);
   int64_t grid = (int64_t)num_sms * occ;
