@@ -14,10 +14,8 @@
 //  * every CTA derives the scale itself from the H history entries, so no
 //    launch has to wait for another;
 //  * phase 1: a thread reads 32 consecutive bf16 of rows r and r+64 with two
-//    32-byte loads each, converts them with the one scale (two multiplies
-//    and a bracket test per element instead of a division, see codes2),
-//    writes their 32 codes as one 32-byte store per row, and parks them in a
-//    shared tile;
+//    32-byte loads each, converts them with the one scale, writes their 32
+//    codes as one 32-byte store per row, and parks them in a shared tile;
 //  * phase 2 (transposed copy): a thread gathers two columns over 32 rows from
 //    the shared tile, 16 bits per row, regroups the bytes with byte permutes
 //    and writes each column's 32 codes as one 32-byte store.  With a single
@@ -49,50 +47,18 @@ __device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&r)[8]) {
                : "l"(p));
 }
 
-// Codes of x/s for two elements.  POW2: x * (1/s), exact.  FP32: the scale
-// is an arbitrary float (any history value), so the codes are bracketed
-// rather than divided (the rounding test of A. Ziv, ACM TOMS 17(3), 1991):
-// with y_lo < 1/s < y_hi as real numbers, x*y_lo, x/s and x*y_hi are ordered
-// and RN and the saturating conversion are monotone, so when the codes of
-// RN(x*y_lo) and RN(x*y_hi) agree they are the code of RN(x/s); otherwise
-// (a rounding boundary within 2^-20 relative, or a scale outside the range
-// where y_lo, y_hi are set, see scale_bracket) the elements are divided.
-template <int MODE, int FMT>
-__device__ __forceinline__ uint32_t codes2(float a, float b, float s, float inv, float ylo,
-                                           float yhi) {
-  if (MODE == FP8BW_SCALE_POW2) return cvt_fp8x2<FMT>(__fmul_rn(a, inv), __fmul_rn(b, inv));
-  const uint32_t lo = cvt_fp8x2<FMT>(__fmul_rn(a, ylo), __fmul_rn(b, ylo));
-  const uint32_t hi = cvt_fp8x2<FMT>(__fmul_rn(a, yhi), __fmul_rn(b, yhi));
-  if (lo == hi) return lo;
-  return cvt_fp8x2<FMT>(__fdiv_rn(a, s), __fdiv_rn(b, s));
-}
-
-// y_lo = RN(y(1 - 2^-20)) and y_hi = RN(y(1 + 2^-20)) with y = RN(1/s): for
-// s in [2^-125, 2^125] all three are normal, |y - 1/s| <= 2^-24/s, and the
-// 2^-20 step dominates the two roundings, so y_lo < 1/s < y_hi.  Outside
-// that range y_lo = 0, y_hi = +inf: the two codes then differ for every
-// non-NaN x (0 against the saturated or NaN code), so every element divides.
-__device__ __forceinline__ void scale_bracket(float s, float& ylo, float& yhi) {
-  ylo = 0.0f;
-  yhi = __int_as_float(0x7f800000);
-  if (s >= 0x1p-125f && s <= 0x1p125f) {
-    const float y = __frcp_rn(s);
-    ylo = __fmul_rn(y, 1.0f - 0x1p-20f);
-    yhi = __fmul_rn(y, 1.0f + 0x1p-20f);
-  }
-}
-
 // 16 bf16 (one 32-byte load) -> 16 codes in 4 words; updates the |x| maximum.
 template <int MODE, int FMT>
-__device__ __forceinline__ void convert16(const uint32_t (&w)[8], float s, float inv, float ylo,
-                                          float yhi, float& amax, uint32_t* out) {
+__device__ __forceinline__ void convert16(const uint32_t (&w)[8], float s, float inv,
+                                          float& amax, uint32_t* out) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float a = bf16lo(w[2 * i]), b = bf16hi(w[2 * i]);
     const float c = bf16lo(w[2 * i + 1]), d = bf16hi(w[2 * i + 1]);
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d))));
-    out[i] = codes2<MODE, FMT>(a, b, s, inv, ylo, yhi) |
-             (codes2<MODE, FMT>(c, d, s, inv, ylo, yhi) << 16);
+    const uint32_t lo = cvt_fp8x2<FMT>(scale_div<MODE>(a, s, inv), scale_div<MODE>(b, s, inv));
+    const uint32_t hi = cvt_fp8x2<FMT>(scale_div<MODE>(c, s, inv), scale_div<MODE>(d, s, inv));
+    out[i] = lo | (hi << 16);
   }
 }
 
@@ -109,8 +75,6 @@ __global__ void __launch_bounds__(256) k_quant_tensor(
   for (int i = 0; i < H; ++i) h = fmaxf(h, __ldg(hist + i));
   const float s = block_scale<MODE, FMT>(h);
   const float inv = scale_inv<MODE>(s);
-  float ylo, yhi;
-  scale_bracket(s, ylo, yhi);
   if (blockIdx.x == 0 && tid == 0) *scale_out = s;
   for (int64_t i = (int64_t)blockIdx.x * 256 + tid; i < s_grid_len; i += (int64_t)gridDim.x * 256)
     s_grid[i] = s;
@@ -133,8 +97,8 @@ __global__ void __launch_bounds__(256) k_quant_tensor(
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       uint32_t c[8];
-      convert16<MODE, FMT>(v[2 * hh], s, inv, ylo, yhi, amax, c);
-      convert16<MODE, FMT>(v[2 * hh + 1], s, inv, ylo, yhi, amax, c + 4);
+      convert16<MODE, FMT>(v[2 * hh], s, inv, amax, c);
+      convert16<MODE, FMT>(v[2 * hh + 1], s, inv, amax, c + 4);
       const int row = r + 64 * hh;
       st_global_v8(q + (m0 + row) * K + k0 + 32 * seg, make_uint4(c[0], c[1], c[2], c[3]),
                    make_uint4(c[4], c[5], c[6], c[7]));

@@ -77,9 +77,7 @@ def test_shapes_rowwise_only_and_edges(fb, orc, fmt):
     x[5, 200] = -2.0 ** -133
     x = x.to(torch.bfloat16)
     x[200:, :64] = -0.0
-    # 1e-37 makes the FP32 scale subnormal (every element divides); 1.06e-35
-    # puts it just above 2^-125, the edge of the bracketed range
-    for h in ([0.0], [1e-30], [3e38], [7.0, float("nan")], [1e-37], [1.06e-35]):
+    for h in ([0.0], [1e-30], [3e38], [7.0, float("nan")]):
         hist_cpu = np.array(h, np.float32)
         check_step(fb, orc, x, fmt, 0, torch.from_numpy(hist_cpu.copy()).to(DEV), hist_cpu)
         check_step(fb, orc, x, fmt, 1, torch.from_numpy(hist_cpu.copy()).to(DEV), hist_cpu)
