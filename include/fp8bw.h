@@ -272,10 +272,15 @@ FP8BW_API fp8bw_status fp8bw_gemm_bf16(int64_t M, int64_t N, int64_t K, const vo
  *            block carries s.  A grid of M*K/128 values serves both
  *            activation layouts; a weight needs N*K/16384.
  * All outputs are device memory; hist, scale, amax and s_grid must not
- * overlap each other or the tensors.  An empty tensor (M or K zero; x, q,
- * qT may then be NULL) still sets scale, amax = 0, s_grid and the history.  Requires M, K multiples of 128,
- * ldx >= K and a multiple of 16, x, q and qT 32-byte aligned,
- * 1 <= H <= FP8BW_MAX_HISTORY. */
+ * overlap each other or the tensors.  The history is read and rewritten in
+ * stream order (a 4-byte memset of amax, the quantizing kernel, a one-thread
+ * history push), so calls that share a history must be ordered: the same
+ * stream, or events between streams.  An empty tensor (M or K zero; x, q,
+ * qT may then be NULL) still sets scale, amax = 0, s_grid and the history.
+ * Requires M, K multiples of 128, ldx >= K and a multiple of 16, x, q and qT
+ * 32-byte aligned, hist, scale, amax, s_grid 4-byte aligned,
+ * 1 <= H <= FP8BW_MAX_HISTORY; else FP8BW_ERR_INVALID_ARG or
+ * FP8BW_ERR_ALIGNMENT, with nothing launched. */
 #define FP8BW_MAX_HISTORY 1024
 FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int64_t K, int64_t ldx,
                                         fp8bw_format fmt, fp8bw_scale_mode mode, float* hist,
