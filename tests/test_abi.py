@@ -112,3 +112,28 @@ def test_host_validation(lib):
     # testing hook: only chunk >= -1 is accepted; -1 cancels
     assert r.fp8bw_testing_stall_next_gemm(-2) == 1
     assert r.fp8bw_testing_stall_next_gemm(-1) == 0
+
+
+def _param_counts():
+    """Parameter count of every FP8BW_API function in the header."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"FP8BW_API\s+[\w\s\*]+?\b(fp8bw_\w+)\s*\(([^)]*)\)", src):
+        params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_argtypes_match_the_header(lib):
+    """The ctypes binding declares, for every call it wraps, as many arguments
+    as the header's prototype has (a drifted wrapper would shift arguments)."""
+    raw = lib.load()
+    counts = _param_counts()
+    checked = 0
+    for name, n in counts.items():
+        fn = getattr(raw, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        checked += 1
+    assert checked >= 14
