@@ -25,12 +25,20 @@ against the fp64 product of the bf16 operands.
 Run ``python -m oracle.quant_error`` for the table of the Llama-3.1-8B-like
 layers (config of 8192-token layers, sampled at 1024 tokens) and the packed
 Student-t batch.
+
+A second table follows one activation tensor over training steps whose
+magnitude drifts, for the delayed per-tensor recipe of the same page
+(section "Transformer Engine: de softwarebasis": a history of 16 amax
+values, the "max" rule): its scale comes from earlier steps, so a tensor
+that grows saturates and, after a spike, the inflated history wastes
+dynamic range until the spike leaves the window.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from . import MODE_FP32, MODE_POW2, e4m3_decode, e4m3_encode_array, quant_act_1x128, quant_weight_128x128
+from . import (MODE_FP32, MODE_POW2, e4m3_decode, e4m3_encode_array, quant_act_1x128,
+               quant_tensor_delayed, quant_weight_128x128)
 
 _TABLE = None
 
@@ -140,6 +148,45 @@ def study(tokens: int = 1024, seed: int = 0) -> list:
     return rows
 
 
+def dq_delayed(bits: np.ndarray, hist: np.ndarray):
+    """Per-tensor delayed scaling (E4M3, fp32 scale) of a bf16 tensor with the
+    given history.  Returns (dequantized tensor, new history, fraction of
+    elements at the saturated code)."""
+    q, _, s, _, h = quant_tensor_delayed(bits, hist, MODE_FP32, transposed=False)
+    sat = float(np.mean((q & 0x7F) == 0x7E))
+    return decode_table()[q] * np.float64(s), h, sat
+
+
+def magnitude_schedule(steps: int = 40) -> list:
+    """Per-step magnitude of the drifting tensor: 3 % growth per step, one
+    4x spike at step 12, back on the trend after it."""
+    return [1.03 ** t * (4.0 if t == 12 else 1.0) for t in range(steps)]
+
+
+def delayed_study(tokens: int = 256, seed: int = 0, history: int = 16, schedule=None) -> list:
+    """Rows of (step, magnitude, errors) for the o_proj input (with the
+    workloads' outlier channels) scaled by `schedule` (default
+    `magnitude_schedule()`): blockwise (current 1x128 scales), per-tensor
+    current scaling, and per-tensor delayed scaling with a `history`-long
+    amax history (zero at step 0)."""
+    import torch
+
+    import workloads
+
+    X, _, _ = workloads.llama_layer("o_proj", seed=seed, M=tokens)
+    base = X.float()
+    hist = np.zeros(history, np.float32)
+    rows = []
+    for t, m in enumerate(magnitude_schedule() if schedule is None else schedule):
+        xb = (base * m).to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+        x = bf16_bits_to_f32(xb)
+        dq, hist, sat = dq_delayed(xb, hist)
+        rows.append((t, m, {"blockwise": rel_err(x, dq_blockwise_act(xb, MODE_FP32)),
+                            "tensor": rel_err(x, dq_tensor(x)),
+                            "delayed": rel_err(x, dq), "saturated": sat}))
+    return rows
+
+
 def main():
     rows = study()
     print("| tensor | blockwise (fp32 s) | blockwise (pow2 s) | per-tensor | MX-32 (floor) | "
@@ -149,6 +196,13 @@ def main():
         red = 1.0 - e["blockwise"] / e["tensor"]
         print(f"| {name} | {e['blockwise']:.4f} | {e['blockwise_pow2']:.4f} | {e['tensor']:.4f} | "
               f"{e['mx32']:.4f} | {e['mx32_up']:.4f} | {100 * red:.0f} % lower |")
+    print()
+    print("| step | magnitude | blockwise | per-tensor (current) | per-tensor (delayed, 16) | "
+          "saturated (delayed) |")
+    print("|---|---|---|---|---|---|")
+    for t, m, e in delayed_study():
+        print(f"| {t} | {m:.2f} | {e['blockwise']:.4f} | {e['tensor']:.4f} | {e['delayed']:.4f} | "
+              f"{100 * e['saturated']:.3f} % |")
 
 
 if __name__ == "__main__":

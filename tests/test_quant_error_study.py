@@ -62,3 +62,33 @@ def test_block_scaling_beats_per_tensor_on_outlier_activations():
     assert e["blockwise"] < 0.7 * e["tensor"]          # at least 30 % lower
     y = qe.gemm_errors(xb, wb, 128, 256)
     assert y["blockwise"] < y["tensor"]
+
+
+def test_delayed_scaling_on_a_constant_tensor_is_current_scaling():
+    # the same tensor every step: from step 1 on the history's maximum is the
+    # tensor's own amax, so delayed and current per-tensor scaling coincide
+    rows = qe.delayed_study(tokens=128, history=4, schedule=[1.0, 1.0, 1.0])
+    for _, _, e in rows[1:]:
+        assert e["delayed"] == e["tensor"] and e["saturated"] < 1e-4
+
+
+def test_delayed_scaling_first_step_uses_unit_scale():
+    # zero history: s = 1, so the codes are the plain E4M3 encodings of x
+    X, _, _ = workloads.llama_layer("o_proj", seed=0, M=128)
+    xb = bits(X)
+    dq, h, _ = qe.dq_delayed(xb, np.zeros(4, np.float32))
+    x = qe.bf16_bits_to_f32(xb)
+    plain = qe.decode_table()[qe.e4m3_encode_array(np.ascontiguousarray(x))]
+    assert np.array_equal(dq, plain)
+    assert h[0] == np.abs(x).max() and np.all(h[1:] == 0)
+
+
+def test_delayed_scaling_spike_saturates_then_recovers():
+    # a 4x spike after steady steps: the delayed scale lags, the outlier
+    # channels saturate and the error jumps; on the next step (back to the
+    # old magnitude, history inflated by the spike) it is back near current
+    # scaling, since E4M3's relative spacing does not depend on the scale
+    rows = qe.delayed_study(tokens=128, history=4, schedule=[1.0, 1.0, 4.0, 1.0, 1.0])
+    spike, after = rows[2][2], rows[3][2]
+    assert spike["saturated"] > 0 and spike["delayed"] > 5 * spike["tensor"]
+    assert after["delayed"] < 1.1 * after["tensor"]
