@@ -37,8 +37,9 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (MODE_FP32, MODE_POW2, e4m3_decode, e4m3_encode_array, quant_act_1x128,
-               quant_tensor_delayed, quant_weight_128x128)
+from . import (FMT_E4M3, FMT_E5M2, MODE_FP32, MODE_POW2, e4m3_decode, e4m3_encode_array,
+               e5m2_decode, e5m2_encode_array, quant_act_1x128, quant_tensor_delayed,
+               quant_weight_128x128)
 
 _TABLE = None
 
@@ -148,6 +149,66 @@ def study(tokens: int = 1024, seed: int = 0) -> list:
     return rows
 
 
+_TABLE5 = None
+
+
+def decode_table_e5m2() -> np.ndarray:
+    """fp64 value of each of the 256 E5M2 codes."""
+    global _TABLE5
+    if _TABLE5 is None:
+        _TABLE5 = np.array([e5m2_decode(c) for c in range(256)], np.float64)
+    return _TABLE5
+
+
+def dq_blockwise_act_fmt(bits: np.ndarray, fmt: int) -> np.ndarray:
+    """Dequantized 1x128 row blocks (fp32 scale) in E4M3 or E5M2."""
+    q, s, _, _ = quant_act_1x128(bits, MODE_FP32, colwise=False, fmt=fmt)
+    table = decode_table_e5m2() if fmt == FMT_E5M2 else decode_table()
+    return table[q] * np.repeat(s.T.astype(np.float64), 128, axis=1)
+
+
+def dq_tensor_fmt(x: np.ndarray, fmt: int) -> np.ndarray:
+    """One fp32 scale amax/Q for the whole tensor, Q = 448 (E4M3) or 57344
+    (E5M2)."""
+    if fmt == FMT_E4M3:
+        return dq_tensor(x)
+    amax = np.float32(np.max(np.abs(x)))
+    s = np.float32(amax / np.float32(57344.0)) if amax > 0 else np.float32(1.0)
+    codes = e5m2_encode_array(np.ascontiguousarray((x / s).astype(np.float32)))
+    return decode_table_e5m2()[codes] * np.float64(s)
+
+
+def gradient_study(tokens: int = 256, seed: int = 0, cols: int = 512) -> list:
+    """Rows of (layer, errors) for the gradient dY [tokens, N] of each
+    Llama-like layer in four encodings (E4M3 / E5M2, 1x128 blocks / one
+    scale per tensor, fp32 scales), and for the data gradient
+    dX[:, :cols] = dY W[:, :cols] with W in 128x128 E4M3 blocks."""
+    import torch
+
+    import workloads
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    rows = []
+    for name, K, N in workloads.LLAMA8B_LAYERS:
+        _, W, dY = workloads.llama_layer(name, seed=seed, M=tokens)
+        db = bits(dY)
+        d = bf16_bits_to_f32(db)
+        w = bf16_bits_to_f32(bits(W))[:, :cols].astype(np.float64)
+        wq = dq_blockwise_weight(bits(W[:, :cols]), MODE_FP32)
+        ref = d.astype(np.float64) @ w
+        e = {}
+        for key, dq in [("block_e4m3", dq_blockwise_act_fmt(db, FMT_E4M3)),
+                        ("block_e5m2", dq_blockwise_act_fmt(db, FMT_E5M2)),
+                        ("tensor_e4m3", dq_tensor_fmt(d, FMT_E4M3)),
+                        ("tensor_e5m2", dq_tensor_fmt(d, FMT_E5M2))]:
+            e[key] = rel_err(d, dq)
+            e["dX_" + key] = rel_err(ref, dq @ wq)
+        rows.append((f"{name} dY [{tokens},{N}]", e))
+    return rows
+
+
 def dq_delayed(bits: np.ndarray, hist: np.ndarray):
     """Per-tensor delayed scaling (E4M3, fp32 scale) of a bf16 tensor with the
     given history.  Returns (dequantized tensor, new history, fraction of
@@ -196,6 +257,14 @@ def main():
         red = 1.0 - e["blockwise"] / e["tensor"]
         print(f"| {name} | {e['blockwise']:.4f} | {e['blockwise_pow2']:.4f} | {e['tensor']:.4f} | "
               f"{e['mx32']:.4f} | {e['mx32_up']:.4f} | {100 * red:.0f} % lower |")
+    print()
+    print("| gradient | 1x128 E4M3 | 1x128 E5M2 | tensor E4M3 | tensor E5M2 | dX: 1x128 E4M3 | "
+          "dX: 1x128 E5M2 | dX: tensor E4M3 | dX: tensor E5M2 |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for name, e in gradient_study():
+        print(f"| {name} | {e['block_e4m3']:.4f} | {e['block_e5m2']:.4f} | {e['tensor_e4m3']:.4f} | "
+              f"{e['tensor_e5m2']:.4f} | {e['dX_block_e4m3']:.4f} | {e['dX_block_e5m2']:.4f} | "
+              f"{e['dX_tensor_e4m3']:.4f} | {e['dX_tensor_e5m2']:.4f} |")
     print()
     print("| step | magnitude | blockwise | per-tensor (current) | per-tensor (delayed, 16) | "
           "saturated (delayed) |")

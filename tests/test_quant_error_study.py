@@ -92,3 +92,23 @@ def test_delayed_scaling_spike_saturates_then_recovers():
     spike, after = rows[2][2], rows[3][2]
     assert spike["saturated"] > 0 and spike["delayed"] > 5 * spike["tensor"]
     assert after["delayed"] < 1.1 * after["tensor"]
+
+
+def test_e5m2_per_tensor_on_one_block_equals_blockwise():
+    g = torch.Generator().manual_seed(6)
+    x = (torch.randn((1, 128), generator=g) * 1e-3).to(torch.bfloat16)
+    b = bits(torch.cat([x] * 128))
+    xf = qe.bf16_bits_to_f32(b)
+    assert np.array_equal(qe.dq_tensor_fmt(xf[:1], qe.FMT_E5M2),
+                          qe.dq_blockwise_act_fmt(b, qe.FMT_E5M2)[:1])
+
+
+def test_e5m2_gradient_error_is_twice_e4m3():
+    # one mantissa bit fewer doubles the grid spacing, hence the relative
+    # rounding error of values in the normal range
+    _, _, dY = workloads.llama_layer("o_proj", seed=0, M=128)
+    db = bits(dY)
+    d = qe.bf16_bits_to_f32(db)
+    e4 = qe.rel_err(d, qe.dq_blockwise_act_fmt(db, qe.FMT_E4M3))
+    e5 = qe.rel_err(d, qe.dq_blockwise_act_fmt(db, qe.FMT_E5M2))
+    assert 1.8 < e5 / e4 < 2.2
