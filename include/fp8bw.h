@@ -21,7 +21,9 @@
  *    with fp8bw_last_device_error().
  *  - Shapes: M, N, K are multiples of 128 (else FP8BW_ERR_ALIGNMENT), and
  *    every pointer is 16-byte aligned with leading dimensions that keep rows
- *    16-byte aligned.  Invalid arguments never reach the GPU.
+ *    16-byte aligned (32-byte where a call says so: the activation
+ *    quantizers' code outputs, the per-tensor quantizer's input and codes).
+ *    Invalid arguments never reach the GPU.
  *  - bf16 tensors are IEEE bfloat16 bit patterns; E4M3 codes are bytes
  *    (sign | 4-bit exponent field, bias 7 | 3-bit mantissa; 0x7F/0xFF NaN).
  *  - Scale rule (identical in every quantizer): amax = max |x| over the block;
