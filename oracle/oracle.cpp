@@ -338,6 +338,24 @@ static double b_scale(int kind, const float* sB, int64_t N, int64_t K,
   return sB[kb * N + n];
 }
 
+// The decoded value of every code of one format, taken from the decoder
+// above once (a lookup saves the per-product decode in the GEMM references;
+// the values are the decoder's own).
+struct DecodeTable {
+  double v[2][256];
+  DecodeTable() {
+    for (int c = 0; c < 256; ++c) {
+      v[FMT_E4M3][c] = e4m3_decode(static_cast<uint8_t>(c));
+      v[FMT_E5M2][c] = e5m2_decode(static_cast<uint8_t>(c));
+    }
+  }
+};
+
+static const double* decode_table(int fmt) {
+  static const DecodeTable t;  // initialised once, thread-safe
+  return t.v[fmt == FMT_E5M2 ? FMT_E5M2 : FMT_E4M3];
+}
+
 // One output element of the GEMM reference over K-chunks [kb0, kb1):
 // sum_k (qA[m][k] * sA[k/128][m]) * (qB[n][k] * sB(n, k/128)) in fp64 from
 // the dequantized operands, and sum_k |a * b|.
@@ -347,14 +365,16 @@ static void ref_element(int kind, int64_t M, int64_t N, int64_t K,
                         const float* sB, int64_t kb0, int64_t kb1, int64_t m,
                         int64_t n, double* y, double* yabs, int fa = FMT_E4M3,
                         int fb = FMT_E4M3) {
+  const double* da = decode_table(fa);
+  const double* db = decode_table(fb);
   double acc = 0.0, aacc = 0.0;
   for (int64_t kb = kb0; kb < kb1; ++kb) {
     double sa = sA[kb * M + m];
     double sb = b_scale(kind, sB, N, K, n, kb);
     for (int64_t j = 0; j < 128; ++j) {
       int64_t k = kb * 128 + j;
-      double a = decode(A[m * K + k], fa) * sa;
-      double b = decode(B[n * K + k], fb) * sb;
+      double a = da[A[m * K + k]] * sa;
+      double b = db[B[n * K + k]] * sb;
       acc += a * b;
       aacc += std::fabs(a * b);
     }
@@ -409,6 +429,7 @@ void orc_grouped_gemm_ref_tile(int kind, int32_t G, const int32_t* off,
   if (kind == 2) {
     // GEMM dims: rows N, cols K, contraction Mtot.
     int64_t kb0 = off[expert] / 128, kb1 = off[expert + 1] / 128;
+#pragma omp parallel for schedule(static)
     for (int64_t m = m0; m < m1; ++m)
       for (int64_t n = n0; n < n1; ++n)
         ref_element(2, N, K, Mtot, A, sA, B, sB, kb0, kb1, m, n,
@@ -416,6 +437,7 @@ void orc_grouped_gemm_ref_tile(int kind, int32_t G, const int32_t* off,
                     &yabs[(m - m0) * W + (n - n0)]);
     return;
   }
+#pragma omp parallel for schedule(static)
   for (int64_t m = m0; m < m1; ++m) {
     int32_t g = 0;
     while (g < G && !(m >= off[g] && m < off[g + 1])) ++g;
