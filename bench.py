@@ -46,6 +46,7 @@ def parse():
     p.add_argument("--mode", default="fp32", choices=["fp32", "pow2"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-steady", action="store_true", help="skip the >= 1.5 s steady-state region")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--case", default=None,
                    help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
@@ -70,18 +71,18 @@ def peaks():
 
 
 def gemm_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, or None if
-    the kernel source changed since those counters were taken."""
+    """DRAM bytes per GEMM launch from profiles/k_gemm_fp8_traffic.json (an
+    ncu capture, summarised by hand), or None if the kernel source changed
+    since those counters were taken."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "k_gemm_fp8_llama8b_step.md")
+    path = os.path.join(ROOT, "profiles", "k_gemm_fp8_traffic.json")
     src = os.path.join(ROOT, "blockwise_scaled_fp8_fp8bw_b200", "csrc", "gemm.cu")
     try:
-        text = open(prof).read()
-        want = [l.split(":", 1)[1].strip() for l in text.splitlines() if l.startswith("gemm_cu_sha256_16:")][0]
-        val = [l.split(":", 1)[1].strip() for l in text.splitlines() if l.startswith("traffic_bytes_per_launch:")][0]
+        with open(path) as f:
+            d = json.load(f)
         have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return int(val) if have == want else None
-    except (OSError, IndexError, ValueError):
+        return int(d["traffic_bytes_per_launch"]) if have == d["gemm_cu_sha256_16"] else None
+    except (OSError, KeyError, ValueError):
         return None
 
 
@@ -255,28 +256,68 @@ def _cores():
     return min(cores, int(os.environ.get("OMP_NUM_THREADS", cores)))
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_quant_timing(name="qkv"):
+    """The oracle's activation quantizer (1x128 row blocks + the column-wise
+    copy) on one full tensor of the step, X of `name` at 8192 tokens, single
+    threaded and on all host threads."""
+    import oracle
+    X, _, _ = workloads.llama_layer(name, seed=0, device="cpu")
+    xb = X.view(torch.int16).numpy().view(np.uint16)
+    M, K = xb.shape
+    nbytes = M * K * (2 + 1 + 1) + 2 * 4 * M * K // 128
+    out = {"tensor": f"X of {name} [{M},{K}] bf16, row blocks + column-wise copy, in full",
+           "bytes": nbytes}
+    allt = _cores()
+    for label, n in (("single_thread", 1), ("all_threads", allt)):
+        oracle.set_threads(n)
+        t0 = time.perf_counter()
+        oracle.quant_act_1x128(xb, 0)
+        dt = time.perf_counter() - t0
+        out[label] = {"threads": n, "s": dt, "GB/s": nbytes / dt / 1e9}
+    oracle.set_threads(allt)
+    return out
+
+
 def oracle_sample(target_s=10.0, rows=8, cols=512):
-    """Times the CPU oracle's fp64 reference GEMM on a bounded sample of the
-    step (blocks of `rows` x `cols` outputs of each layer's fprop, full K),
-    cycling through the layers until about `target_s` seconds of GEMM work."""
+    """Times the CPU oracle on the machine's host cores: its fp64 reference GEMM
+    on a bounded sample of the step (blocks of `rows` x `cols` outputs of
+    each layer's fprop, full K, cycling through the layers until about
+    `target_s` seconds of GEMM work; `value`, extrapolated per FLOP), and its
+    quantizer on one full tensor, single threaded and on all threads."""
     names = [n for n, _, _ in workloads.LLAMA8B_LAYERS]
     for n in names:
         _oracle_operands(n)
     flops = secs = 0.0
-    done = []
     i = 0
-    while secs < target_s and i < 1000:
+    while secs < target_s and i < 100000:
         n = names[i % len(names)]
         f, dt = _oracle_gemm(n, rows, cols)
         flops += f
         secs += dt
-        done.append(n)
         i += 1
+    quant = oracle_quant_timing()
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "sample": f"fp64 reference GEMM (oracle.gemm_ref_tile, fprop) on {i} blocks of "
                       f"{rows} rows x {cols} cols x full K cycling over the four layers "
                       f"({secs:.1f} s of CPU work), operands quantized by the oracle; "
-                      "TFLOP/s = 2*rows*cols*K / time"}
+                      "TFLOP/s = 2*rows*cols*K / time, extrapolated per FLOP to the step",
+            "step_s_extrapolated": sum(l_flops for l_flops in
+                                       [6 * workloads.LLAMA8B_TOKENS * N * K for _, K, N in workloads.LLAMA8B_LAYERS]
+                                       ) / (flops / secs),
+            "quant_act": quant}
 
 
 def reference_arm(args):
@@ -509,6 +550,38 @@ def main():
     timed_long = ms_total > 1000.0
     fp8_peak = 2.0 * (pk["bf16_sustained"] if timed_long else pk["bf16_burst"])
 
+    # ---- steady state: the same step timed for at least 1.5 s, so that the
+    # clock has settled under the power cap (roofline against the sustained
+    # BF16 figure)
+    steady = None
+    if not args.no_steady:
+        n_steady = max(args.steps, int(np.ceil(1500.0 / ms_step)))
+        ck2 = ClockSampler(clocks.index)
+        ck2.start()
+        time.sleep(0.3)
+        ev2 = {}
+        barrier()
+        torch.cuda.synchronize()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record()
+        for _ in range(n_steady):
+            run_step(fb, layers, mode, ev2)
+        q1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ck2s = ck2.stop()
+        q_ms = max_over_ranks(q0.elapsed_time(q1), dist, dev)
+        st = fb.fp8bw_last_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error (steady state): {fb.status_string(st)}")
+        g2_ms = sum(a.elapsed_time(b) for a, b in ev2["gemm"]) / n_steady
+        g2_tflops = step_flops / (g2_ms * 1e-3) / 1e12
+        steady = {"value": job_rate(step_flops * n_steady, world, q_ms) / 1e12, "unit": "TFLOP/s",
+                  "ms_per_step": q_ms / n_steady, "steps": n_steady, "timed_s": q_ms / 1e3,
+                  "gemm_tflops": g2_tflops, "gemm_peak": 2.0 * pk["bf16_sustained"],
+                  "gemm_frac": g2_tflops / (2.0 * pk["bf16_sustained"]),
+                  "peak_note": f"FP8 = 2 x {pk['src']} cuBLAS bf16 (sustained)", "clocks": ck2s}
+
     # ---- the same step with power-of-2 scales (block-scaled MMA path)
     pow2 = None
     if args.mode == "fp32":
@@ -639,8 +712,11 @@ def main():
                       "hbm_peak_gbs": pk["hbm_gbs"],
                       "bf16_gemm_tflops": bf16, "fp8_over_bf16": (gemm_tflops / bf16) if bf16 else None,
                       "requant_over_step": req_ms / ms_step},
+            "steady_state": steady,
             "pow2_scales": pow2,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches_note": "library kernels in the timed region (K steps x 21); the steady-state, "
+                                 "power-of-2 and e2e regions are timed separately",
             "clocks": ck,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -25,6 +25,7 @@ cudaError_t launch_quant_tensor(const void* x, int64_t M, int64_t K, int64_t ldx
                                 float* scale, float* amax, float* s_grid, int64_t s_grid_len,
                                 int num_sms, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
+cudaError_t quant_read_clear_error(uint32_t* out, cudaStream_t st);
 extern int gemm_stall_chunk;
 }  // namespace fp8bw
 
@@ -105,8 +106,11 @@ FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk) {
 }
 
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {
-  uint32_t v = 0;
-  if (fp8bw::gemm_read_clear_error(&v, stream) != cudaSuccess) return FP8BW_ERR_CUDA;
+  uint32_t v = 0, vq = 0;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (fp8bw::gemm_read_clear_error(&v, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
+  if (fp8bw::quant_read_clear_error(&vq, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
+  v |= vq;
   if (v & 1u) return FP8BW_ERR_TIMEOUT;
   if (v & 2u) return FP8BW_ERR_DEVICE_CHECK;
   return FP8BW_OK;

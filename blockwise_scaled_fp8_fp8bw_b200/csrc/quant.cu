@@ -32,6 +32,11 @@
 #include "tmap.cuh"
 
 namespace fp8bw {
+
+// Device error word of the quantizers (a bounded wait that ran out), read
+// and cleared by fp8bw_last_device_error() through quant_read_clear_error().
+__device__ uint32_t g_quant_error;
+
 namespace {
 
 constexpr int QT = 256;  // threads per tile CTA
@@ -222,7 +227,16 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
   for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
     const int cur = i & 1;
     const int64_t k0 = (int64_t)(t % nK) * 128, m0 = (int64_t)(t / nK) * 128;
-    if (!mbar_wait(smem_u32(&sm.full[cur]), (i >> 1) & 1)) return;  // bounded: never expected
+    if (!mbar_wait(smem_u32(&sm.full[cur]), (i >> 1) & 1)) {
+      // A tile load that never lands (not expected): latch the timeout and
+      // give the other buffer's load, if one was issued, a bounded chance to
+      // land before this CTA's shared memory goes away.
+      if (tid == 0) {
+        atomicOr(&g_quant_error, DEV_ERR_TIMEOUT);
+        if (t + (int)gridDim.x < tiles) (void)mbar_wait(smem_u32(&sm.full[cur ^ 1]), ((i + 1) >> 1) & 1);
+      }
+      return;
+    }
     const uint8_t* tb = &sm.buf[cur][0][0];
 
     // ---- row pass
@@ -475,6 +489,16 @@ cudaError_t launch_requant(const fp8bw_weight_desc* d, int32_t n, int mode, cuda
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t quant_read_clear_error(uint32_t* out, cudaStream_t st) {
+  uint32_t v = 0, z = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_quant_error, sizeof v, 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbolAsync(g_quant_error, &z, sizeof z, 0, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *out = v;
+  return e;
 }
 
 }  // namespace fp8bw

@@ -84,18 +84,22 @@ FP8BW_API fp8bw_status fp8bw_init(int device);
 /* Static, human-readable name of a status. */
 FP8BW_API const char* fp8bw_status_string(fp8bw_status s);
 
-/* Synchronizes `stream`, then returns (and clears) the device error word of
- * the current device: FP8BW_ERR_TIMEOUT if a kernel's bounded wait ran out,
- * FP8BW_ERR_DEVICE_CHECK if a kernel rejected its device-side arguments
- * (e.g. grouped offsets), else FP8BW_OK.  FP8BW_ERR_CUDA if the sync failed. */
+/* Synchronizes `stream`, then returns (and clears) the device error words of
+ * the current device (one for the GEMMs, one for the quantizers):
+ * FP8BW_ERR_TIMEOUT if a kernel's bounded wait ran out, FP8BW_ERR_DEVICE_CHECK
+ * if a kernel rejected its device-side arguments (grouped offsets, or
+ * FP8BW_SCALE_POW2 scales that are not powers of two), else FP8BW_OK.
+ * FP8BW_ERR_CUDA if the sync failed. */
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream);
 
-/* Testing hook for the failure path (not part of the method): the next
- * fp8bw_gemm / fp8bw_grouped_gemm launch on this host thread's process has
- * its first CTA's operand producer skip K-chunk number `chunk` (counted over
- * that CTA's tiles), so the kernel's bounded waits run out: it abandons its
- * loops within a few seconds, writes an incomplete result and latches
- * FP8BW_ERR_TIMEOUT for fp8bw_last_device_error(); the context stays usable.
+/* Testing hook for the failure path (not part of the method): the next FP8
+ * GEMM launch of the process (any fp8bw_gemm* / fp8bw_grouped_* call, from
+ * any host thread) has its first CTA's operand producer skip K-chunk number
+ * `chunk` (counted over that CTA's tiles), so the kernel's bounded waits run
+ * out: it abandons its loops within a few seconds, writes an incomplete
+ * result and latches FP8BW_ERR_TIMEOUT for fp8bw_last_device_error(); the
+ * context stays usable.  The pending stall is one process-wide value with no
+ * synchronization: set it only while no other host thread launches GEMMs.
  * chunk = -1 cancels a pending stall.  FP8BW_ERR_INVALID_ARG if chunk < -1. */
 FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk);
 
@@ -167,9 +171,13 @@ FP8BW_API fp8bw_status fp8bw_requant_weights(const fp8bw_weight_desc* descs, int
  *   B  [N][K] codes, K-major; sB as above
  *   D  [M][ldd] bf16; ldd >= N, a multiple of 8
  * `mode` states how the scales were made; FP8BW_SCALE_POW2 promises exact
- * powers of two (the kernel may then fold them into the tensor-core MMA).
+ * powers of two in [2^-127, 2^127] (the kernel then folds them into the
+ * tensor-core MMA as UE8M0 scale factors).  A POW2 scale that is not a power
+ * of two latches FP8BW_ERR_DEVICE_CHECK and leaves D undefined (written with
+ * the scale's exponent only).
  * The result is within |D - ref| <= 1e-2 * sum_k |a_k b_k| + 1 bf16 ulp(ref)
- * of the fp64 product of the dequantized operands. */
+ * of the fp64 product of the dequantized operands.  K = 0 writes exact zeros;
+ * M = 0 or N = 0 does nothing. */
 FP8BW_API fp8bw_status fp8bw_gemm(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
                         const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                         void* D, int64_t ldd, fp8bw_scale_mode mode, fp8bw_stream_t stream);
@@ -224,7 +232,10 @@ FP8BW_API fp8bw_status fp8bw_gemm_f32(fp8bw_gemm_kind kind, int64_t M, int64_t N
  *                B = q_col(X)  [K][M_total_pad], sB [M_total_pad/128][K];
  *                D [G][N][K]: expert g contracts only its own tokens; an
  *                expert with no tokens gets exact zeros.
- * Requires G <= FP8BW_MAX_EXPERTS. */
+ * Requires G <= FP8BW_MAX_EXPERTS.  FPROP/DGRAD with K = 0 return
+ * FP8BW_ERR_INVALID_ARG (the routed rows are known only on the device, so
+ * the host cannot zero them); M_total_pad = 0 or N = 0 does nothing, and
+ * WGRAD with N = 0 or K = 0 does nothing.  Scales as in fp8bw_gemm. */
 #define FP8BW_MAX_EXPERTS 512
 FP8BW_API fp8bw_status fp8bw_grouped_gemm(fp8bw_gemm_kind kind, int32_t G, const int32_t* d_offsets,
                                 int64_t M_total_pad, int64_t N, int64_t K,

@@ -87,6 +87,8 @@ def lib():
         L.orc_bf16_ulp.restype = dbl
         L.orc_check_tol.argtypes = [vp, vp, vp, i64, dbl, vp]
         L.orc_check_tol.restype = i64
+        L.orc_set_threads.argtypes = [i32]
+        L.orc_max_threads.restype = i32
         _lib = L
     return _lib
 
@@ -107,6 +109,15 @@ def _f32(a):
     a = np.ascontiguousarray(a)
     assert a.dtype == np.float32, a.dtype
     return a
+
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops (for timing; results do not depend on it)."""
+    lib().orc_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().orc_max_threads())
 
 
 # ----------------------------------------------------------------- scalars --

@@ -41,6 +41,7 @@
 #include <cstdint>
 #include <cstring>
 #include <cstdlib>
+#include <omp.h>
 
 namespace {
 
@@ -189,6 +190,11 @@ uint8_t quant_one(uint16_t xb, float s, int fmt = FMT_E4M3) {
 }  // namespace
 
 extern "C" {
+
+// Thread count of the OpenMP loops below (timing of the CPU baseline only;
+// no value depends on it).
+void orc_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+int orc_max_threads() { return omp_get_max_threads(); }
 
 double orc_e4m3_decode(uint8_t code) { return e4m3_decode(code); }
 uint8_t orc_e4m3_encode(float v) { return e4m3_encode(v); }

@@ -1,15 +1,20 @@
-"""Full-size GPU parity, in the launch configurations the benchmark uses.
+"""Full-size GPU parity, in the launch configurations the benchmark uses, in
+both scale modes (FP32 scales on the promotion kernel, power-of-2 scales on
+the tensor core's block-scaled MMA).
 
 Workloads (seeded, synthetic, shaped like the pages' models — "NVIDIA NeMo
-RL erreicht 48% ...": Llama 3.1 8B; "NeMo-RL v0.3 mit Megatron-Core ...":
-sequence packing, 16K-token contexts):
+RL erreicht 48% ...": Llama 3.1 8B, scales recalibrated every step,
+optional power-of-2 scales; "NeMo-RL v0.3 mit Megatron-Core ...": sequence
+packing, 16K-token contexts):
   * Llama-3.1-8B-like linear layers, 8192 tokens, 0.1% outlier channels x50;
-  * the per-step requant sweep of 32 layers of those weights (Adam-like
-    N(0, 1e-4^2) update, 10 steps);
   * a packed long-sequence batch (4 sequences, 32768 tokens, Student-t
-    activations, zero-padding blocks).
+    activations, zero padding rows) on all four layer shapes;
+  * the per-step requant sweep of 32 layers of those weights (Adam-like
+    N(0, 1e-4^2) update, 10 steps).
 The oracle recomputes sampled 128x128 quantizer tiles (bit-exact) and
-sampled 32x32 GEMM output tiles (tolerance) one by one."""
+sampled 128x128 GEMM output tiles (tolerance) one by one: the four corner
+tiles, 16 seeded random tiles, tiles over outlier channels and tiles over
+zero padding rows, for every GEMM."""
 import numpy as np
 import pytest
 import torch
@@ -19,6 +24,8 @@ from util import act_buffers, assert_bytes_equal, bits, weight_buffers
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+T = 128          # side of a sampled tile
+N_RANDOM = 16    # seeded random GEMM tiles per GEMM
 
 
 def np_u8(t):
@@ -27,7 +34,6 @@ def np_u8(t):
 
 def check_act_tiles(orc, x, q_row, s_row, q_col, s_col, tiles, mode=0):
     """Oracle on sampled 128x128 tiles of x (tile-aligned blocks are local)."""
-    M, K = x.shape
     qr, sr, qc, sc = np_u8(q_row), s_row.cpu().numpy(), np_u8(q_col), s_col.cpu().numpy()
     for (m0, k0) in tiles:
         xt = bits(x[m0:m0 + 128, k0:k0 + 128])
@@ -55,20 +61,25 @@ def sample_tiles(rng, M, N, n, extra=()):
     return t
 
 
-def check_gemm_tiles(orc, kind, A, sA, B, sB, D, pts):
-    """pts: (m0, n0) corners of 32x32 output tiles."""
+def gemm_tiles(rng, M, N, rows=(), cols=()):
+    """128x128 output tiles: the four corners, N_RANDOM seeded random tiles,
+    a tile in the block row of every row in `rows` and in the block column
+    of every column in `cols` (random along the other axis)."""
+    t = [(0, 0), (M - T, N - T), (M - T, 0), (0, N - T)]
+    t += [(T * int(rng.integers(0, M // T)), T * int(rng.integers(0, N // T))) for _ in range(N_RANDOM)]
+    t += [((r // T) * T, T * int(rng.integers(0, N // T))) for r in rows]
+    t += [(T * int(rng.integers(0, M // T)), (c // T) * T) for c in cols]
+    return list(dict.fromkeys(t))
+
+
+def check_gemm_tiles(orc, kind, A, sA, B, sB, D, tiles):
+    """Every element of each 128x128 tile within the acceptance gate
+    |y - y_ref| <= 1e-2 sum|a b| + 1 bf16 ulp(y_ref)."""
     Ah, sAh, Bh, sBh, Dh = np_u8(A), sA.cpu().numpy(), np_u8(B), sB.cpu().numpy(), bits(D)
-    for (m0, n0) in pts:
-        y, ya = orc.gemm_ref_tile(kind, Ah, sAh, Bh, sBh, m0, m0 + 32, n0, n0 + 32)
-        bad, worst = orc.check_tol(np.ascontiguousarray(Dh[m0:m0 + 32, n0:n0 + 32]), y, ya)
+    for (m0, n0) in tiles:
+        y, ya = orc.gemm_ref_tile(kind, Ah, sAh, Bh, sBh, m0, m0 + T, n0, n0 + T)
+        bad, worst = orc.check_tol(np.ascontiguousarray(Dh[m0:m0 + T, n0:n0 + T]), y, ya)
         assert bad == 0, (kind, m0, n0, worst)
-
-
-def gemm_points(rng, M, N, n, extra_cols=()):
-    p = [(0, 0), (M - 32, N - 32), (M - 32, 0), (0, N - 32)]
-    p += [(32 * int(rng.integers(0, M // 32)), 32 * int(rng.integers(0, N // 32))) for _ in range(n)]
-    p += [(32 * int(rng.integers(0, M // 32)), (c // 32) * 32) for c in extra_cols]
-    return p
 
 
 def run_layer(fb, orc, X, W, dY, rng, mode=0, outlier_cols=(), pad_rows=()):
@@ -90,44 +101,49 @@ def run_layer(fb, orc, X, W, dY, rng, mode=0, outlier_cols=(), pad_rows=()):
     assert fb.fp8bw_last_device_error() == 0
     extra = [((r // 128) * 128, 128 * int(rng.integers(0, K // 128))) for r in pad_rows]
     extra += [(128 * int(rng.integers(0, M // 128)), (c // 128) * 128) for c in outlier_cols]
-    check_act_tiles(orc, X, qx, sx, qxc, sxc, sample_tiles(rng, M, K, 6, extra))
-    check_act_tiles(orc, dY, qd, sd, qdc, sdc, sample_tiles(rng, M, N, 4))
-    check_weight_blocks(orc, W, qw, sw, qwT, sample_tiles(rng, N, K, 6))
-    check_gemm_tiles(orc, 0, qx, sx, qw, sw, Y, gemm_points(rng, M, N, 5))
-    check_gemm_tiles(orc, 1, qd, sd, qwT, sw, dX, gemm_points(rng, M, K, 5, outlier_cols))
-    check_gemm_tiles(orc, 2, qdc, sdc, qxc, sxc, dW, gemm_points(rng, N, K, 5, outlier_cols))
+    check_act_tiles(orc, X, qx, sx, qxc, sxc, sample_tiles(rng, M, K, 6, extra), mode)
+    check_act_tiles(orc, dY, qd, sd, qdc, sdc, sample_tiles(rng, M, N, 4), mode)
+    check_weight_blocks(orc, W, qw, sw, qwT, sample_tiles(rng, N, K, 6), mode)
+    check_gemm_tiles(orc, 0, qx, sx, qw, sw, Y, gemm_tiles(rng, M, N, rows=pad_rows))
+    check_gemm_tiles(orc, 1, qd, sd, qwT, sw, dX, gemm_tiles(rng, M, K, rows=pad_rows, cols=outlier_cols))
+    check_gemm_tiles(orc, 2, qdc, sdc, qxc, sxc, dW, gemm_tiles(rng, N, K, cols=outlier_cols))
     return Y, dX
 
 
+@pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("name", [n for n, _, _ in workloads.LLAMA8B_LAYERS])
-def test_llama8b_layer(fb, orc, name):
+def test_llama8b_layer(fb, orc, name, mode):
     X, W, dY = workloads.llama_layer(name, seed=0, device=DEV)
     idx = [n for n, _, _ in workloads.LLAMA8B_LAYERS].index(name)
     K = workloads.LLAMA8B_LAYERS[idx][1]
     outl = workloads.outlier_channels(K, 0 * 1000 + idx * 10 + 1)
-    rng = np.random.default_rng(idx)
-    run_layer(fb, orc, X, W, dY, rng, outlier_cols=outl[:2])
+    rng = np.random.default_rng(idx + 10 * mode)
+    run_layer(fb, orc, X, W, dY, rng, mode, outlier_cols=outl)
 
 
-def test_packed_long_sequence(fb, orc):
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("name", [n for n, _, _ in workloads.LLAMA8B_LAYERS])
+def test_packed_long_sequence(fb, orc, name, mode):
     """4 packed sequences, 32768 tokens, heavy-tailed activations and zero
-    padding rows: padding rows give all-zero blocks (scale 1, zero codes) and
-    exact zeros in the forward output."""
-    name, K, N = workloads.LLAMA8B_LAYERS[0]
-    M = workloads.PACKED_TOKENS
+    padding rows on every Llama-like layer shape: padding rows give all-zero
+    blocks (scale 1, zero codes) and exact zeros in fprop and dgrad."""
+    idx = [n for n, _, _ in workloads.LLAMA8B_LAYERS].index(name)
+    _, K, N = workloads.LLAMA8B_LAYERS[idx]
     mask = workloads.packed_rows_mask(0)
     X = workloads.packed_activations(K, 0, DEV)
     dY = workloads.packed_activations(N, 1, DEV, scale=1e-3)
     W = workloads.llama_weight(name, 0, device=DEV)
     pad = np.nonzero(~mask.numpy())[0]
-    rng = np.random.default_rng(5)
-    pad_rows = [int(pad[0]), int(pad[-1])] if pad.size else []
-    Y, _ = run_layer(fb, orc, X, W, dY, rng, pad_rows=pad_rows)
+    rng = np.random.default_rng(5 + idx + 10 * mode)
+    pad_rows = sorted({int(pad[0]), int(pad[len(pad) // 2]), int(pad[-1])}) if pad.size else []
+    Y, dX = run_layer(fb, orc, X, W, dY, rng, mode, pad_rows=pad_rows)
     if pad.size:
-        assert torch.all(Y[torch.from_numpy(pad).to(DEV)] == 0)
+        rows = torch.from_numpy(pad).to(DEV)
+        assert torch.all(Y[rows] == 0) and torch.all(dX[rows] == 0)
 
 
-def test_requant_sweep(fb, orc):
+@pytest.mark.parametrize("mode", [0, 1])
+def test_requant_sweep(fb, orc, mode):
     """32 layers x 4 weights (about 7B bf16 parameters), Adam-like update
     N(0, 1e-4^2) and one batched requant per step for 10 steps; step 0 and
     step 9 are checked on sampled blocks, and the batched call must equal the
@@ -140,22 +156,26 @@ def test_requant_sweep(fb, orc):
             Ws.append(workloads.llama_weight(n, l, device=DEV))
             outs.append(weight_buffers(N, K, DEV))
     items = [(w, q, s, qT) for w, (q, s, qT) in zip(Ws, outs)]
-    rng = np.random.default_rng(9)
+    rng = np.random.default_rng(9 + mode)
     for step in range(10):
         if step > 0:
             for i, w in enumerate(Ws):
                 workloads.requant_update_(w, step, i // 4, i % 4)
-        fb.fp8bw_requant_weights(items, 0)
+        fb.fp8bw_requant_weights(items, mode)
         torch.cuda.synchronize()
         assert fb.fp8bw_last_device_error() == 0
         if step in (0, 9):
             for i in rng.choice(len(Ws), 6, replace=False):
                 w, (q, s, qT) = Ws[i], outs[i]
-                check_weight_blocks(orc, w, q, s, qT, sample_tiles(rng, *w.shape, 3))
+                check_weight_blocks(orc, w, q, s, qT, sample_tiles(rng, *w.shape, 3), mode)
+        else:
+            i = int(rng.integers(0, len(Ws)))
+            w, (q, s, qT) = Ws[i], outs[i]
+            check_weight_blocks(orc, w, q, s, qT, sample_tiles(rng, *w.shape, 1), mode)
     # batched == single call, on two of the largest weights
     for i in (2, 6):
         q, s, qT = weight_buffers(*Ws[i].shape, DEV)
-        fb.fp8bw_quant_weight_128x128(Ws[i], 0, q, s, qT)
+        fb.fp8bw_quant_weight_128x128(Ws[i], mode, q, s, qT)
         torch.cuda.synchronize()
         assert torch.equal(q, outs[i][0]) and torch.equal(qT, outs[i][2])
         assert torch.equal(s.view(torch.int32), outs[i][1].view(torch.int32))
@@ -164,8 +184,8 @@ def test_requant_sweep(fb, orc):
 def test_wgrad_accumulates_into_fp32_main_grad(fb, orc):
     """Gradient accumulation over two micro-batches of the down layer
     (8192 tokens each, 14336 -> 4096): dW of each is added to an fp32 main
-    gradient by fp8bw_gemm_f32(accumulate); sampled 32x32 tiles are checked
-    against main_grad0 + the fp64 references of both micro-batches."""
+    gradient by fp8bw_gemm_f32(accumulate); sampled 128x128 tiles are
+    checked against main_grad0 + the fp64 references of both micro-batches."""
     name, K, N = workloads.LLAMA8B_LAYERS[3]
     M = workloads.LLAMA8B_TOKENS
     rng = np.random.default_rng(77)
@@ -184,12 +204,12 @@ def test_wgrad_accumulates_into_fp32_main_grad(fb, orc):
     assert fb.fp8bw_last_device_error() == 0
     got = main.cpu().numpy()
     host = [tuple(np_u8(t) if t.dtype == torch.uint8 else t.cpu().numpy() for t in o) for o in ops]
-    for (m0, n0) in gemm_points(rng, N, K, 8):
-        ref = main0[m0:m0 + 32, n0:n0 + 32].copy()
-        yabs = np.zeros((32, 32))
+    for (m0, n0) in gemm_tiles(rng, N, K):
+        ref = main0[m0:m0 + T, n0:n0 + T].copy()
+        yabs = np.zeros((T, T))
         for A, sA, B, sB in host:
-            y, ya = orc.gemm_ref_tile(2, A, sA, B, sB, m0, m0 + 32, n0, n0 + 32)
+            y, ya = orc.gemm_ref_tile(2, A, sA, B, sB, m0, m0 + T, n0, n0 + T)
             ref += y
             yabs += ya
-        bad, worst = orc.check_tol_f32(got[m0:m0 + 32, n0:n0 + 32], ref, yabs)
+        bad, worst = orc.check_tol_f32(got[m0:m0 + T, n0:n0 + T], ref, yabs)
         assert bad == 0, (m0, n0, worst)

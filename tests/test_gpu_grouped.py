@@ -96,61 +96,100 @@ def test_grouped_bad_offsets(fb, orc):
     assert fb.fp8bw_last_device_error() == 0   # the error word was cleared
 
 
-def test_grouped_moe_full_size_sampled(fb, orc):
-    """Qwen3-30B-A3B-like expert layer (hidden 2048 -> 1536, 128 experts,
-    top-8 of 16384 tokens, Zipf(1.1) popularity) at full size, in the launch
-    configuration the benchmark uses; one 128x128 output tile per expert is
-    checked against the oracle (smallest and largest experts included)."""
+MOE_SHAPES = {"gate_up": (workloads.MOE_HIDDEN, 2 * workloads.MOE_INTER),
+              "down": (workloads.MOE_INTER, workloads.MOE_HIDDEN)}
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("layer", ["gate_up", "down"])
+def test_grouped_moe_full_size_sampled(fb, orc, layer, mode):
+    """Qwen3-30B-A3B-like expert layers (gate_up 2048 -> 1536 and down
+    768 -> 2048, 128 experts, top-8 of 16384 tokens, Zipf(1.1) popularity)
+    at full size, in the launch configuration the benchmark uses, in both
+    scale modes: fprop, dgrad and wgrad.  Checked against the oracle: one
+    128x128 output tile per expert for each GEMM (smallest and largest
+    experts included), a tile over each expert's zero padding rows (exact
+    zeros in fprop and dgrad), 16 seeded random tiles, and sampled
+    quantizer tiles (bit-exact)."""
     r = workloads.moe_routing(0)
-    G, K, N = workloads.MOE_EXPERTS, workloads.MOE_HIDDEN, 2 * workloads.MOE_INTER
-    X = workloads.moe_permuted(r, K, 1.0, seed=5, device=DEV)
-    W = workloads.moe_experts(G, N, K, seed=6, device=DEV)
+    G = workloads.MOE_EXPERTS
+    K, N = MOE_SHAPES[layer]
+    seeds = {"gate_up": (5, 6, 7), "down": (15, 16, 17)}[layer]
+    X = workloads.moe_permuted(r, K, 1.0, seed=seeds[0], device=DEV)
+    W = workloads.moe_experts(G, N, K, seed=seeds[1], device=DEV)
+    dY = workloads.moe_permuted(r, N, 1e-3, seed=seeds[2], device=DEV)
     Mtot = r.m_total_pad
-    qx = torch.empty((Mtot, K), dtype=torch.uint8, device=DEV)
-    sx = torch.empty((K // 128, Mtot), dtype=torch.float32, device=DEV)
-    fb.fp8bw_quant_act_1x128(X, 0, qx, sx)
-    qw = torch.empty((G, N, K), dtype=torch.uint8, device=DEV)
-    sw = torch.empty((G, N // 128, K // 128), dtype=torch.float32, device=DEV)
-    fb.fp8bw_requant_weights([(W[e], qw[e], sw[e], None) for e in range(G)], 0)
+    u8, f32 = torch.uint8, torch.float32
+    e = lambda *sh, dt=u8: torch.empty(sh, dtype=dt, device=DEV)  # noqa: E731
+    qx, sx, qxc, sxc = e(Mtot, K), e(K // 128, Mtot, dt=f32), e(K, Mtot), e(Mtot // 128, K, dt=f32)
+    qd, sd, qdc, sdc = e(Mtot, N), e(N // 128, Mtot, dt=f32), e(N, Mtot), e(Mtot // 128, N, dt=f32)
+    qw, sw, qwT = e(G, N, K), e(G, N // 128, K // 128, dt=f32), e(G, K, N)
+    fb.fp8bw_quant_act_1x128(X, mode, qx, sx, qxc, sxc)
+    fb.fp8bw_quant_act_1x128(dY, mode, qd, sd, qdc, sdc)
+    fb.fp8bw_requant_weights([(W[g], qw[g], sw[g], qwT[g]) for g in range(G)], mode)
     off = torch.tensor(r.offsets, dtype=torch.int32, device=DEV)
-    D = torch.empty((Mtot, N), dtype=torch.bfloat16, device=DEV)
-    fb.fp8bw_grouped_gemm(0, off, qx, sx, qw, sw, D, 0)
+    bf = torch.bfloat16
+    Y, dX, dW = e(Mtot, N, dt=bf), e(Mtot, K, dt=bf), e(G, N, K, dt=bf)
+    fb.fp8bw_grouped_gemm(0, off, qx, sx, qw, sw, Y, mode)
+    fb.fp8bw_grouped_gemm(1, off, qd, sd, qwT, sw, dX, mode)
+    fb.fp8bw_grouped_gemm(2, off, qdc, sdc, qxc, sxc, dW, mode)
     torch.cuda.synchronize()
     assert fb.fp8bw_last_device_error() == 0
-    qx_h, sx_h, qw_h, sw_h = qx.cpu().numpy(), sx.cpu().numpy(), qw.cpu().numpy(), sw.cpu().numpy()
-    Dh = bits(D)
-    rng = np.random.default_rng(0)
+
+    rng = np.random.default_rng(100 + 10 * mode + (layer == "down"))
     counts = np.array(r.counts)
     offs = np.array(r.offsets, np.int32)
-    for e in range(G):
-        if counts[e] == 0:
-            continue
-        nblk = (offs[e + 1] - offs[e]) // 128
-        rb = int(offs[e]) + 128 * int(rng.integers(0, nblk)) + 32 * int(rng.integers(0, 4))
-        cb = 32 * int(rng.integers(0, N // 32))
-        y, ya = orc.grouped_gemm_ref_tile(0, offs, qx_h, sx_h, qw_h, sw_h, 0, rb, rb + 32, cb, cb + 32)
-        bad, worst = orc.check_tol(np.ascontiguousarray(Dh[rb:rb + 32, cb:cb + 32]), y, ya)
-        assert bad == 0, (e, worst)
-    # wgrad for the largest and smallest experts: dW_g = dY_g^T X_g
-    dY = workloads.moe_permuted(r, N, 1e-3, seed=7, device=DEV)
-    qxc = torch.empty((K, Mtot), dtype=torch.uint8, device=DEV)
-    sxc = torch.empty((Mtot // 128, K), dtype=torch.float32, device=DEV)
-    qd = torch.empty((Mtot, N), dtype=torch.uint8, device=DEV)
-    sd = torch.empty((N // 128, Mtot), dtype=torch.float32, device=DEV)
-    qdc = torch.empty((N, Mtot), dtype=torch.uint8, device=DEV)
-    sdc = torch.empty((Mtot // 128, N), dtype=torch.float32, device=DEV)
-    fb.fp8bw_quant_act_1x128(X, 0, qx, sx, qxc, sxc)
-    fb.fp8bw_quant_act_1x128(dY, 0, qd, sd, qdc, sdc)
-    dW = torch.empty((G, N, K), dtype=torch.bfloat16, device=DEV)
-    fb.fp8bw_grouped_gemm(2, off, qdc, sdc, qxc, sxc, dW, 0)
-    torch.cuda.synchronize()
-    assert fb.fp8bw_last_device_error() == 0
-    A, sA, B, sB = qdc.cpu().numpy(), sdc.cpu().numpy(), qxc.cpu().numpy(), sxc.cpu().numpy()
-    for e in [int(np.argmax(counts)), int(np.argmin(counts))]:
-        nb, kb = 32 * int(rng.integers(0, N // 32)), 32 * int(rng.integers(0, K // 32))
-        y, ya = orc.grouped_gemm_ref_tile(2, offs, A, sA, B, sB, e, nb, nb + 32, kb, kb + 32)
-        bad, worst = orc.check_tol(np.ascontiguousarray(bits(dW[e])[nb:nb + 32, kb:kb + 32]), y, ya)
-        assert bad == 0, (e, worst)
+    h = lambda t: t.cpu().numpy()  # noqa: E731
+    qx_h, sx_h, qxc_h, sxc_h = h(qx), h(sx), h(qxc), h(sxc)
+    qd_h, sd_h, qdc_h, sdc_h = h(qd), h(sd), h(qdc), h(sdc)
+    qw_h, sw_h, qwT_h = h(qw), h(sw), h(qwT)
+
+    # quantizers: tiles at expert boundaries and random tiles, bit-exact
+    for (m0, k0) in [(int(offs[g]), 0) for g in rng.choice(G, 4, replace=False) if counts[g]] + \
+            [(128 * int(rng.integers(0, Mtot // 128)), 128 * int(rng.integers(0, K // 128)))]:
+        oq, os_, oqc, osc = orc.quant_act_1x128(bits(X[m0:m0 + 128, k0:k0 + 128]), mode)
+        assert np.array_equal(qx_h[m0:m0 + 128, k0:k0 + 128], oq)
+        assert np.array_equal(qxc_h[k0:k0 + 128, m0:m0 + 128], oqc)
+        assert np.array_equal(sx_h[k0 // 128, m0:m0 + 128].view(np.uint32), os_.view(np.uint32)[0])
+        assert np.array_equal(sxc_h[m0 // 128, k0:k0 + 128].view(np.uint32), osc.view(np.uint32)[0])
+    g = int(rng.integers(0, G))
+    oq, os_, oqT = orc.quant_weight_128x128(bits(W[g]), mode)
+    assert np.array_equal(qw_h[g], oq) and np.array_equal(qwT_h[g], oqT)
+    assert np.array_equal(sw_h[g].view(np.uint32), os_.view(np.uint32))
+
+    # fprop / dgrad: a tile per expert, a padding tile per padded expert,
+    # random tiles over the routed rows
+    for kind, D, (A, sA, B, sB), width in [(0, Y, (qx_h, sx_h, qw_h, sw_h), N),
+                                           (1, dX, (qd_h, sd_h, qwT_h, sw_h), K)]:
+        Dh = bits(D)
+        rows = []
+        for g in range(G):
+            nblk = (offs[g + 1] - offs[g]) // 128
+            if nblk == 0:
+                continue
+            rows.append(int(offs[g]) + 128 * int(rng.integers(0, nblk)))
+            if counts[g] % 128:
+                rows.append(int(offs[g + 1]) - 128)      # the block holding the padding rows
+        rows += [128 * int(rng.integers(0, int(offs[-1]) // 128)) for _ in range(16)]
+        for rb in dict.fromkeys(rows):
+            cb = 128 * int(rng.integers(0, width // 128))
+            y, ya = orc.grouped_gemm_ref_tile(kind, offs, A, sA, B, sB, 0, rb, rb + 128, cb, cb + 128)
+            bad, worst = orc.check_tol(np.ascontiguousarray(Dh[rb:rb + 128, cb:cb + 128]), y, ya)
+            assert bad == 0, (kind, rb, cb, worst)
+        pad_rows = np.nonzero((r.row_token < 0).numpy())[0]
+        if pad_rows.size:
+            assert torch.all(D[torch.from_numpy(pad_rows).to(DEV)] == 0)
+
+    # wgrad: one 128x128 tile of every expert's dW_g (contraction over the
+    # expert's own tokens only), empty experts exact zeros
+    dWh = bits(dW)
+    for g in range(G):
+        nb, kb = 128 * int(rng.integers(0, N // 128)), 128 * int(rng.integers(0, K // 128))
+        y, ya = orc.grouped_gemm_ref_tile(2, offs, qdc_h, sdc_h, qxc_h, sxc_h, g, nb, nb + 128, kb, kb + 128)
+        bad, worst = orc.check_tol(np.ascontiguousarray(dWh[g, nb:nb + 128, kb:kb + 128]), y, ya)
+        assert bad == 0, (g, nb, kb, worst)
+        if counts[g] == 0:
+            assert torch.all(dW[g] == 0)
 
 
 @pytest.mark.parametrize("mode", [0, 1])
