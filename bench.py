@@ -54,6 +54,8 @@ def parse():
                         "--tokens, requant_sweep (32 layers), or "
                         "moe_fprop|moe_dgrad|moe_wgrad "
                         "on the MoE expert layer --layer gate_up|down")
+    p.add_argument("--sweep", action="store_true",
+                   help="time every call of the Llama-like and MoE layers, both scale modes (one JSON line each)")
     p.add_argument("--layer", default="gate_up", choices=[n for n, _, _ in workloads.LLAMA8B_LAYERS])
     p.add_argument("--tokens", type=int, default=workloads.LLAMA8B_TOKENS,
                    help="tokens of the --case layer (32768 = the packed long-sequence batch)")
@@ -405,8 +407,16 @@ def run_case(args):
                 nbytes += N * K * 4 + 4 * (N // 128) * (K // 128)
         time_call(fb, args, "all", mode, lambda: fb.fp8bw_requant_weights(items, mode), nbytes, "GB/s")
         return
+    calls = layer_calls(fb, mode, name, args.tokens, wgrad_acc=args.case == "wgrad_acc")
+    fn, work, unit = calls[args.case]
+    time_call(fb, args, name, mode, fn, work, unit)
+
+
+def layer_calls(fb, mode, name, tokens, wgrad_acc=False):
+    """Every timed call of one Llama-like layer at `tokens` tokens, with its
+    algorithmic work (FLOP or bytes) and unit."""
     K, N = [(k, n) for nm, k, n in workloads.LLAMA8B_LAYERS if nm == name][0]
-    l = Layer(name, K, N, args.tokens, torch.device("cuda", 0))
+    l = Layer(name, K, N, tokens, torch.device("cuda", 0))
     fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT)], mode)
     fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)
     fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)
@@ -429,12 +439,41 @@ def run_case(args):
         l.dY, fb.FP8BW_FMT_E5M2, mode, hist, l.qd, l.qdc, sc, am), 4 * l.M * l.N, "GB/s")
     calls["quant_delayed_x"] = (lambda: fb.fp8bw_quant_tensor_delayed(
         l.X, fb.FP8BW_FMT_E4M3, mode, hist, l.qx, l.qxc, sc, am), 4 * l.M * l.K, "GB/s")
-    if args.case == "wgrad_acc":   # wgrad added into an fp32 main gradient
+    if wgrad_acc:   # wgrad added into an fp32 main gradient
         main_grad = torch.zeros((N, K), dtype=torch.float32, device=l.X.device)
         calls["wgrad_acc"] = (lambda: fb.fp8bw_gemm_f32(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, main_grad,
                                                         accumulate=True, mode=mode), l.flops / 3, "TFLOP/s")
-    fn, work, unit = calls[args.case]
-    time_call(fb, args, name, mode, fn, work, unit)
+    return calls
+
+
+SWEEP_CASES = ("fprop", "dgrad", "wgrad", "quant_x", "quant_dy", "requant")
+
+
+def run_sweep(args):
+    """Per-call table: every GEMM and quantizer call of the four Llama-like
+    layers (at --tokens) and the two MoE expert layers, both scale modes, and
+    the BF16 comparison GEMM, in one process; one JSON line per call."""
+    import blockwise_scaled_fp8_fp8bw_b200 as fb
+    torch.cuda.set_device(0)
+    fb.fp8bw_init(0)
+    for mname, mode in (("fp32", fb.FP8BW_SCALE_FP32), ("pow2", fb.FP8BW_SCALE_POW2)):
+        args.mode = mname
+        for name, _, _ in workloads.LLAMA8B_LAYERS:
+            calls = layer_calls(fb, mode, name, args.tokens)
+            for c in SWEEP_CASES + (("bf16_fprop",) if mname == "fp32" else ()):
+                args.case = c
+                fn, work, unit = calls[c]
+                time_call(fb, args, name, mode, fn, work, unit)
+            del calls
+            torch.cuda.empty_cache()
+        for name in ("gate_up", "down"):
+            mc = moe_calls(fb, mode, name)
+            for c in ("moe_fprop", "moe_dgrad", "moe_wgrad"):
+                args.case = c
+                fn, work, unit = mc[c]
+                time_call(fb, args, name, mode, fn, work, unit)
+            del mc
+            torch.cuda.empty_cache()
 
 
 def time_call(fb, args, name, mode, fn, work, unit):
@@ -476,6 +515,9 @@ def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     if args.case:
         run_case(args)

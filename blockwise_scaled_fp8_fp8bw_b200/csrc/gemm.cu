@@ -24,10 +24,11 @@
 //               (2 block scales, or 256 column scales for wgrad) into an
 //               8-slot shared ring with cp.async.
 //   warps 4-11  promotion: each warp owns a 32-row quarter of TMEM lanes and
-//               128 columns (fprop/dgrad: a thread per row, 32x32b loads;
-//               wgrad: 4 rows x 32 columns per thread, 16x256b loads, so the
-//               per-column scales need few shared loads); per chunk it reads
-//               the chunk product from TMEM, multiplies by sA*sB in fp32 and
+//               128 columns, a thread per row (32x32b loads in four groups of
+//               32 columns, the next group's load in flight while the current
+//               one is scaled; wgrad's per-column scales arrive as warp-wide
+//               16-byte shared-memory broadcasts); per chunk it reads the
+//               chunk product from TMEM, multiplies by sA*sB in fp32 and
 //               adds it to its registers (packed f32x2 FMAs), releasing the
 //               TMEM buffer as soon as it is read so the MMA of the next
 //               chunk overlaps.  At the end of a tile the results are
@@ -223,22 +224,6 @@ __device__ __forceinline__ void stage_rows_f32(uint8_t* epi, int lane, const flo
   for (int c = 0; c < 4; ++c)
     *reinterpret_cast<float4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) =
         make_float4(a[2 * c].x, a[2 * c].y, a[2 * c + 1].x, a[2 * c + 1].y);
-}
-
-// Accumulators of the 16x256b shape (wgrad promotion): acc[16 i + g] holds
-// row 8i + lane/4 and columns 8g + 2(lane%4) + {0, 1}; piece pp covers the
-// column groups g = 2pp, 2pp + 1.
-__device__ __forceinline__ void stage_quad_f32(uint8_t* epi, int lane, const float2* acc, int pp) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = 8 * i + (lane >> 2);
-#pragma unroll
-    for (int gg = 0; gg < 2; ++gg) {
-      const int chunk = 2 * gg + ((lane & 3) >> 1);
-      *reinterpret_cast<float2*>(epi + row * 64 + 16 * (chunk ^ ((row >> 1) & 3)) + 8 * (lane & 1)) =
-          acc[16 * i + 2 * pp + gg];
-    }
-  }
 }
 
 // Writes (or adds) one staged fp32 piece.
@@ -489,78 +474,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const ScaleSlot* sl = &slots[ss];
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
-        if (KIND == FP8BW_WGRAD) {
-          // Column scales change with every column, so each thread needs the
-          // scale of every column it holds.  The 16x256b TMEM shape gives a
-          // thread 4 rows x 32 columns (instead of 1 row x 128 columns), so
-          // a chunk costs 4 row-scale and 16 column-pair loads from shared
-          // memory instead of 128 column-scale loads.
-          // acc[16 * i + g] holds row 8i + lane/4 of the quarter and columns
-          // 8g + 2(lane%4) + {0, 1} of the warp's 128.
-          float sa[4];
+        // The thread owns row q*32 + lane of the CTA's 128 and the 128
+        // columns of its half: four groups of 32 columns (32x32b TMEM
+        // loads).  The next group's load is issued before the current
+        // group's arithmetic, so the TMEM read latency hides behind it, and
+        // the buffer goes back to the MMA warp as soon as its last group has
+        // landed in registers.
+        const float sa = sl->sa[q * 32 + lane];
+        float2 s2 = make_float2(sa, sa);
+        if (KIND != FP8BW_WGRAD) {
+          const float sc = sa * sl->sb[half];   // one scale for the row's 128 columns
+          s2 = make_float2(sc, sc);
+        }
+        // wgrad: a scale per column; all lanes read the same 16 bytes
+        // (a shared-memory broadcast), four column scales per load
+        const float4* sb4 = reinterpret_cast<const float4*>(&sl->sb[half * 128]);
+        uint32_t r[2][32];
+        tmem_ld32(taddr, r[0]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sa[i] = sl->sa[q * 32 + 8 * i + (lane >> 2)];
-          const float* sbw = &sl->sb[half * 128 + 2 * (lane & 3)];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {  // 64-column halves of the warp's 128 columns
-            uint32_t r[2][32];
-            tmem_ld16x64(taddr + h2 * 64, r[0]);                      // quarter lanes 0-15
-            tmem_ld16x64(taddr + (16u << 16) + h2 * 64, r[1]);        // quarter lanes 16-31
-            tmem_wait_ld();
-            if (h2 == 1) {
-              // chunk fully read: hand the TMEM buffer back to the MMA warp
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) {
-                if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
-                else mbar_arrive(smem_u32(&bars->tempty[buf]));
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int g = h2 * 8 + j;
-              const float2 b2 = *reinterpret_cast<const float2*>(sbw + 8 * g);
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                  const int i = 2 * u + v;
-                  const float2 sc = fmul2(make_float2(sa[i], sa[i]), b2);
-                  acc[16 * i + g] = ffma2(make_float2(__uint_as_float(r[u][4 * j + 2 * v]),
-                                                      __uint_as_float(r[u][4 * j + 2 * v + 1])),
-                                          sc, acc[16 * i + g]);
-                }
-              }
+        for (int g = 0; g < 4; ++g) {
+          tmem_wait_ld();
+          tmem_fence_regs(r[g & 1]);
+          if (g < 3) {
+            tmem_ld32(taddr + (g + 1) * 32, r[(g + 1) & 1]);
+          } else {
+            // chunk fully read: hand the TMEM buffer back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
+              else mbar_arrive(smem_u32(&bars->tempty[buf]));
             }
           }
-        } else {
-          const float sa = sl->sa[q * 32 + lane];
-          // Two rounds of two 32-column loads: one wait per 64 columns keeps
-          // the staging at 64 registers next to the 128 accumulators.
+          const uint32_t* rg = r[g & 1];
+          if (KIND == FP8BW_WGRAD) {
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t r[2][32];
-            tmem_ld64(taddr + h2 * 64, r[0], r[1]);
-            tmem_wait_ld();
-            if (h2 == 1) {
-              // chunk fully read: hand the TMEM buffer back to the MMA warp
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) {
-                if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
-                else mbar_arrive(smem_u32(&bars->tempty[buf]));
-              }
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 b = sb4[8 * g + j4];
+              const float2 c0 = fmul2(s2, make_float2(b.x, b.y));
+              const float2 c1 = fmul2(s2, make_float2(b.z, b.w));
+              acc[16 * g + 2 * j4] = ffma2(make_float2(__uint_as_float(rg[4 * j4]), __uint_as_float(rg[4 * j4 + 1])),
+                                           c0, acc[16 * g + 2 * j4]);
+              acc[16 * g + 2 * j4 + 1] = ffma2(make_float2(__uint_as_float(rg[4 * j4 + 2]), __uint_as_float(rg[4 * j4 + 3])),
+                                               c1, acc[16 * g + 2 * j4 + 1]);
             }
-            const float s = sa * sl->sb[half];
-            const float2 s2 = make_float2(s, s);
+          } else {
 #pragma unroll
-            for (int p2 = 0; p2 < 2; ++p2) {
-              const int p = h2 * 2 + p2;
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                acc[p * 16 + j] = ffma2(make_float2(__uint_as_float(r[p2][2 * j]), __uint_as_float(r[p2][2 * j + 1])),
-                                        s2, acc[p * 16 + j]);
-            }
+            for (int j = 0; j < 16; ++j)
+              acc[16 * g + j] = ffma2(make_float2(__uint_as_float(rg[2 * j]), __uint_as_float(rg[2 * j + 1])),
+                                      s2, acc[16 * g + j]);
           }
         }
         __syncwarp();
@@ -584,8 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_wait_read<C::kEpiBufs - 1>();
           }
           __syncwarp();
-          if (KIND == FP8BW_WGRAD) stage_quad_f32(epi, lane, acc, pp);
-          else stage_rows_f32(epi, lane, &acc[8 * pp]);
+          stage_rows_f32(epi, lane, &acc[8 * pp]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -602,21 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_wait_read<C::kEpiBufs - 1>();
         }
         __syncwarp();
-        if (KIND == FP8BW_WGRAD) {
-          // rows 8i + lane/4, columns 8c + 2(lane%4) + {0, 1} of the piece:
-          // one bf16 pair per store; the 64-byte swizzle keeps the 32 lanes
-          // of each store on 32 distinct banks
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = 8 * i + (lane >> 2);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float2 v2 = acc[16 * i + 4 * p + c];
-              *reinterpret_cast<uint32_t*>(epi + row * 64 + 16 * (c ^ ((row >> 1) & 3)) + 4 * (lane & 3)) =
-                  pack_bf16x2(v2.x, v2.y);
-            }
-          }
-        } else {
+        {
           // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
 #pragma unroll
           for (int c = 0; c < 4; ++c) {

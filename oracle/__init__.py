@@ -87,6 +87,8 @@ def lib():
         L.orc_bf16_ulp.restype = dbl
         L.orc_check_tol.argtypes = [vp, vp, vp, i64, dbl, vp]
         L.orc_check_tol.restype = i64
+        L.orc_attention_fwd_rows.argtypes = [i64, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp,
+                                             vp, vp, i64, vp, vp, vp, vp, vp]
         L.orc_set_threads.argtypes = [i32]
         L.orc_max_threads.restype = i32
         _lib = L
@@ -312,3 +314,43 @@ def check_tol_f32(y, yref, yabs, rel=REL_TOL):
     ratio = np.where(lim > 0, err / np.where(lim > 0, lim, 1.0), np.where(err > 0, np.inf, 0.0))
     worst = float(np.max(np.where(np.isnan(ratio), np.inf, ratio))) if ratio.size else 0.0
     return int(np.count_nonzero(~ok)), worst
+
+
+# ------------------------------------------------------------- attention --
+HEAD_DIM = 128
+
+
+def attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, seg_off, seg_len, causal, rows_t, rows_h):
+    """FP8 attention forward reference ("NVIDIA NeMo RL erreicht 48% ...",
+    "Leistungsgewinne in der Praxis": FP8 KV cache and attention) for the
+    (token, head) rows given.  q [T, Hq*128] codes, sq [Hq, T]; k [T, Hkv*128],
+    sk [Hkv, T]; vT [Hkv*128, T] codes of V's column-wise copy, sv
+    [T/128, Hkv*128]; seg_off [nseg+1] (multiples of 128), seg_len [nseg].
+    Returns (O [n,128], oabs [n,128], oflip [n,128]) in fp64."""
+    q, k, vT = _u8(q), _u8(k), _u8(vT)
+    sq, sk, sv = _f32(sq), _f32(sk), _f32(sv)
+    T = q.shape[0]
+    off = np.ascontiguousarray(seg_off, np.int32)
+    ln = np.ascontiguousarray(seg_len, np.int32)
+    rt = np.ascontiguousarray(rows_t, np.int64)
+    rh = np.ascontiguousarray(rows_h, np.int32)
+    n = rt.size
+    out = np.empty((n, HEAD_DIM), np.float64)
+    oa = np.empty_like(out)
+    of = np.empty_like(out)
+    lib().orc_attention_fwd_rows(T, int(Hq), int(Hkv), ln.size, _p(off), _p(ln), int(bool(causal)),
+                                 _p(q), _p(sq), _p(k), _p(sk), _p(vT), _p(sv), n, _p(rt), _p(rh),
+                                 _p(out), _p(oa), _p(of))
+    return out, oa, of
+
+
+def check_tol_attn(y_bits, oref, oabs, oflip, rel=REL_TOL):
+    """Attention gate: |y - O| <= rel * oabs + oflip + 1 bf16 ulp(O), with y
+    bf16 bits.  Returns (violations, worst error/allowance ratio)."""
+    y = _u16(y_bits).ravel()
+    oref = np.ascontiguousarray(oref, np.float64).ravel()
+    yabs = (np.ascontiguousarray(oabs, np.float64).ravel() +
+            np.ascontiguousarray(oflip, np.float64).ravel() / rel)
+    worst = np.zeros(1, np.float64)
+    bad = lib().orc_check_tol(_p(y), _p(oref), _p(yabs), y.size, rel, _p(worst))
+    return int(bad), float(worst[0])

@@ -548,4 +548,125 @@ int64_t orc_check_tol(const uint16_t* y, const double* yref,
   return bad;
 }
 
+// -------------------------------------------------------------- attention --
+// FP8 attention forward [P1 "Leistungsgewinne in der Praxis": the recipe
+// extends FP8 to the KV cache and the attention operations; no granularity
+// or numerics are given].  Readings taken, each the recipe's own rule carried
+// over:
+//  * every FP8 operand is E4M3 with 1x128 blocks along its contraction
+//    ("Der technische Durchbruch": 1x128 for activations): Q and K carry one
+//    scale per token and head (head dimension 128 = one block), V is the
+//    column-wise copy of the activation quantizer (one scale per 128 tokens
+//    of one channel, codes stored channel-major [H*128][T]), and the softmax
+//    numerator P carries one scale per query row and 128-key block;
+//  * logits z_j = (q^ . k^_j) / sqrt(128) from the dequantized operands,
+//    p_j = exp(z_j - max_j z_j) over the query's keys, l = sum_j p_j taken
+//    from the unquantized p;
+//  * P's block scale follows the FP32 rule s_b = amax_b / 448 and its codes
+//    are E4M3(fp32(p_j / s_b)); the power-of-two rule is not used for P,
+//    because p / amax is what a streaming kernel can reproduce (it meets the
+//    keys relative to a running maximum, which scales a block by a constant);
+//  * O_d = sum_j p^_j v^_{j,d} / l, p^_j = decode(code_j) * s_b.
+// Sequences: segment g covers tokens [off[g], off[g+1]) (multiples of 128),
+// of which the first len[g] are real tokens; a query token's keys are the
+// real tokens of its segment, and with `causal` only those j <= t.  Query
+// head h reads key/value head h / (Hq / Hkv).
+//
+// For each requested (token, head) row: out[d] = O_d in fp64; oabs[d] =
+// sum_j |p^_j v^_{j,d}| / l (the GEMM gate's magnitude term for P.V); and
+// oflip[d] = sum over ambiguous codes of (one E4M3 step of p_j/s_b) * s_b *
+// |v^_{j,d}| / l.  A code is ambiguous when p_j / s_b lies within eta of an
+// E4M3 rounding midpoint, eta bounding the relative error with which an fp32
+// kernel forms p_j / s_b: the tensor core's fp32 sum of the 128 code
+// products (at most 2^-16 of their absolute sum), the fp32 scaling of the
+// logits (2^-21 relative), the exponential (2^-21) and the running maximum
+// (the largest logit error of the row).  Either rounding is then correct.
+// Padding query rows (t beyond its segment's real tokens) give O = 0.
+void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
+                            const int32_t* off, const int32_t* len, int32_t causal,
+                            const uint8_t* q, const float* sq, const uint8_t* k,
+                            const float* sk, const uint8_t* vT, const float* sv,
+                            int64_t nrows, const int64_t* row_t, const int32_t* row_h,
+                            double* out, double* oabs, double* oflip) {
+  const int64_t D = 128;
+  const double* dec = decode_table(FMT_E4M3);
+  const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(D));
+  const int32_t group = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t t = row_t[r];
+    const int32_t h = row_h[r], g = h / group;
+    double* o = out + r * D;
+    double* oa = oabs + r * D;
+    double* of = oflip + r * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = oa[d] = of[d] = 0.0;
+    int32_t seg = 0;
+    while (seg + 1 < nseg && off[seg + 1] <= t) ++seg;
+    const int64_t j0 = off[seg], jreal = off[seg] + len[seg];
+    if (t >= jreal) continue;                       // a padding row
+    const int64_t j1 = causal ? t + 1 : jreal;      // keys [j0, j1)
+    const int64_t nk = j1 - j0;
+    // logits and their error bounds
+    double* z = static_cast<double*>(std::malloc(sizeof(double) * nk * 2));
+    double* dz = z + nk;
+    const double sqv = sq[static_cast<int64_t>(h) * T + t];
+    double zmax = -INFINITY, dzmax = 0.0;
+    for (int64_t j = j0; j < j1; ++j) {
+      const double skv = sk[static_cast<int64_t>(g) * T + j];
+      double acc = 0.0, aabs = 0.0;
+      for (int64_t d = 0; d < D; ++d) {
+        const double prod = dec[q[t * Hq * D + h * D + d]] * dec[k[j * Hkv * D + g * D + d]];
+        acc += prod;
+        aabs += std::fabs(prod);
+      }
+      const double c = sqv * skv * inv_sqrt_d;
+      z[j - j0] = acc * c;
+      dz[j - j0] = std::fabs(c) * aabs * std::ldexp(1.0, -16) + std::fabs(z[j - j0]) * std::ldexp(1.0, -21);
+      if (z[j - j0] > zmax) zmax = z[j - j0];
+      if (dz[j - j0] > dzmax) dzmax = dz[j - j0];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < nk; ++j) {
+      z[j] = std::exp(z[j] - zmax);                  // z now holds p
+      l += z[j];
+    }
+    // P . V block by block (128-key blocks at absolute multiples of 128)
+    for (int64_t b0 = (j0 / 128) * 128; b0 < j1; b0 += 128) {
+      const int64_t lo = b0 > j0 ? b0 : j0, hi = (b0 + 128 < j1) ? b0 + 128 : j1;
+      double amax = 0.0, dzb = 0.0;
+      for (int64_t j = lo; j < hi; ++j)
+        if (z[j - j0] > amax) { amax = z[j - j0]; dzb = dz[j - j0]; }
+      const double sb = amax > 0.0 ? amax / 448.0 : 1.0;   // an all-zero block has s = 1
+      const float* svb = sv + (b0 / 128) * (static_cast<int64_t>(Hkv) * D) + static_cast<int64_t>(g) * D;
+      for (int64_t j = lo; j < hi; ++j) {
+        const double tq = z[j - j0] / sb;
+        const uint8_t code = e4m3_encode(static_cast<float>(tq));
+        const double phat = dec[code] * sb;
+        // ambiguity: the nearest rounding midpoint of the E4M3 grid
+        const double eta = dz[j - j0] + dzb + 2.0 * dzmax + std::ldexp(1.0, -19);
+        double step = 0.0;
+        if (tq < 448.0) {
+          const double v = dec[code];
+          const double lo_g = v <= tq ? v : (code > 0 ? dec[code - 1] : 0.0);
+          const double hi_g = v <= tq ? (code < 0x7E ? dec[code + 1] : v) : v;
+          const double mid = 0.5 * (lo_g + hi_g);
+          if (hi_g > lo_g && std::fabs(tq - mid) <= eta * tq) step = hi_g - lo_g;
+        }
+        for (int64_t d = 0; d < D; ++d) {
+          const double vv = dec[vT[(static_cast<int64_t>(g) * D + d) * T + j]] * svb[d];
+          o[d] += phat * vv;
+          oa[d] += std::fabs(phat * vv);
+          of[d] += step * sb * std::fabs(vv);
+        }
+      }
+    }
+    for (int64_t d = 0; d < D; ++d) {
+      o[d] /= l;
+      oa[d] /= l;
+      of[d] /= l;
+    }
+    std::free(z);
+  }
+}
+
 }  // extern "C"
