@@ -49,7 +49,7 @@ def parse():
     p.add_argument("--no-steady", action="store_true", help="skip the >= 1.5 s steady-state region")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--case", default=None,
-                   help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|"
+                   help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|attn|"
                         "requant|bf16_fprop|wgrad_acc|quant_delayed_dy|quant_delayed_x on --layer at "
                         "--tokens, requant_sweep (32 layers), or "
                         "moe_fprop|moe_dgrad|moe_wgrad "
@@ -383,6 +383,32 @@ def moe_calls(fb, mode, layer):
     }
 
 
+def attn_call(fb, seed=0):
+    """FP8 attention forward over the packed long-sequence batch (32768
+    tokens, 4 sequences), Llama-3.1-8B-like heads (32 query heads, 8 KV heads
+    of 128), causal; Q, K, V quantized by the library's activation quantizer.
+    FLOPs count the causal (query, key) pairs of the real tokens only:
+    4 * 128 * Hq * sum_s n_s (n_s + 1) / 2 (Q.K^T and P.V)."""
+    dev = torch.device("cuda", 0)
+    T, Hq, Hkv, D = workloads.PACKED_TOKENS, 32, 8, 128
+    off, ln = workloads.packed_segments(seed)
+    Q = workloads.normal_bf16((T, Hq * D), 1.0, 31, dev)
+    K = workloads.normal_bf16((T, Hkv * D), 1.0, 32, dev)
+    V = workloads.normal_bf16((T, Hkv * D), 1.0, 33, dev)
+    u8, f32 = torch.uint8, torch.float32
+    e = lambda *sh, dt=u8: torch.empty(sh, dtype=dt, device=dev)  # noqa: E731
+    q, sq, k, sk = e(T, Hq * D), e(Hq, T, dt=f32), e(T, Hkv * D), e(Hkv, T, dt=f32)
+    vr, svr, vT, sv = e(T, Hkv * D), e(Hkv, T, dt=f32), e(Hkv * D, T), e(T // 128, Hkv * D, dt=f32)
+    fb.fp8bw_quant_act_1x128(Q, 0, q, sq)
+    fb.fp8bw_quant_act_1x128(K, 0, k, sk)
+    fb.fp8bw_quant_act_1x128(V, 0, vr, svr, vT, sv)
+    o = e(T, Hq * D, dt=torch.bfloat16)
+    offd = torch.tensor(off, dtype=torch.int32, device=dev)
+    lnd = torch.tensor(ln, dtype=torch.int32, device=dev)
+    flops = 4 * D * Hq * sum(n * (n + 1) // 2 for n in ln)
+    return (lambda: fb.fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, offd, lnd, 1), flops, "TFLOP/s")
+
+
 def run_case(args):
     """Times a single call of one layer (used for ncu captures and sweeps)."""
     import blockwise_scaled_fp8_fp8bw_b200 as fb
@@ -393,6 +419,10 @@ def run_case(args):
     if args.case.startswith("moe_"):
         fn, work, unit = moe_calls(fb, mode, name)[args.case]
         time_call(fb, args, name, mode, fn, work, unit)
+        return
+    if args.case == "attn":
+        fn, work, unit = attn_call(fb)
+        time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
         return
     if args.case == "requant_sweep":
         # the per-step requant of 32 layers x 4 weights (about 7B parameters)
@@ -465,6 +495,11 @@ def run_sweep(args):
                 fn, work, unit = calls[c]
                 time_call(fb, args, name, mode, fn, work, unit)
             del calls
+            torch.cuda.empty_cache()
+        if mname == "fp32":
+            args.case = "attn"
+            fn, work, unit = attn_call(fb)
+            time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
             torch.cuda.empty_cache()
         for name in ("gate_up", "down"):
             mc = moe_calls(fb, mode, name)

@@ -26,6 +26,8 @@ FP8BW_FMT_E4M3, FP8BW_FMT_E5M2 = 0, 1
 FP8BW_REQUANT_MAX_PER_LAUNCH = 256
 FP8BW_MAX_EXPERTS = 512
 FP8BW_MAX_HISTORY = 1024
+FP8BW_ATTN_MAX_SEGMENTS = 65536
+FP8BW_ATTN_MAX_HEADS = 1024
 STATUS = {0: "FP8BW_OK", 1: "FP8BW_ERR_INVALID_ARG", 2: "FP8BW_ERR_ALIGNMENT",
           3: "FP8BW_ERR_UNSUPPORTED_ARCH", 4: "FP8BW_ERR_CUDA", 5: "FP8BW_ERR_TIMEOUT",
           6: "FP8BW_ERR_DEVICE_CHECK", 7: "FP8BW_ERR_TOO_LARGE"}
@@ -66,7 +68,9 @@ def _load():
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
     L.fp8bw_quant_tensor_delayed.argtypes = [vp, i64, i64, i64, i32, i32, vp, ctypes.c_int32, vp, vp,
                                              vp, vp, vp, i64, vp]
-    for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm",
+    L.fp8bw_attention_fwd.argtypes = [i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp,
+                                      ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp]
+    for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm", "fp8bw_attention_fwd",
               "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
               "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16",
@@ -233,3 +237,14 @@ def fp8bw_gemm_bf16(A, B, D, stream=None):
     N = B.shape[0]
     _check("fp8bw_gemm_bf16", load().fp8bw_gemm_bf16(M, N, K, _ptr(A), _ptr(B), _ptr(D), D.stride(0),
                                                   _stream(stream)))
+
+
+def fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, seg_off, seg_len, causal=True, stream=None):
+    """FP8 attention forward.  q [T, Hq*128] u8, sq [Hq, T]; k [T, Hkv*128] u8,
+    sk [Hkv, T]; vT [Hkv*128, T] u8, sv [T/128, Hkv*128]; o [T, Hq*128] bf16;
+    seg_off [nseg+1], seg_len [nseg]: device int32."""
+    T = q.shape[0]
+    Hq, Hkv = q.shape[1] // 128, k.shape[1] // 128
+    _check("fp8bw_attention_fwd", load().fp8bw_attention_fwd(
+        T, Hq, Hkv, seg_len.numel(), _ptr(seg_off), _ptr(seg_len), int(bool(causal)), _ptr(q), _ptr(sq),
+        _ptr(k), _ptr(sk), _ptr(vT), _ptr(sv), _ptr(o), _stream(stream)))

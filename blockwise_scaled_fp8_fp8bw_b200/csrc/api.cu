@@ -24,8 +24,13 @@ cudaError_t launch_quant_tensor(const void* x, int64_t M, int64_t K, int64_t ldx
                                 int fmt, float* hist, int H, uint8_t* q, uint8_t* qT,
                                 float* scale, float* amax, float* s_grid, int64_t s_grid_len,
                                 int num_sms, cudaStream_t st);
+cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int32_t* d_off,
+                                 const int32_t* d_len, int causal, const uint8_t* q, const float* sq,
+                                 const uint8_t* k, const float* sk, const uint8_t* vT, const float* sv,
+                                 void* o, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
 cudaError_t quant_read_clear_error(uint32_t* out, cudaStream_t st);
+cudaError_t attn_read_clear_error(uint32_t* out, cudaStream_t st);
 extern int gemm_stall_chunk;
 }  // namespace fp8bw
 
@@ -106,11 +111,12 @@ FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk) {
 }
 
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {
-  uint32_t v = 0, vq = 0;
+  uint32_t v = 0, vq = 0, va = 0;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (fp8bw::gemm_read_clear_error(&v, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
   if (fp8bw::quant_read_clear_error(&vq, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
-  v |= vq;
+  if (fp8bw::attn_read_clear_error(&va, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
+  v |= vq | va;
   if (v & 1u) return FP8BW_ERR_TIMEOUT;
   if (v & 2u) return FP8BW_ERR_DEVICE_CHECK;
   return FP8BW_OK;
@@ -331,6 +337,28 @@ FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int6
   return from_cuda(fp8bw::launch_quant_tensor(x, M, K, ldx, mode, fmt, hist, H, q, qT, scale, amax,
                                               s_grid_len > 0 ? s_grid : nullptr, s_grid_len, sms,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
+                                           const int32_t* d_seg_off, const int32_t* d_seg_len,
+                                           int32_t causal, const uint8_t* q, const float* sq,
+                                           const uint8_t* k, const float* sk, const uint8_t* vT,
+                                           const float* sv, void* o, fp8bw_stream_t stream) {
+  if (!d_seg_off || !d_seg_len || !q || !sq || !k || !sk || !vT || !sv || !o) return FP8BW_ERR_INVALID_ARG;
+  if (T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || nseg < 1 || (causal != 0 && causal != 1))
+    return FP8BW_ERR_INVALID_ARG;
+  if (nseg > FP8BW_ATTN_MAX_SEGMENTS || Hq > FP8BW_ATTN_MAX_HEADS) return FP8BW_ERR_TOO_LARGE;
+  if (T > kMaxDim || T * Hq * 128 > (int64_t(1) << 40)) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(T)) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vT) || !aligned16(sq) || !aligned16(sk) ||
+      !aligned16(sv) || !aligned32(o) || !aligned4(d_seg_off) || !aligned4(d_seg_len))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (T == 0) return FP8BW_OK;
+  return from_cuda(fp8bw::launch_attention_fwd(T, Hq, Hkv, nseg, d_seg_off, d_seg_len, causal, q, sq, k,
+                                               sk, vT, sv, o, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

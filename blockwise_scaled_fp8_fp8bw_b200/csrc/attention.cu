@@ -1,0 +1,518 @@
+// FP8 attention forward for sm_100a: E4M3 Q, K, V with the recipe's 1x128
+// blocks, softmax in fp32, P quantized to E4M3 per 128-key block, both
+// contractions on tcgen05 tensor cores.
+//
+// Method: "NVIDIA NeMo RL erreicht 48% ..." section "Leistungsgewinne in der
+// Praxis": the recipe extends FP8 from the linear layers to the KV cache and
+// the attention operations.  Every FP8 operand carries one scale per 128
+// elements along its contraction ("Der technische Durchbruch": 1x128 blocks
+// for activations): Q and K one per token and head (head dimension 128), V
+// the activation quantizer's column-wise copy (one per 128 tokens of a
+// channel, codes channel-major), and the softmax numerator P one per query
+// row and 128-key block, by the FP32 rule s = amax / 448.
+//
+// One CTA computes a 128-query block of one head over its keys (causal or
+// not, inside one packed sequence; GQA: query head h reads KV head
+// h / (Hq / Hkv)).  384 threads:
+//   warp 0      TMA producer: the Q tile once, then per 128-key block the K
+//               tile [128 keys][128] and the V tile [128 channels][128 keys]
+//               into a 3-stage ring, and the block's 128 key scales and 128
+//               channel scales (bulk copies) into a 4-slot ring
+//   warp 1      MMA issuer (one thread): S_b = Q K_b^T into one of two TMEM
+//               buffers, then O_(b-1) = P_(b-1) V_(b-1)^T into one of two
+//               more, so the tensor core computes the next S while the
+//               softmax warps work on the current one
+//   warps 4-11  softmax and correction, two warps per TMEM lane quarter
+//               (64 of the 128 columns each; a thread owns one query row):
+//               read S_b, scale by the key and query scales, block maximum
+//               (exchanged between the two halves of the row), running
+//               maximum, p = 2^(z - m), partial row sums, P codes into a
+//               shared tile in the MMA's layout; then fold O_(b-1) into the
+//               fp32 output accumulator, kept in TMEM: O = O * 2^(m_old -
+//               m_new) + s_P * s_V[channel] * O_(b-1).
+// At the end O / l is rounded to bf16 and stored; padding query rows get 0.
+// TMEM: S buffers at columns 0 and 128, the P.V product at 256, the output
+// accumulator at 384.  Every wait is bounded; a timeout latches an error bit
+// and the CTA leaves.
+
+#include "common.cuh"
+#include "tmap.cuh"
+
+namespace fp8bw {
+
+__device__ uint32_t g_attn_error;
+
+namespace {
+
+constexpr int kD = 128;              // head dimension (one 1x128 block)
+constexpr int kThreads = 384;
+constexpr int kStages = 3;           // K/V ring
+constexpr int kScSlots = 4;          // scale ring
+constexpr uint32_t kTile = 128 * 128;  // one 128x128 E4M3 tile
+constexpr uint32_t kIdesc = idesc_make(0, 0, 128, 128);  // E4M3 x E4M3 -> F32, M = N = 128
+constexpr float kLog2e = 1.4426950408889634f;
+// setmaxnreg split: 56 registers for warps 0-3, 224 for the softmax warps;
+// 56*128 + 224*256 = 64512 <= 384 * 168, the launch allocation (checked
+// on the host before the launch).
+constexpr int kRegsLow = 56, kRegsHigh = 224, kRegsLaunch = 168;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
+
+struct ScSlot {
+  float sk[128];   // key scales of the block (one per key)
+  float sv[128];   // V scales of the block (one per channel)
+};
+
+struct AttnBars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t sc_full[kScSlots], sc_empty[kScSlots];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t o_full, o_empty;  // the single P.V product buffer
+  uint64_t pair[4];          // the two warps of a TMEM lane quarter meet here
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct AttnSmem {
+  uint8_t q[kTile];                    // 1024-aligned tiles first
+  uint8_t kv[kStages][2][kTile];       // [stage][K, V^T]
+  uint8_t p[2][kTile];
+  ScSlot sc[kScSlots];
+  float red[2][2][128];                // [block parity][half][row]: block maxima
+  float lsum[2][128];                  // [half][row]: row sums at the end
+  AttnBars bars;
+};
+
+struct AttnArgs {
+  int T, Hq, Hkv, nseg, causal;
+  const int32_t* off;   // device [nseg + 1]
+  const int32_t* len;   // device [nseg]
+  const float* sq;      // [Hq][T]
+  const float* sk;      // [Hkv][T]
+  const float* sv;      // [T/128][Hkv*128]
+  uint16_t* o;          // [T][Hq*128] bf16
+};
+
+__device__ __forceinline__ void raise_attn_timeout(AttnBars* b) {
+  atomicOr(&g_attn_error, DEV_ERR_TIMEOUT);
+  atomicExch(&b->abort, 1);
+}
+
+// A bounded wait whose outcome is the same for the whole warp (the warp's
+// tcgen05.ld / st that follow must be executed by all 32 lanes together).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+// Folds O_c (block c's P.V product in TMEM) into the output accumulator
+// (TMEM columns 384..511, this thread's row and 64 columns):
+// acc = acc * alpha + s_P * s_V[channel] * O_c (acc = 0 before block 0),
+// then hands the product buffer and the block's scale slot back.  False if
+// a wait ran out.
+__device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_t tmem, uint32_t lane_off,
+                                          int col0, int lane, int c, float alpha, float sp) {
+  if (!warp_wait(smem_u32(&bars->o_full), c & 1)) return false;
+  tc_fence_after();
+  const uint32_t tp = tmem + lane_off + 256 + col0, to = tmem + lane_off + 384 + col0;
+  const float2 sp2 = make_float2(sp, sp), a2 = make_float2(alpha, alpha);
+  const float4* sv4 = reinterpret_cast<const float4*>(&sm.sc[c % kScSlots].sv[col0]);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint32_t r[32], o[32];
+    tmem_ld32(tp + 32 * u, r);
+    if (c > 0) tmem_ld32(to + 32 * u, o);
+    tmem_wait_ld();
+    tmem_fence_regs(r);
+    if (c > 0) tmem_fence_regs(o);
+    if (u == 1) {
+      // the product is in registers: the next P.V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->o_empty));
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+      const float4 v = sv4[u * 8 + j4];
+      const float2 c0 = fmul2(sp2, make_float2(v.x, v.y));
+      const float2 c1 = fmul2(sp2, make_float2(v.z, v.w));
+      float2 o0 = c > 0 ? fmul2(make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1])), a2)
+                        : make_float2(0.f, 0.f);
+      float2 o1 = c > 0 ? fmul2(make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3])), a2)
+                        : make_float2(0.f, 0.f);
+      o0 = ffma2(make_float2(__uint_as_float(r[4 * j4]), __uint_as_float(r[4 * j4 + 1])), c0, o0);
+      o1 = ffma2(make_float2(__uint_as_float(r[4 * j4 + 2]), __uint_as_float(r[4 * j4 + 3])), c1, o1);
+      o[4 * j4] = __float_as_uint(o0.x);
+      o[4 * j4 + 1] = __float_as_uint(o0.y);
+      o[4 * j4 + 2] = __float_as_uint(o1.x);
+      o[4 * j4 + 3] = __float_as_uint(o1.y);
+    }
+    tmem_st32(to + 32 * u, o);
+  }
+  tmem_wait_st();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars->sc_empty[c % kScSlots]));
+  return true;
+}
+
+// The two warps of lane quarter q meet (each after writing its half's value
+// to shared memory); `uses` counts this quarter's earlier meetings.  False if
+// the other warp did not arrive in time.
+__device__ __forceinline__ bool pair_meet(AttnBars* bars, int q, int lane, uint32_t uses) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars->pair[q]));
+  return warp_wait(smem_u32(&bars->pair[q]), uses & 1);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  AttnBars* bars = &sm.bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- which block: heavy (late) query blocks first
+  const int nqb = a.T / 128;
+  const int qb = nqb - 1 - (int)(blockIdx.x / a.Hq);
+  const int h = (int)(blockIdx.x % a.Hq);
+  const int g = h / (a.Hq / a.Hkv);
+  const int q0 = qb * 128;
+
+  // ---- validate the segment table (every CTA; nothing written if invalid)
+  __shared__ int s_seg;
+  if (threadIdx.x == 0) s_seg = -1;
+  __syncthreads();
+  {
+    int bad = 0;
+    for (int i = threadIdx.x; i < a.nseg; i += kThreads) {
+      const int o0 = a.off[i], o1 = a.off[i + 1], ln = a.len[i];
+      if (o1 < o0 || (o0 & 127) || (o1 & 127) || ln < 0 || ln > o1 - o0 || (i == 0 && o0 != 0)) bad = 1;
+      if (o0 <= q0 && q0 < o1) s_seg = i;   // at most one segment holds the block
+    }
+    if (threadIdx.x == 0 && a.off[a.nseg] > a.T) bad = 1;
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) atomicOr(&g_attn_error, DEV_ERR_CHECK);
+      return;
+    }
+  }
+  const int seg = s_seg;                      // -1: past the last segment
+  const int j0 = seg >= 0 ? a.off[seg] : q0;
+  const int jreal = seg >= 0 ? j0 + a.len[seg] : q0;   // first padding token of the segment
+  uint16_t* orow_base = a.o + (size_t)h * kD;
+  const size_t ostride = (size_t)a.Hq * kD;
+
+  if (q0 >= jreal) {
+    // the whole query block is padding: zeros
+    for (int idx = threadIdx.x; idx < 128 * 8; idx += kThreads) {
+      const int r = idx >> 3, c = idx & 7;
+      st_global_v8(orow_base + (size_t)(q0 + r) * ostride + c * 16, make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0));
+    }
+    return;
+  }
+  const int kb_first = j0 / 128;
+  const int kb_last = a.causal ? min(qb, (jreal - 1) / 128) : (jreal - 1) / 128;
+  const int nb = kb_last - kb_first + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->kv_full[i]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < kScSlots; ++i) {
+      mbar_init(smem_u32(&bars->sc_full[i]), 1);
+      mbar_init(smem_u32(&bars->sc_empty[i]), 8);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->s_empty[i]), 8);
+      mbar_init(smem_u32(&bars->p_full[i]), 8);
+      mbar_init(smem_u32(&bars->p_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&bars->o_full), 1);
+    mbar_init(smem_u32(&bars->o_empty), 8);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), 2);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kTile);
+      tma_load_2d(smem_u32(sm.q), &tmQ, smem_u32(&bars->q_full), h * kD, q0);
+      for (int b = 0; b < nb; ++b) {
+        const int kb = kb_first + b, s = b % kStages, sl = b % kScSlots;
+        if (!mbar_wait(smem_u32(&bars->kv_empty[s]), ((b / kStages) & 1) ^ 1)) {
+          raise_attn_timeout(bars);
+          break;
+        }
+        mbar_arrive_expect_tx(smem_u32(&bars->kv_full[s]), 2 * kTile);
+        tma_load_2d(smem_u32(sm.kv[s][0]), &tmK, smem_u32(&bars->kv_full[s]), g * kD, kb * 128);
+        tma_load_2d(smem_u32(sm.kv[s][1]), &tmV, smem_u32(&bars->kv_full[s]), kb * 128, g * kD);
+        if (!mbar_wait(smem_u32(&bars->sc_empty[sl]), ((b / kScSlots) & 1) ^ 1)) {
+          raise_attn_timeout(bars);
+          break;
+        }
+        mbar_arrive_expect_tx(smem_u32(&bars->sc_full[sl]), 1024);
+        bulk_load(smem_u32(sm.sc[sl].sk), a.sk + (size_t)g * a.T + kb * 128, 512, smem_u32(&bars->sc_full[sl]));
+        bulk_load(smem_u32(sm.sc[sl].sv), a.sv + (size_t)kb * a.Hkv * kD + g * kD, 512,
+                  smem_u32(&bars->sc_full[sl]));
+        if (bars->abort) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
+      tc_fence_after();
+      const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q));
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
+          const int s = b % kStages;
+          if (!mbar_wait(smem_u32(&bars->kv_full[s]), (b / kStages) & 1) ||
+              !mbar_wait(smem_u32(&bars->s_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.kv[s][0]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f8f6f4(tmem + (b & 1) * 128, dq + 2 * kk, dk + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+          umma_commit(smem_u32(&bars->s_full[b & 1]));
+        }
+        if (b >= 1) {
+          const int c = b - 1, s = c % kStages;
+          if (!mbar_wait(smem_u32(&bars->p_full[c & 1]), (c >> 1) & 1) ||
+              !mbar_wait(smem_u32(&bars->o_empty), (c & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dp = sdesc_k_sw128(smem_u32(sm.p[c & 1]));
+          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.kv[s][1]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f8f6f4(tmem + 256, dp + 2 * kk, dv + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+          umma_commit(smem_u32(&bars->p_empty[c & 1]));
+          umma_commit(smem_u32(&bars->o_full));
+          umma_commit(smem_u32(&bars->kv_empty[s]));
+        }
+        if (bars->abort) break;
+      }
+      if (!ok) raise_attn_timeout(bars);
+    }
+  }
+  } else {
+    regs_inc<kRegsHigh>();
+    // --------------------------------------------- softmax and correction --
+    const int q = warp & 3, hf = (warp - 4) >> 2;
+    const int i = q * 32 + lane, t = q0 + i;
+    const int col0 = hf * 64;                       // this thread's 64 columns
+    const float cq = a.sq[(size_t)h * a.T + t] * (kLog2e * 0.08838834764831845f);  // sq * log2(e) / sqrt(128)
+    // keys of this row: [j0, jend); a block needs a mask where it reaches jend
+    const int jend = a.causal ? min(jreal, t + 1) : jreal;
+    float m = -INFINITY, lh = 0.0f;
+    float a_prev = 0.0f, sp_prev = 0.0f;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    uint32_t meets = 0;
+
+    for (int b = 0; b < nb && ok; ++b) {
+      const int kb = kb_first + b;
+      if (!warp_wait(smem_u32(&bars->sc_full[b % kScSlots]), (b / kScSlots) & 1) ||
+          !warp_wait(smem_u32(&bars->s_full[b & 1]), (b >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[2][32];
+      const uint32_t ta = tmem + lane_off + (b & 1) * 128 + col0;
+      tmem_ld32(ta, r[0]);
+      tmem_ld32(ta + 32, r[1]);
+      tmem_wait_ld();
+      tmem_fence_regs(r[0]);
+      tmem_fence_regs(r[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b & 1]));
+
+      // y = (q . k) * s_k per key; the query scale and 1/sqrt(d) log2(e)
+      // (cq > 0) are applied after the maximum
+      const int lim = jend - kb * 128 - col0;      // columns >= lim are masked
+      const float4* sk4 = reinterpret_cast<const float4*>(&sm.sc[b % kScSlots].sk[col0]);
+      // in place: r becomes y = s_k * (q . k), then p (as fp32 bits)
+      float mh = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 kv4 = sk4[u * 8 + j4];
+          const float2 p0 = fmul2(make_float2(__uint_as_float(r[u][4 * j4]), __uint_as_float(r[u][4 * j4 + 1])),
+                                  make_float2(kv4.x, kv4.y));
+          const float2 p1 = fmul2(make_float2(__uint_as_float(r[u][4 * j4 + 2]), __uint_as_float(r[u][4 * j4 + 3])),
+                                  make_float2(kv4.z, kv4.w));
+          r[u][4 * j4] = __float_as_uint(p0.x);
+          r[u][4 * j4 + 1] = __float_as_uint(p0.y);
+          r[u][4 * j4 + 2] = __float_as_uint(p1.x);
+          r[u][4 * j4 + 3] = __float_as_uint(p1.y);
+        }
+      }
+      if (lim < 64) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+      }
+#pragma unroll
+      for (int j = 0; j < 64; ++j) mh = fmaxf(mh, __uint_as_float(r[j >> 5][j & 31]));
+      // block maximum of the row: combine the two halves
+      sm.red[b & 1][hf][i] = mh;
+      if (!pair_meet(bars, q, lane, meets++)) {
+        ok = false;
+        break;
+      }
+      const float mb = fmaxf(sm.red[b & 1][0][i], sm.red[b & 1][1][i]) * cq;
+      const float m_new = fmaxf(m, mb);
+      const float alpha = ex2(m - m_new);       // 0 on the first block
+      m = m_new;
+      float ps = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const float pj = ex2(__fmaf_rn(__uint_as_float(r[j >> 5][j & 31]), cq, -m_new));
+        r[j >> 5][j & 31] = __float_as_uint(pj);
+        ps += pj;
+      }
+      lh = lh * alpha + ps;
+      // P's block scale: amax / 448 with amax = 2^(mb - m) the block's largest p
+      const float amax = ex2(mb - m_new);
+      const float sp = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      const float inv = amax > 0.0f ? __fdiv_rn(1.0f, sp) : 0.0f;
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int u = j >> 3, k = 4 * (j & 7);
+        w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]) * inv, __uint_as_float(r[u][k + 1]) * inv) |
+               (cvt_e4m3x2(__uint_as_float(r[u][k + 2]) * inv, __uint_as_float(r[u][k + 3]) * inv) << 16);
+      }
+      if (!warp_wait(smem_u32(&bars->p_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      // row i of the P tile: 16-byte chunk c at c ^ (i & 7) (128-byte swizzle)
+      uint8_t* prow = sm.p[b & 1] + i * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(prow + (((hf * 4 + c) ^ (i & 7)) << 4)) =
+            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[b & 1]));
+      if (b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) ok = false;
+      a_prev = alpha;
+      sp_prev = sp;
+      if (bars->abort) ok = false;
+    }
+    if (ok && !fold_block(sm, bars, tmem, lane_off, col0, lane, nb - 1, a_prev, sp_prev)) ok = false;
+    if (!ok) raise_attn_timeout(bars);
+    // row sum of both halves, then O / l in bf16 (padding rows: 0)
+    sm.lsum[hf][i] = lh;
+    if (!pair_meet(bars, q, lane, meets++)) ok = false;
+    const float l = sm.lsum[0][i] + sm.lsum[1][i];
+    const bool real = t < jreal && ok;
+    const float il = real ? __fdiv_rn(1.0f, l) : 0.0f;
+    uint16_t* orow = orow_base + (size_t)t * ostride + col0;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_off + 384 + col0 + 32 * u, o);
+      tmem_wait_ld();
+      tmem_fence_regs(o);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          o8[j] = real ? pack_bf16x2(__uint_as_float(o[16 * c + 2 * j]) * il, __uint_as_float(o[16 * c + 2 * j + 1]) * il)
+                       : 0u;
+        st_global_v8(orow + 32 * u + 16 * c, make_uint4(o8[0], o8[1], o8[2], o8[3]),
+                     make_uint4(o8[4], o8[5], o8[6], o8[7]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int32_t* d_off,
+                                 const int32_t* d_len, int causal, const uint8_t* q, const float* sq,
+                                 const uint8_t* k, const float* sk, const uint8_t* vT, const float* sv,
+                                 void* o, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, (uint64_t)Hq * kD, (uint64_t)T,
+                (uint64_t)Hq * kD, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, (uint64_t)Hkv * kD, (uint64_t)T,
+                (uint64_t)Hkv * kD, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, vT, (uint64_t)T, (uint64_t)Hkv * kD,
+                (uint64_t)T, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  AttnArgs a;
+  a.T = (int)T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.nseg = nseg;
+  a.causal = causal;
+  a.off = d_off;
+  a.len = d_len;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.o = static_cast<uint16_t*>(o);
+  const size_t smem = sizeof(AttnSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, k_attn_fwd);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg draws on the launch allocation: refuse to launch if the
+  // compiled register count could not cover the split.
+  if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
+  const unsigned grid = (unsigned)((T / 128) * Hq);
+  k_attn_fwd<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+cudaError_t attn_read_clear_error(uint32_t* out, cudaStream_t st) {
+  uint32_t v = 0, z = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_attn_error, sizeof v, 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbolAsync(g_attn_error, &z, sizeof z, 0, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *out = v;
+  return e;
+}
+
+}  // namespace fp8bw

@@ -85,7 +85,7 @@ FP8BW_API fp8bw_status fp8bw_init(int device);
 FP8BW_API const char* fp8bw_status_string(fp8bw_status s);
 
 /* Synchronizes `stream`, then returns (and clears) the device error words of
- * the current device (one for the GEMMs, one for the quantizers):
+ * the current device (one each for the GEMMs, the quantizers and attention):
  * FP8BW_ERR_TIMEOUT if a kernel's bounded wait ran out, FP8BW_ERR_DEVICE_CHECK
  * if a kernel rejected its device-side arguments (grouped offsets, or
  * FP8BW_SCALE_POW2 scales that are not powers of two), else FP8BW_OK.
@@ -300,6 +300,44 @@ FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int6
                                         int32_t H, uint8_t* q, uint8_t* qT, float* scale,
                                         float* amax, float* s_grid, int64_t s_grid_len,
                                         fp8bw_stream_t stream);
+
+/* FP8 attention forward ("NVIDIA NeMo RL erreicht 48% ...", section
+ * "Leistungsgewinne in der Praxis": the recipe extends FP8 to the KV cache
+ * and the attention operations).  Head dimension 128.  Every operand is
+ * E4M3 with one scale per 128 elements along its contraction, as the
+ * activation quantizer makes them:
+ *   q   [T][Hq*128] codes, sq [Hq][T]: fp8bw_quant_act_1x128 of Q [T][Hq*128]
+ *       (row-wise; one scale per token and head)
+ *   k   [T][Hkv*128] codes, sk [Hkv][T]: the same for K (the key cache)
+ *   vT  [Hkv*128][T] codes, sv [T/128][Hkv*128]: the column-wise copy
+ *       (q_col, s_col) of V [T][Hkv*128] (one scale per 128 tokens of one
+ *       channel; the value cache, channel-major)
+ *   o   [T][Hq*128] bf16 output, 32-byte aligned.
+ * Query head h reads key/value head h / (Hq / Hkv).  Tokens are packed
+ * sequences: segment s covers tokens [off[s], off[s+1]) (DEVICE arrays
+ * d_seg_off [nseg+1], d_seg_len [nseg]; offsets non-decreasing multiples of
+ * 128, off[0] = 0, off[nseg] <= T), of which the first len[s] are real.  A
+ * real query token t attends to the real tokens of its segment (causal = 1:
+ * only those j <= t).  Per query row: logits z_j = (q^ . k^_j) / sqrt(128)
+ * (q^, k^ dequantized), p_j = exp(z_j - max z), l = sum_j p_j; P is
+ * quantized to E4M3 per 128-key block with the FP32 scale rule s = amax/448
+ * (codes E4M3(p / s)); o = sum_j p^_j v^_j / l in bf16.  Padding rows (past
+ * len[s], or past off[nseg]) are written as zeros.  The result is within
+ * |o - ref| <= 1e-2 * sum_j |p^_j v^_j| / l + (one E4M3 step of each p_j
+ * whose p / s lies within the kernel's fp32 error of a rounding midpoint)
+ * + 1 bf16 ulp of the fp64 reference of the same definition.
+ * Requires T a multiple of 128, Hq a multiple of Hkv, Hq <=
+ * FP8BW_ATTN_MAX_HEADS, 1 <= nseg <= FP8BW_ATTN_MAX_SEGMENTS, 16-byte
+ * aligned codes and scales.  Invalid offsets are rejected on the device:
+ * nothing is written and fp8bw_last_device_error() reports
+ * FP8BW_ERR_DEVICE_CHECK. */
+#define FP8BW_ATTN_MAX_SEGMENTS 65536
+#define FP8BW_ATTN_MAX_HEADS 1024
+FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
+                                           const int32_t* d_seg_off, const int32_t* d_seg_len,
+                                           int32_t causal, const uint8_t* q, const float* sq,
+                                           const uint8_t* k, const float* sk, const uint8_t* vT,
+                                           const float* sv, void* o, fp8bw_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -81,3 +81,16 @@ def test_packed_batch_padding():
     v = x[mask].float().flatten()
     kurt = float(((v - v.mean()) ** 4).mean() / v.var() ** 2) - 3.0
     assert kurt > 3.0
+
+
+def test_packed_segments_match_mask():
+    """The segment table of the packing marks exactly the mask's real tokens,
+    with 128-aligned segment starts covering the whole batch."""
+    off, ln = wl.packed_segments(0)
+    mask = wl.packed_rows_mask(0)
+    assert off[0] == 0 and off[-1] == wl.PACKED_TOKENS
+    assert all(o % 128 == 0 for o in off)
+    want = torch.zeros(wl.PACKED_TOKENS, dtype=torch.bool)
+    for a, n in zip(off, ln):
+        want[a:a + n] = True
+    assert torch.equal(want, mask)

@@ -194,6 +194,22 @@ def packed_rows_mask(seed: int = 0, total: int = PACKED_TOKENS):
     return mask
 
 
+def packed_segments(seed: int = 0, total: int = PACKED_TOKENS):
+    """(offsets, lengths) of the packing drawn by packed_rows_mask: segment s
+    covers tokens [off[s], off[s+1]) (each sequence padded to a multiple of
+    128, the last one cut at `total`), of which the first len[s] are real."""
+    lens = packed_lengths(seed, total=total)
+    off, ln = [0], []
+    pos = 0
+    for L in lens:
+        if pos >= total:
+            break
+        ln.append(min(L, total - pos))
+        pos += min(((L + 127) // 128) * 128, total - pos)
+        off.append(pos)
+    return off, ln
+
+
 def packed_activations(K: int, seed: int = 0, device="cpu", total: int = PACKED_TOKENS,
                        scale: float = 1.0, mask_seed: int = 0):
     """[total, K] Student-t (nu=3) values times `scale`, zero on the padding
