@@ -68,9 +68,11 @@ def _load():
     L.fp8bw_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp]
     L.fp8bw_quant_tensor_delayed.argtypes = [vp, i64, i64, i64, i32, i32, vp, ctypes.c_int32, vp, vp,
                                              vp, vp, vp, i64, vp]
+    L.fp8bw_gemm_quant.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, i32, vp, i64, vp, vp, vp, vp, vp]
     L.fp8bw_attention_fwd.argtypes = [i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp,
                                       ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm", "fp8bw_attention_fwd",
+              "fp8bw_gemm_quant",
               "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
               "fp8bw_gemm_f32", "fp8bw_grouped_gemm", "fp8bw_grouped_wgrad_f32", "fp8bw_gemm_bf16",
@@ -248,3 +250,16 @@ def fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, seg_off, seg_len, causal=True, 
     _check("fp8bw_attention_fwd", load().fp8bw_attention_fwd(
         T, Hq, Hkv, seg_len.numel(), _ptr(seg_off), _ptr(seg_len), int(bool(causal)), _ptr(q), _ptr(sq),
         _ptr(k), _ptr(sk), _ptr(vT), _ptr(sv), _ptr(o), _stream(stream)))
+
+
+def fp8bw_gemm_quant(kind, A, sA, B, sB, q_row, s_row, q_col=None, s_col=None, D=None,
+                     mode=FP8BW_SCALE_FP32, stream=None):
+    """The GEMM with its bf16 output quantized in the epilogue (scale rule
+    `mode`): q_row [M,N] u8, s_row [N/128,M]; q_col [N,M] / s_col [M/128,N] or
+    None; D [M, ldd>=N] bf16 or None."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check("fp8bw_gemm_quant", load().fp8bw_gemm_quant(
+        int(kind), M, N, K, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), int(mode), _ptr(D),
+        D.stride(0) if D is not None else 0, _ptr(q_row), _ptr(s_row), _ptr(q_col), _ptr(s_col),
+        _stream(stream)))

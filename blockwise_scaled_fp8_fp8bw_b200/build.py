@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libfp8bw.so")
 SOURCES = ["quant.cu", "quant_tensor.cu", "gemm.cu", "attention.cu", "api.cu"]
-HEADERS = ["common.cuh", "tmap.cuh"]
+HEADERS = ["common.cuh", "tmap.cuh", "blockquant.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 # IEEE division and denormals stay on (no --use_fast_math, no -ftz): the

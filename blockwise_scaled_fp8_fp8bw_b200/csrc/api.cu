@@ -18,6 +18,10 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
                             int64_t N, int64_t K, const uint8_t* A, const float* sA,
                             const uint8_t* B, const float* sB, void* D, int64_t ldd, int mode,
                             int num_sms, cudaStream_t st, int out_mode, int a_fmt = 0, int b_fmt = 0);
+cudaError_t launch_gemm_quant(int kind, int64_t M, int64_t N, int64_t K, const uint8_t* A, const float* sA,
+                              const uint8_t* B, const float* sB, int qmode, void* D, int64_t ldd,
+                              uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, int num_sms,
+                              cudaStream_t st);
 cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                              void* D, int64_t ldd, int num_sms, cudaStream_t st);
 cudaError_t launch_quant_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, int mode,
@@ -337,6 +341,30 @@ FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int6
   return from_cuda(fp8bw::launch_quant_tensor(x, M, K, ldx, mode, fmt, hist, H, q, qT, scale, amax,
                                               s_grid_len > 0 ? s_grid : nullptr, s_grid_len, sms,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_gemm_quant(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                                        const uint8_t* A, const float* sA, const uint8_t* B,
+                                        const float* sB, fp8bw_scale_mode out_mode, void* D, int64_t ldd,
+                                        uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
+                                        fp8bw_stream_t stream) {
+  if (kind != FP8BW_FPROP && kind != FP8BW_DGRAD && kind != FP8BW_WGRAD) return FP8BW_ERR_INVALID_ARG;
+  if (out_mode != FP8BW_SCALE_FP32 && out_mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
+  if (!A || !sA || !B || !sB || !q_row || !s_row) return FP8BW_ERR_INVALID_ARG;
+  if ((q_col == nullptr) != (s_col == nullptr)) return FP8BW_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || (D && ldd < N)) return FP8BW_ERR_INVALID_ARG;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(M) || !mult128(N) || !mult128(K) || (D && (ldd & 7) != 0)) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sA) || !aligned16(sB) || (D && !aligned16(D)) ||
+      !aligned32(q_row) || !aligned16(s_row) || (q_col && !aligned32(q_col)) || (s_col && !aligned16(s_col)))
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (M == 0 || N == 0) return FP8BW_OK;
+  if (K == 0) return FP8BW_ERR_INVALID_ARG;
+  return from_cuda(fp8bw::launch_gemm_quant(kind, M, N, K, A, sA, B, sB, out_mode, D, ldd, q_row, s_row,
+                                            q_col, s_col, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,

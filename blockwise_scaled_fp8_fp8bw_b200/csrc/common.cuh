@@ -487,6 +487,17 @@ __device__ __forceinline__ void umma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc
       : "memory");
 }
 
+// Pair form of umma_f16 (BF16 x BF16 -> F32, M = 256 over the pair).
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the mbarrier at offset `bar` in every CTA of `mask` once the
 // pair's tcgen05.mma issued so far by this thread are done.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {

@@ -41,6 +41,9 @@
 // Every wait is bounded; on a timeout the kernel latches an error bit and
 // leaves its loops.
 
+#include <cstring>
+
+#include "blockquant.cuh"
 #include "common.cuh"
 #include "tmap.cuh"
 
@@ -61,18 +64,27 @@ constexpr uint32_t kEpiPiece = 2048;  // 32 rows x 32 bf16 (or 16 fp32): one TMA
 // Output of the FP8 GEMMs: bf16 (the default), fp32, or fp32 added to D.
 enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F32_ADD = 2 };
 
-template <bool PAIR>
+// Epilogue kind of the promotion kernel (a template parameter): bf16 tiles,
+// fp32 tiles (stored or added, per OutMode), or the bf16 result quantized
+// into 1x128 row blocks and the column-wise copy (FP32 or POW2 scale rule).
+enum OutKind : int { OK_BF16 = 0, OK_F32 = 1, OK_QUANT_FP32 = 2, OK_QUANT_POW2 = 3 };
+
+// Quantizing epilogue: per column half of the tile (4 warps, 128 rows x 128
+// columns) a swizzled bf16 tile, the partial column maxima and a barrier.
+constexpr uint32_t kQHalfBytes = 40960;
+constexpr uint32_t kQColmaxOff = 32768, kQBarOff = 33280;
+
+template <bool PAIR, bool QOUT = false>
 struct Cfg {
   static constexpr uint32_t kBTile = PAIR ? (BN / 2) * BK : BN * BK;  // this CTA's B rows
   static constexpr uint32_t kStageBytes = kATile + kBTile;
-  static constexpr int kStages = PAIR ? 5 : 4;
+  static constexpr int kStages = QOUT ? 4 : (PAIR ? 5 : 4);
   static constexpr int kEpiBufs = PAIR ? 3 : 1;  // staging pieces per promotion warp
-  static constexpr uint32_t kEpiBytes = kEpiBufs * kEpiPiece;
+  static constexpr uint32_t kEpiBytes = QOUT ? kQHalfBytes / 4 : kEpiBufs * kEpiPiece;
   static constexpr uint32_t kIdesc = idesc_make(0, 0, PAIR ? 2 * BM : BM, BN);  // E4M3 -> F32
   static constexpr uint32_t kTemptyCount = PAIR ? 16 : 8;
 };
 
-constexpr uint32_t kIdescBF16 = idesc_make(1, 1, BM, BN);  // BF16 x BF16 -> F32
 
 constexpr int kRegsLow = 56, kRegsHigh = 224, kRegsLaunch = 168;
 static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
@@ -99,20 +111,124 @@ struct GemmArgs {
   const float* sB;     // per kind
   const int32_t* offsets;  // grouped: device [G+1]
   int G;
-  uint16_t* D;         // BF16 kernel only (the FP8 kernel stores through a tensor map)
+  uint16_t* D;         // quantizing epilogue: optional bf16 copy of the result
   int64_t ldd;
+  uint8_t* q_row;      // quantizing epilogue: [M][N] codes, s_row [N/128][M]
+  float* s_row;
+  uint8_t* q_col;      // column-wise copy [N][M], s_col [M/128][N]
+  float* s_col;
   int out_mode;        // OutMode of the FP8 kernels' epilogue
   uint32_t fmt_bits;   // operand formats in the MMA instruction descriptor (0: both E4M3)
   int stall_chunk;     // testing: CTA 0's producer never fills this chunk (-1: off)
 };
 
-template <bool PAIR>
+template <bool PAIR, bool QOUT = false>
 constexpr size_t smem_fp8() {
-  return 1024 + size_t(Cfg<PAIR>::kStages) * Cfg<PAIR>::kStageBytes +
-         size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * Cfg<PAIR>::kEpiBytes + sizeof(Bars) +
+  return 1024 + size_t(Cfg<PAIR, QOUT>::kStages) * Cfg<PAIR, QOUT>::kStageBytes +
+         size_t(kScaleStages) * sizeof(ScaleSlot) + 8 * Cfg<PAIR, QOUT>::kEpiBytes + sizeof(Bars) +
          2 * sizeof(int32_t) * (kMaxGroups + 1);
 }
-static_assert(smem_fp8<true>() <= 232448 && smem_fp8<false>() <= 232448, "shared memory budget");
+static_assert(smem_fp8<true>() <= 232448 && smem_fp8<false>() <= 232448 && smem_fp8<true, true>() <= 232448,
+              "shared memory budget");
+
+// The four warps of one column half meet (bounded); `uses` counts the
+// half's earlier meetings.  False if a warp did not arrive in time.
+__device__ __forceinline__ bool half_meet(uint32_t bar, int lane, uint32_t uses) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  return __all_sync(0xffffffffu, mbar_wait(bar, uses & 1));
+}
+
+// Quantizing epilogue of one column half: this thread holds row `rr` (of the
+// CTA's 128) of the bf16-rounded result, 128 columns as 64 packed words.
+// Writes D (if requested), the row codes and scale of its 1x128 block, and,
+// with the other 127 threads of the half, the column-wise copy of the
+// 128x128 tile: exactly what fp8bw_quant_act_1x128 makes of D.
+template <int QM>
+__device__ __forceinline__ bool quant_epilogue(const GemmArgs& a, uint8_t* hb, int tid, int lane,
+                                               uint32_t& uses, int row0, int col0, const uint32_t (&w)[64]) {
+  const int rr = tid;                      // the thread's row within the tile
+  const int64_t grow = row0 + rr;
+  const int64_t M = a.M, N = a.N;
+  if (a.D) {
+    uint4* drow = reinterpret_cast<uint4*>(a.D + grow * a.ldd + col0);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) drow[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  }
+  // row pass: the thread's 128 values are one 1x128 block
+  {
+    uint32_t m = 0;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) m = umax2(m, w[k] & kAbsMask);
+    const Divisor d = make_divisor<QM>(halves_max(m));
+    a.s_row[(col0 / 128) * M + grow] = d.s;
+    uint8_t* qr = a.q_row + grow * N + col0;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const uint2 c0 = quant8<QM>(make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]), d);
+      const uint2 c1 = quant8<QM>(make_uint4(w[4 * k + 4], w[4 * k + 5], w[4 * k + 6], w[4 * k + 7]), d);
+      const uint2 c2 = quant8<QM>(make_uint4(w[4 * k + 8], w[4 * k + 9], w[4 * k + 10], w[4 * k + 11]), d);
+      const uint2 c3 = quant8<QM>(make_uint4(w[4 * k + 12], w[4 * k + 13], w[4 * k + 14], w[4 * k + 15]), d);
+      st_global_v8(qr + 8 * k, make_uint4(c0.x, c0.y, c1.x, c1.y), make_uint4(c2.x, c2.y, c3.x, c3.y));
+    }
+  }
+  if (!a.q_col) return true;
+  // column-wise copy: the tile goes through shared memory (two boxes of 64
+  // columns, 128-byte swizzle), a thread takes two columns x 64 rows
+  const uint32_t bar = smem_u32(hb + kQBarOff);
+  uint32_t* colmax = reinterpret_cast<uint32_t*>(hb + kQColmaxOff);
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    *reinterpret_cast<uint4*>(hb + act_off(k >> 3, rr, k & 7)) = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  if (!half_meet(bar, lane, uses++)) return false;
+  const int wc = tid & 63, rg = tid >> 6;
+  const int cbox = wc >> 5, cchunk = (wc & 31) >> 2, cword = wc & 3;
+  ColWords cw[2];
+  uint32_t m = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      cw[h].w[r] = *reinterpret_cast<const uint32_t*>(hb + act_off(cbox, rg * 64 + h * 32 + r, cchunk) + 4 * cword);
+      m = umax2(m, cw[h].w[r] & kAbsMask);
+    }
+  colmax[rg * 64 + wc] = m;
+  if (!half_meet(bar, lane, uses++)) return false;
+  m = umax2(colmax[wc], colmax[64 + wc]);
+  const Divisor d0 = make_divisor<QM>(__uint_as_float((m & 0xFFFFu) << 16));
+  const Divisor d1 = make_divisor<QM>(__uint_as_float(m & 0xFFFF0000u));
+  if (rg == 0) *reinterpret_cast<float2*>(a.s_col + (int64_t)(row0 / 128) * N + col0 + 2 * wc) = make_float2(d0.s, d1.s);
+  const bool slow = QM == FP8BW_SCALE_FP32 && __any_sync(0xffffffffu, d0.exact || d1.exact);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t c0[8], c1[8];
+    if (slow) {
+      const ColCodes c = column_codes_exact<FP8BW_FMT_E4M3>(cw[h], d0, d1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c0[j] = c.c0[j];
+        c1[j] = c.c1[j];
+      }
+    } else {
+      const float2 s2 = make_float2(d0.s, d1.s), y2 = make_float2(d0.y, d1.y);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float2 qv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t x = cw[h].w[4 * j + u];
+          qv[u] = div2<QM>(make_float2(bf16lo(x), bf16hi(x)), s2, y2);
+        }
+        c0[j] = cvt_e4m3x2(qv[0].x, qv[1].x) | (cvt_e4m3x2(qv[2].x, qv[3].x) << 16);
+        c1[j] = cvt_e4m3x2(qv[0].y, qv[1].y) | (cvt_e4m3x2(qv[2].y, qv[3].y) << 16);
+      }
+    }
+    uint8_t* qc = a.q_col + (int64_t)(col0 + 2 * wc) * M + row0 + rg * 64 + h * 32;
+    st_global_v8(qc, make_uint4(c0[0], c0[1], c0[2], c0[3]), make_uint4(c0[4], c0[5], c0[6], c0[7]));
+    st_global_v8(qc + M, make_uint4(c1[0], c1[1], c1[2], c1[3]), make_uint4(c1[4], c1[5], c1[6], c1[7]));
+  }
+  return true;
+}
 
 struct TileInfo {
   int mt, nt, g, kb0, kb1;
@@ -243,11 +359,14 @@ __device__ __forceinline__ void raise_timeout_mx(B* bars) {
   atomicExch(&bars->abort, 1);
 }
 
-template <int KIND, bool GROUPED, bool PAIR, bool F32OUT>
+template <int KIND, bool GROUPED, bool PAIR, int OUTK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
-  using C = Cfg<PAIR>;
+  constexpr bool F32OUT = OUTK == OK_F32;
+  constexpr bool QOUT = OUTK == OK_QUANT_FP32 || OUTK == OK_QUANT_POW2;
+  static_assert(!(QOUT && GROUPED), "quantizing epilogue: dense GEMMs only");
+  using C = Cfg<PAIR, QOUT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -278,6 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->tfull[i]), 1);
       mbar_init(smem_u32(&bars->tempty[i]), C::kTemptyCount);
     }
+    if (QOUT)
+      for (int h = 0; h < 2; ++h) mbar_init(smem_u32(epi_base + h * kQHalfBytes + kQBarOff), 4);
     bars->abort = 0;
     bars->bad_offsets = 0;
     fence_barrier_init();
@@ -453,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int half = (warp - 4) >> 2;  // column half of the 256-wide tile
     uint8_t* epi0 = epi_base + (warp - 4) * C::kEpiBytes;
+    uint32_t qmeets = 0;  // quantizing epilogue: meetings of this column half
     int ss = 0;
     uint32_t sphase = 0;
     int buf = 0;
@@ -537,6 +659,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // segment, computed nothing real)
       if (row0 >= ti.mend) {
         // nothing of this CTA's rows is part of the result
+      } else if (QOUT) {
+        if (col0 < a.N) {
+          uint32_t w[64];
+#pragma unroll
+          for (int j = 0; j < 64; ++j) w[j] = pack_bf16x2(acc[j].x, acc[j].y);
+          if (!quant_epilogue<OUTK == OK_QUANT_POW2 ? FP8BW_SCALE_POW2 : FP8BW_SCALE_FP32>(
+                  a, epi_base + half * kQHalfBytes, q * 32 + lane, lane, qmeets, row0, col0, w)) {
+            raise_timeout(bars);
+            goto done;
+          }
+        }
       } else if (F32OUT) {
         // fp32 output: eight 32x16 pieces per warp, stored or added to D
 #pragma unroll
@@ -1062,151 +1195,187 @@ done:
 }
 
 // ------------------------------------------------------------ BF16 GEMM ---
-// Same pipeline without scales: BK = 64 bf16 (128-byte rows), four
-// kind::f16 MMAs (K = 16) per stage, the accumulator stays in TMEM for the
-// whole K loop, and the 8 epilogue warps drain a finished tile (double
-// buffered in TMEM) while the next tile accumulates.
+// The BF16 comparison GEMM on the same CTA-pair tiles as the FP8 kernels
+// (256x256 per pair, tcgen05.mma.cta_group::2.kind::f16, K = 16 per
+// instruction): BK = 64 bf16 (128-byte rows) per stage, four MMAs per stage,
+// the accumulator stays in TMEM for the whole K loop, double-buffered across
+// tiles (2 x 256 columns), and 8 epilogue warps drain a finished tile (bf16,
+// 32x32 pieces through shared memory, TMA stores) while the next one
+// accumulates.
 constexpr int BK16 = 64;
-constexpr int kStages = 4;
-constexpr uint32_t kStageBytes = kATile + BN * BK16 * 2;  // 16 KB + 32 KB
-constexpr size_t kSmemBf16 = 1024 + size_t(kStages) * kStageBytes + sizeof(Bars);
+constexpr int kBf16Stages = 5;
+constexpr uint32_t kBf16StageBytes = BM * BK16 * 2 + (BN / 2) * BK16 * 2;  // A 128x64 + B half 128x64 bf16
+constexpr int kBf16EpiBufs = 2;
+constexpr uint32_t kIdescBF16Pair = idesc_make(1, 1, 2 * BM, BN);         // BF16 x BF16 -> F32, M = 256
+
+struct Bf16Bars {
+  uint64_t full[kBf16Stages], empty[kBf16Stages];
+  uint64_t tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+constexpr size_t smem_bf16() {
+  return 1024 + size_t(kBf16Stages) * kBf16StageBytes + 8 * kBf16EpiBufs * kEpiPiece + sizeof(Bf16Bars);
+}
+static_assert(smem_bf16() <= 232448, "shared memory budget (BF16)");
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs a) {
+                const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  uint8_t* stage_base = smem;
+  uint8_t* epi_base = smem + kBf16Stages * kBf16StageBytes;
+  Bf16Bars* bars = reinterpret_cast<Bf16Bars*>(epi_base + 8 * kBf16EpiBufs * kEpiPiece);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cta_slot = (int)(blockIdx.x >> 1), cta_step = (int)(gridDim.x >> 1);
   int ghint = 0;  // unused by dense tiles
+  const int nkb = a.K / BK16;
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kBf16Stages; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->tfull[i]), 1);
-      mbar_init(smem_u32(&bars->tempty[i]), 8);
+      mbar_init(smem_u32(&bars->tempty[i]), 16);
     }
     bars->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const int nkb = a.K / BK16;
+  const uint32_t full0 = mapa_shared(smem_u32(&bars->full[0]), 0);
+  const uint32_t tempty0 = mapa_shared(smem_u32(&bars->tempty[0]), 0);
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ TMA producer ----
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr, ghint);
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
-          raise_timeout(bars);
-          goto done;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
+        const TileInfo ti = decode_tile<FP8BW_FPROP, false, true>(a, t, nullptr, nullptr, ghint);
+        const int arow = ti.m0 + (int)rank * BM, brow = ti.nt * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(smem_u32(&bars->empty[stage]), phase ^ 1)) {
+            raise_timeout_mx(bars);
+            goto done;
+          }
+          const uint32_t sa = smem_u32(stage_base + stage * kBf16StageBytes);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&bars->full[stage]), 2 * kBf16StageBytes);
+          tma_load_2d_pair(sa, &tmA, full0 + stage * 8, kb * BK16, arow);
+          tma_load_2d_pair(sa + BM * BK16 * 2, &tmB, full0 + stage * 8, kb * BK16, brow);
+          if (++stage == kBf16Stages) { stage = 0; phase ^= 1; }
         }
-        if (lane == 0) {
-          const uint32_t full = smem_u32(&bars->full[stage]);
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-          mbar_arrive_expect_tx(full, kStageBytes);
-          tma_load_2d(sa, &tmA, full, kb * BK16, ti.mt * BM);
-          tma_load_2d(sa + kATile, &tmB, full, kb * BK16, ti.nt * BN);
-        }
-        __syncwarp();
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (bars->abort) break;
       }
-      if (bars->abort) break;
-    }
-  } else if (warp == 1) {
-    int stage = 0;
-    uint32_t phase = 0;
-    int buf = 0;
-    uint32_t bphase = 0;
-    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1)) {
-        raise_timeout(bars);
-        goto done;
-      }
-      tc_fence_after();
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(smem_u32(&bars->full[stage]), phase)) {
-          raise_timeout(bars);
+    } else if (warp == 1 && leader && lane == 0) {
+      // ------------------------------------------------- MMA issuer -----
+      int stage = 0, buf = 0;
+      uint32_t phase = 0, bphase = 0;
+      for (int t = cta_slot; t < a.tiles; t += cta_step) {
+        if (!mbar_wait(smem_u32(&bars->tempty[buf]), bphase ^ 1)) {
+          raise_timeout_mx(bars);
           goto done;
         }
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-          const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + kATile);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(smem_u32(&bars->full[stage]), phase)) {
+            raise_timeout_mx(bars);
+            goto done;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * kBf16StageBytes);
+          const uint64_t da = sdesc_k_sw128(sa), db = sdesc_k_sw128(sa + BM * BK16 * 2);
 #pragma unroll
-          for (int kk = 0; kk < BK16 / 16; ++kk)
-            umma_f16(tmem + buf * BN, da + 2 * kk, db + 2 * kk, kIdescBF16,
-                     (kb > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(smem_u32(&bars->empty[stage]));
-          if (kb == nkb - 1) umma_commit(smem_u32(&bars->tfull[buf]));
+          for (int kk = 0; kk < BK16 / 16; ++kk)  // +32 bytes = +2 in the >>4 address field
+            umma_f16_pair(tmem + buf * BN, da + 2 * kk, db + 2 * kk, kIdescBF16Pair,
+                          (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(smem_u32(&bars->empty[stage]), 0x3);
+          if (++stage == kBf16Stages) { stage = 0; phase ^= 1; }
         }
-        __syncwarp();
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        umma_commit_pair(smem_u32(&bars->tfull[buf]), 0x3);
+        if (++buf == 2) { buf = 0; bphase ^= 1; }
+        if (bars->abort) break;
       }
-      if (++buf == 2) { buf = 0; bphase ^= 1; }
-      if (bars->abort) break;
     }
-  } else if (warp >= 4) {
+  } else {
+    regs_inc<kRegsHigh>();
+    // -------------------------------------------------------- epilogue ---
     const int q = warp & 3, half = (warp - 4) >> 2;
+    uint8_t* epi0 = epi_base + (warp - 4) * kBf16EpiBufs * kEpiPiece;
     int buf = 0;
     uint32_t bphase = 0;
-    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x) {
-      const TileInfo ti = decode_tile<FP8BW_FPROP, false, false>(a, t, nullptr, nullptr, ghint);
+    for (int t = cta_slot; t < a.tiles; t += cta_step) {
+      const TileInfo ti = decode_tile<FP8BW_FPROP, false, true>(a, t, nullptr, nullptr, ghint);
       if (!mbar_wait(smem_u32(&bars->tfull[buf]), bphase)) {
-        raise_timeout(bars);
+        raise_timeout_mx(bars);
         goto done;
       }
       tc_fence_after();
-      const int row = ti.mt * BM + q * 32 + lane;
+      const int row0 = ti.m0 + (int)rank * BM;
       const int col0 = ti.nt * BN + half * 128;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
-      uint4* dst = reinterpret_cast<uint4*>(a.D + (size_t)row * a.ldd + col0);
-      const bool valid = col0 < a.N;
+      const int drow = row0 + q * 32;
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         uint32_t r[32];
         tmem_ld32(taddr + p * 32, r);
         tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-            o.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-            o.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-            o.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-            dst[p * 4 + j] = o;
+        tmem_fence_regs(r);
+        if (p == 3) {
+          // the whole accumulator is in registers: the next tile may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (!leader) mbar_arrive_cluster(tempty0 + buf * 8);
+            else mbar_arrive(smem_u32(&bars->tempty[buf]));
           }
         }
+        uint8_t* epi = epi0 + (p % kBf16EpiBufs) * kEpiPiece;
+        if (lane == 0) bulk_wait_read<kBf16EpiBufs - 1>();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(r[8 * c + 0]), __uint_as_float(r[8 * c + 1]));
+          o.y = pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3]));
+          o.z = pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5]));
+          o.w = pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7]));
+          *reinterpret_cast<uint4*>(epi + lane * 64 + 16 * (c ^ ((lane >> 1) & 3))) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, smem_u32(epi), col0 + p * 32, drow);
+          bulk_commit();
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->tempty[buf]));
       if (++buf == 2) { buf = 0; bphase ^= 1; }
       if (bars->abort) break;
     }
   }
 done:
+  if (warp >= 4 && lane == 0) bulk_wait0();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -1225,11 +1394,11 @@ cudaError_t prepare(K kernel, size_t smem, bool check_regs) {
   return cudaSuccess;
 }
 
-template <int KIND, bool GROUPED, bool PAIR, bool F32OUT = false>
+template <int KIND, bool GROUPED, bool PAIR, int OUTK = OK_BF16>
 cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                        const GemmArgs& a, int grid, cudaStream_t st) {
-  auto kern = k_gemm_fp8<KIND, GROUPED, PAIR, F32OUT>;
-  const size_t smem = smem_fp8<PAIR>();
+  auto kern = k_gemm_fp8<KIND, GROUPED, PAIR, OUTK>;
+  const size_t smem = smem_fp8<PAIR, OUTK == OK_QUANT_FP32 || OUTK == OK_QUANT_POW2>();
   cudaError_t e = prepare(kern, smem, true);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1329,15 +1498,15 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
     if (grouped && kind != FP8BW_WGRAD) return cudaErrorInvalidValue;
     if (grouped) {
       if (mode == FP8BW_SCALE_POW2) e = launch_mx<FP8BW_WGRAD, true, true, true>(ta, tb, td, a, grid, st);
-      else e = launch_one<FP8BW_WGRAD, true, true, true>(ta, tb, td, a, grid, st);
+      else e = launch_one<FP8BW_WGRAD, true, true, OK_F32>(ta, tb, td, a, grid, st);
     } else if (mode == FP8BW_SCALE_POW2) {
       if (kind == FP8BW_FPROP) e = launch_mx<FP8BW_FPROP, false, true, true>(ta, tb, td, a, grid, st);
       else if (kind == FP8BW_DGRAD) e = launch_mx<FP8BW_DGRAD, false, true, true>(ta, tb, td, a, grid, st);
       else e = launch_mx<FP8BW_WGRAD, false, true, true>(ta, tb, td, a, grid, st);
     } else {
-      if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true, true>(ta, tb, td, a, grid, st);
-      else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true, true>(ta, tb, td, a, grid, st);
-      else e = launch_one<FP8BW_WGRAD, false, true, true>(ta, tb, td, a, grid, st);
+      if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true, OK_F32>(ta, tb, td, a, grid, st);
+      else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true, OK_F32>(ta, tb, td, a, grid, st);
+      else e = launch_one<FP8BW_WGRAD, false, true, OK_F32>(ta, tb, td, a, grid, st);
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -1368,32 +1537,92 @@ cudaError_t launch_gemm_fp8(int kind, bool grouped, int G, const int32_t* d_off,
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,
-                             int64_t ldd, int num_sms, cudaStream_t st) {
-  CUtensorMap ta, tb;
-  GemmArgs a;
+// The GEMM with the quantizing epilogue (dense, promotion kernel, any fp32
+// operand scales): D = bf16(A B^T) quantized into q_row/s_row and, if q_col
+// is given, the column-wise copy q_col/s_col with scale rule `qmode`; D
+// itself is written only if non-null.
+cudaError_t launch_gemm_quant(int kind, int64_t M, int64_t N, int64_t K, const uint8_t* A, const float* sA,
+                              const uint8_t* B, const float* sB, int qmode, void* D, int64_t ldd,
+                              uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, int num_sms,
+                              cudaStream_t st) {
+  GemmArgs a = {};
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
-  a.m_tiles = (int)(M / BM);
+  a.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
   a.n_tiles = (int)((N + BN - 1) / BN);
-  a.band = gemm_band_rows;
+  a.band = (gemm_band_rows + 1) / 2;
   a.tiles = a.m_tiles * a.n_tiles;
-  a.sA = a.sB = nullptr;
+  a.sA = sA;
+  a.sB = sB;
   a.D = static_cast<uint16_t*>(D);
   a.ldd = ldd;
-  a.offsets = nullptr;
-  a.G = 0;
+  a.q_row = q_row;
+  a.s_row = s_row;
+  a.q_col = q_col;
+  a.s_col = s_col;
+  a.stall_chunk = gemm_stall_chunk;
+  gemm_stall_chunk = -1;
   if (a.tiles == 0) return cudaSuccess;
+  CUtensorMap ta, tb, td;
+  std::memset(&td, 0, sizeof td);  // no tensor-map store in this epilogue
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, K, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const int clusters = num_sms / 2;
+  const int grid = 2 * (a.tiles < clusters ? a.tiles : clusters);
+  cudaError_t e;
+  if (qmode == FP8BW_SCALE_POW2) {
+    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true, OK_QUANT_POW2>(ta, tb, td, a, grid, st);
+    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true, OK_QUANT_POW2>(ta, tb, td, a, grid, st);
+    else e = launch_one<FP8BW_WGRAD, false, true, OK_QUANT_POW2>(ta, tb, td, a, grid, st);
+  } else {
+    if (kind == FP8BW_FPROP) e = launch_one<FP8BW_FPROP, false, true, OK_QUANT_FP32>(ta, tb, td, a, grid, st);
+    else if (kind == FP8BW_DGRAD) e = launch_one<FP8BW_DGRAD, false, true, OK_QUANT_FP32>(ta, tb, td, a, grid, st);
+    else e = launch_one<FP8BW_WGRAD, false, true, OK_QUANT_FP32>(ta, tb, td, a, grid, st);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* B, void* D,
+                             int64_t ldd, int num_sms, cudaStream_t st) {
+  GemmArgs a = {};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
+  a.n_tiles = (int)((N + BN - 1) / BN);
+  a.band = (gemm_band_rows + 1) / 2;
+  a.tiles = a.m_tiles * a.n_tiles;
+  if (a.tiles == 0) return cudaSuccess;
+  CUtensorMap ta, tb, td;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, K, BK16, BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, K, BK16, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, K, BK16, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const int grid = a.tiles < num_sms ? a.tiles : num_sms;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBf16);
+  if (!make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, M, ldd, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  const int clusters = num_sms / 2;
+  const int grid = 2 * (a.tiles < clusters ? a.tiles : clusters);
+  const size_t smem = smem_bf16();
+  cudaError_t e = prepare(k_gemm_bf16, smem, true);
   if (e != cudaSuccess) return e;
-  k_gemm_bf16<<<grid, kThreads, kSmemBf16, st>>>(ta, tb, a);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_gemm_bf16, ta, tb, td, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

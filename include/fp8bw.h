@@ -217,6 +217,29 @@ FP8BW_API fp8bw_status fp8bw_gemm_f32(fp8bw_gemm_kind kind, int64_t M, int64_t N
                             const float* sB, float* D, int64_t ldd, int32_t accumulate,
                             fp8bw_scale_mode mode, fp8bw_stream_t stream);
 
+/* The GEMM with its output quantized in the epilogue, for an output that is
+ * the next FP8 GEMM's operand ("Der technische Durchbruch": activations and
+ * activation gradients enter the FP8 linear layers as 1x128 blocks;
+ * "Leistungsgewinne in der Praxis": quantization-kernel overhead is part of
+ * the gap between 2x and the measured gain, and fusing the quantizer into
+ * the producer removes the bf16 round trip through HBM).
+ * Computes D = bf16(sum_kb sA sB sum_k A B) exactly as fp8bw_gemm with
+ * FP8BW_SCALE_FP32 (the operand scales may be any fp32 values, powers of two
+ * included), then writes what fp8bw_quant_act_1x128(D, out_mode) writes:
+ *   q_row [M][N] E4M3 codes, s_row [N/128][M]   (1x128 row blocks)
+ *   q_col [N][M] codes, s_col [M/128][N]        (column-wise copy; both
+ *                                                NULL for row-wise only)
+ *   D     [M][ldd] bf16, or NULL to skip it (ldd a multiple of 8 if given).
+ * Bit for bit, the codes and scales equal fp8bw_quant_act_1x128 applied to
+ * this call's D.  Operands, kinds and scale layouts as in fp8bw_gemm.
+ * Requires M, N, K multiples of 128 and K > 0 (else FP8BW_ERR_ALIGNMENT /
+ * FP8BW_ERR_INVALID_ARG), q_row and q_col 32-byte aligned. */
+FP8BW_API fp8bw_status fp8bw_gemm_quant(fp8bw_gemm_kind kind, int64_t M, int64_t N, int64_t K,
+                                        const uint8_t* A, const float* sA, const uint8_t* B,
+                                        const float* sB, fp8bw_scale_mode out_mode, void* D, int64_t ldd,
+                                        uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col,
+                                        fp8bw_stream_t stream);
+
 /* Grouped GEMM for mixture-of-experts layers ("Leistungsgewinne in der
  * Praxis": the recipe also trains the Qwen3-30B MoE model).  Tokens are
  * grouped by expert: expert g owns rows [off[g], off[g+1]) of the permuted

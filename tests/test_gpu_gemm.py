@@ -162,6 +162,27 @@ def test_bf16_gemm(fb, orc, MNK):
     assert bad == 0, worst
 
 
+def test_bf16_gemm_many_tiles(fb, orc):
+    """More 256x256 pair tiles than CTA pairs (each pair runs several tiles,
+    both TMEM accumulators in turn), M and N with a 128-wide remainder:
+    sampled 128x128 tiles, corners included."""
+    M, N, K = 4224, 4224, 1024
+    g = torch.Generator().manual_seed(99)
+    A = torch.randn((M, K), generator=g).to(torch.bfloat16)
+    B = torch.randn((N, K), generator=g).to(torch.bfloat16)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    fb.fp8bw_gemm_bf16(A.to(DEV), B.to(DEV), D)
+    torch.cuda.synchronize()
+    Db, Ab, Bb = bits(D), bits(A), bits(B)
+    rng = np.random.default_rng(5)
+    tiles = [(0, 0), (M - 128, N - 128), (M - 128, 0), (0, N - 128)]
+    tiles += [(128 * int(rng.integers(0, M // 128)), 128 * int(rng.integers(0, N // 128))) for _ in range(6)]
+    for (m0, n0) in tiles:
+        yr, ya = orc.gemm_bf16_ref_tile(Ab, Bb, m0, m0 + 128, n0, n0 + 128)
+        bad, worst = orc.check_tol(np.ascontiguousarray(Db[m0:m0 + 128, n0:n0 + 128]), yr, ya, rel=1e-3)
+        assert bad == 0, (m0, n0, worst)
+
+
 def test_bounded_wait_timeout_is_reported(fb, orc):
     """Failure path: a producer that never fills one K-chunk makes the GEMM's
     bounded waits run out; the call comes back with FP8BW_ERR_TIMEOUT and
