@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int lim = jend - kb * 128 - col0;      // columns >= lim are masked
       const float4* sk4 = reinterpret_cast<const float4*>(&sm.sc[b % kScSlots].sk[col0]);
       // in place: r becomes y = s_k * (q . k), then p (as fp32 bits)
-      float mh = -INFINITY;
+      float mh;
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
 #pragma unroll
@@ -379,8 +379,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 64; ++j)
           if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
       }
+      {
+        // block maximum of the thread's 64 values: a tree of three-input maxima
+        float m1[22], m2[8];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) mh = fmaxf(mh, __uint_as_float(r[j >> 5][j & 31]));
+        for (int t = 0; t < 21; ++t)
+          m1[t] = fmax3(__uint_as_float(r[(3 * t) >> 5][(3 * t) & 31]), __uint_as_float(r[(3 * t + 1) >> 5][(3 * t + 1) & 31]),
+                        __uint_as_float(r[(3 * t + 2) >> 5][(3 * t + 2) & 31]));
+        m1[21] = __uint_as_float(r[1][31]);
+#pragma unroll
+        for (int t = 0; t < 7; ++t) m2[t] = fmax3(m1[3 * t], m1[3 * t + 1], m1[3 * t + 2]);
+        m2[7] = m1[21];
+        mh = fmax3(fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]), fmaxf(m2[6], m2[7]));
+      }
       // block maximum of the row: combine the two halves
       sm.red[b & 1][hf][i] = mh;
       if (!pair_meet(bars, q, lane, meets++)) {
@@ -391,24 +402,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m, mb);
       const float alpha = ex2(m - m_new);       // 0 on the first block
       m = m_new;
-      float ps = 0.0f;
+      // p = 2^(y * cq - m) on packed pairs; four partial pair sums
+      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
+      float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float pj = ex2(__fmaf_rn(__uint_as_float(r[j >> 5][j & 31]), cq, -m_new));
-        r[j >> 5][j & 31] = __float_as_uint(pj);
-        ps += pj;
+      for (int j = 0; j < 64; j += 2) {
+        const int u = j >> 5, k = j & 31;
+        const float2 z = ffma2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), cq2, nm2);
+        const float2 pj = make_float2(ex2(z.x), ex2(z.y));
+        r[u][k] = __float_as_uint(pj.x);
+        r[u][k + 1] = __float_as_uint(pj.y);
+        ps2[(j >> 1) & 3] = fadd2(ps2[(j >> 1) & 3], pj);
       }
-      lh = lh * alpha + ps;
-      // P's block scale: amax / 448 with amax = 2^(mb - m) the block's largest p
+      const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+      lh = lh * alpha + (psum.x + psum.y);
+      // P's block scale: amax / 448 with amax = 2^(mb - m) the block's largest
+      // p; codes of p * 448 / amax (within the kernel's fp32 error of p / s)
       const float amax = ex2(mb - m_new);
-      const float sp = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      const float inv = amax > 0.0f ? __fdiv_rn(1.0f, sp) : 0.0f;
+      const float sp = amax > 0.0f ? amax * (1.0f / 448.0f) : 1.0f;
+      const float inv = amax > 0.0f ? __fdividef(448.0f, amax) : 0.0f;
+      const float2 inv2 = make_float2(inv, inv);
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int u = j >> 3, k = 4 * (j & 7);
-        w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]) * inv, __uint_as_float(r[u][k + 1]) * inv) |
-               (cvt_e4m3x2(__uint_as_float(r[u][k + 2]) * inv, __uint_as_float(r[u][k + 3]) * inv) << 16);
+        const float2 a0 = fmul2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), inv2);
+        const float2 a1 = fmul2(make_float2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])), inv2);
+        w[j] = cvt_e4m3x2(a0.x, a0.y) | (cvt_e4m3x2(a1.x, a1.y) << 16);
       }
       if (!warp_wait(smem_u32(&bars->p_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
         ok = false;

@@ -24,6 +24,15 @@ __device__ __forceinline__ float halves_max(uint32_t m) {
   return __uint_as_float((lo > hi ? lo : hi) << 16);
 }
 
+// Larger-magnitude halves of two packed bf16 words (sign bits arbitrary:
+// mask with kAbsMask before reading the magnitudes).  One instruction per
+// word pair; magnitudes compare exactly as the non-negative bf16 values.
+__device__ __forceinline__ uint32_t magmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t absmax8(uint4 v) {
   return umax2(umax2(v.x & kAbsMask, v.y & kAbsMask), umax2(v.z & kAbsMask, v.w & kAbsMask));
 }

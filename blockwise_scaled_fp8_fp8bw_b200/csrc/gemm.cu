@@ -24,13 +24,15 @@
 //               (2 block scales, or 256 column scales for wgrad) into an
 //               8-slot shared ring with cp.async.
 //   warps 4-11  promotion: each warp owns a 32-row quarter of TMEM lanes and
-//               128 columns, a thread per row (32x32b loads in four groups of
-//               32 columns, the next group's load in flight while the current
-//               one is scaled; wgrad's per-column scales arrive as warp-wide
-//               16-byte shared-memory broadcasts); per chunk it reads the
-//               chunk product from TMEM, multiplies by sA*sB in fp32 and
-//               adds it to its registers (packed f32x2 FMAs), releasing the
-//               TMEM buffer as soon as it is read so the MMA of the next
+//               128 columns (fprop/dgrad: a thread per row, 32x32b loads in
+//               two rounds of 64 columns; wgrad: 4 rows x 32 columns per
+//               thread, 16x256b loads, so the per-column scales need few
+//               shared loads — with the quantizing epilogue a thread per row
+//               and the column scales as warp-wide 16-byte shared
+//               broadcasts); per chunk it reads the chunk product from TMEM,
+//               multiplies by sA*sB in fp32 and adds it to its registers
+//               (packed f32x2 FMAs), releasing the TMEM buffer as soon as
+//               the last round is in registers so the MMA of the next
 //               chunk overlaps.  At the end of a tile the results are
 //               rounded to bf16 (or kept fp32), staged in shared memory
 //               (64-byte swizzle, three pieces per warp) and written by TMA
@@ -87,6 +89,8 @@ struct Cfg {
 
 
 constexpr int kRegsLow = 56, kRegsHigh = 224, kRegsLaunch = 168;
+
+
 static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
 
 struct ScaleSlot {
@@ -342,6 +346,22 @@ __device__ __forceinline__ void stage_rows_f32(uint8_t* epi, int lane, const flo
         make_float4(a[2 * c].x, a[2 * c].y, a[2 * c + 1].x, a[2 * c + 1].y);
 }
 
+// Accumulators of the 16x256b shape (wgrad promotion): acc[16 i + g] holds
+// row 8i + lane/4 and columns 8g + 2(lane%4) + {0, 1}; piece pp covers the
+// column groups g = 2pp, 2pp + 1.
+__device__ __forceinline__ void stage_quad_f32(uint8_t* epi, int lane, const float2* acc, int pp) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 8 * i + (lane >> 2);
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int chunk = 2 * gg + ((lane & 3) >> 1);
+      *reinterpret_cast<float2*>(epi + row * 64 + 16 * (chunk ^ ((row >> 1) & 3)) + 8 * (lane & 1)) =
+          acc[16 * i + 2 * pp + gg];
+    }
+  }
+}
+
 // Writes (or adds) one staged fp32 piece.
 __device__ __forceinline__ void emit_f32(const CUtensorMap* tmD, uint32_t src, int x, int y, int out_mode) {
   if (out_mode == OUT_F32_ADD) tma_reduce_add_2d(tmD, src, x, y);
@@ -367,6 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool QOUT = OUTK == OK_QUANT_FP32 || OUTK == OK_QUANT_POW2;
   static_assert(!(QOUT && GROUPED), "quantizing epilogue: dense GEMMs only");
   using C = Cfg<PAIR, QOUT>;
+  // wgrad promotion layout: the 16x256b shape (4 rows x 32 columns per
+  // thread, PW = 0) in general; the quantizing epilogue needs a thread per
+  // row (32x32b, PW = 2)
+  constexpr int PW = QOUT ? 2 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -596,30 +620,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const ScaleSlot* sl = &slots[ss];
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + half * 128;
-        // The thread owns row q*32 + lane of the CTA's 128 and the 128
-        // columns of its half: four groups of 32 columns (32x32b TMEM
-        // loads).  The next group's load is issued before the current
-        // group's arithmetic, so the TMEM read latency hides behind it, and
-        // the buffer goes back to the MMA warp as soon as its last group has
-        // landed in registers.
-        const float sa = sl->sa[q * 32 + lane];
-        float2 s2 = make_float2(sa, sa);
-        if (KIND != FP8BW_WGRAD) {
-          const float sc = sa * sl->sb[half];   // one scale for the row's 128 columns
-          s2 = make_float2(sc, sc);
-        }
-        // wgrad: a scale per column; all lanes read the same 16 bytes
-        // (a shared-memory broadcast), four column scales per load
-        const float4* sb4 = reinterpret_cast<const float4*>(&sl->sb[half * 128]);
-        uint32_t r[2][32];
-        tmem_ld32(taddr, r[0]);
+        if (KIND == FP8BW_WGRAD && PW == 0) {
+          // 16x256b shape: a thread holds 4 rows x 32 columns, so a chunk
+          // costs 4 row-scale and 16 column-pair loads from shared memory.
+          // acc[16 * i + g] holds row 8i + lane/4 of the quarter and columns
+          // 8g + 2(lane%4) + {0, 1} of the warp's 128.
+          float sa4[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          tmem_wait_ld();
-          tmem_fence_regs(r[g & 1]);
-          if (g < 3) {
-            tmem_ld32(taddr + (g + 1) * 32, r[(g + 1) & 1]);
-          } else {
+          for (int i = 0; i < 4; ++i) sa4[i] = sl->sa[q * 32 + 8 * i + (lane >> 2)];
+          const float* sbw = &sl->sb[half * 128 + 2 * (lane & 3)];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {  // 64-column halves of the warp's 128 columns
+            uint32_t r[2][32];
+            tmem_ld16x64(taddr + h2 * 64, r[0]);                      // quarter lanes 0-15
+            tmem_ld16x64(taddr + (16u << 16) + h2 * 64, r[1]);        // quarter lanes 16-31
+            tmem_wait_ld();
+            tmem_fence_regs(r[0]);
+            tmem_fence_regs(r[1]);
+            if (h2 == 1) {
+              // chunk fully read: hand the TMEM buffer back to the MMA warp
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
+                else mbar_arrive(smem_u32(&bars->tempty[buf]));
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int g = h2 * 8 + j;
+              const float2 b2 = *reinterpret_cast<const float2*>(sbw + 8 * g);
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                  const int i = 2 * u + v;
+                  const float2 sc = fmul2(make_float2(sa4[i], sa4[i]), b2);
+                  acc[16 * i + g] = ffma2(make_float2(__uint_as_float(r[u][4 * j + 2 * v]),
+                                                      __uint_as_float(r[u][4 * j + 2 * v + 1])),
+                                          sc, acc[16 * i + g]);
+                }
+              }
+            }
+          }
+        } else {
+          // The thread owns row q*32 + lane of the CTA's 128 and the 128
+          // columns of its half (32x32b TMEM loads); wgrad's per-column
+          // scales arrive as warp-wide 16-byte shared-memory broadcasts.
+          const float sa = sl->sa[q * 32 + lane];
+          float2 s2 = make_float2(sa, sa);
+          if (KIND != FP8BW_WGRAD) {
+            const float sc = sa * sl->sb[half];   // one scale for the row's 128 columns
+            s2 = make_float2(sc, sc);
+          }
+          const float4* sb4 = reinterpret_cast<const float4*>(&sl->sb[half * 128]);
+          // 32 columns (group g, registers rg) into the accumulators
+          auto promote_group = [&](int g, const uint32_t* rg) {
+            if (KIND == FP8BW_WGRAD) {
+#pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+                const float4 b = sb4[8 * g + j4];
+                const float2 c0 = fmul2(s2, make_float2(b.x, b.y));
+                const float2 c1 = fmul2(s2, make_float2(b.z, b.w));
+                acc[16 * g + 2 * j4] = ffma2(make_float2(__uint_as_float(rg[4 * j4]), __uint_as_float(rg[4 * j4 + 1])),
+                                             c0, acc[16 * g + 2 * j4]);
+                acc[16 * g + 2 * j4 + 1] = ffma2(make_float2(__uint_as_float(rg[4 * j4 + 2]), __uint_as_float(rg[4 * j4 + 3])),
+                                                 c1, acc[16 * g + 2 * j4 + 1]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                acc[16 * g + j] = ffma2(make_float2(__uint_as_float(rg[2 * j]), __uint_as_float(rg[2 * j + 1])),
+                                        s2, acc[16 * g + j]);
+            }
+          };
+          auto release = [&]() {
             // chunk fully read: hand the TMEM buffer back to the MMA warp
             tc_fence_before();
             __syncwarp();
@@ -627,24 +702,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (PAIR && !leader) mbar_arrive_cluster(tempty0 + buf * 8);
               else mbar_arrive(smem_u32(&bars->tempty[buf]));
             }
-          }
-          const uint32_t* rg = r[g & 1];
-          if (KIND == FP8BW_WGRAD) {
+          };
+          {
+            // two rounds of 64 columns: release after the second round lands
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 b = sb4[8 * g + j4];
-              const float2 c0 = fmul2(s2, make_float2(b.x, b.y));
-              const float2 c1 = fmul2(s2, make_float2(b.z, b.w));
-              acc[16 * g + 2 * j4] = ffma2(make_float2(__uint_as_float(rg[4 * j4]), __uint_as_float(rg[4 * j4 + 1])),
-                                           c0, acc[16 * g + 2 * j4]);
-              acc[16 * g + 2 * j4 + 1] = ffma2(make_float2(__uint_as_float(rg[4 * j4 + 2]), __uint_as_float(rg[4 * j4 + 3])),
-                                               c1, acc[16 * g + 2 * j4 + 1]);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint32_t r[2][32];
+              tmem_ld64(taddr + h2 * 64, r[0], r[1]);
+              tmem_wait_ld();
+              tmem_fence_regs(r[0]);
+              tmem_fence_regs(r[1]);
+              if (h2 == 1) release();
+              promote_group(2 * h2, r[0]);
+              promote_group(2 * h2 + 1, r[1]);
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[16 * g + j] = ffma2(make_float2(__uint_as_float(rg[2 * j]), __uint_as_float(rg[2 * j + 1])),
-                                      s2, acc[16 * g + j]);
           }
         }
         __syncwarp();
@@ -679,7 +750,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_wait_read<C::kEpiBufs - 1>();
           }
           __syncwarp();
-          stage_rows_f32(epi, lane, &acc[8 * pp]);
+          if (KIND == FP8BW_WGRAD && PW == 0) stage_quad_f32(epi, lane, acc, pp);
+          else stage_rows_f32(epi, lane, &acc[8 * pp]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -696,7 +768,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_wait_read<C::kEpiBufs - 1>();
         }
         __syncwarp();
-        {
+        if (KIND == FP8BW_WGRAD && PW == 0) {
+          // rows 8i + lane/4, columns 8c + 2(lane%4) + {0, 1} of the piece:
+          // one bf16 pair per store; the 64-byte swizzle keeps the 32 lanes
+          // of each store on 32 distinct banks
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = 8 * i + (lane >> 2);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 v2 = acc[16 * i + 4 * p + c];
+              *reinterpret_cast<uint32_t*>(epi + row * 64 + 16 * (c ^ ((row >> 1) & 3)) + 4 * (lane & 3)) =
+                  pack_bf16x2(v2.x, v2.y);
+            }
+          }
+        } else {
           // row `lane` of the piece: 64 bytes = 4 chunks, 64-byte swizzle
 #pragma unroll
           for (int c = 0; c < 4; ++c) {

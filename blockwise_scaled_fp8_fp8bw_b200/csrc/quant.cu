@@ -124,9 +124,13 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
       uint4 v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(tb + act_off(hh, rr, j));
-      uint32_t m = absmax8(v[0]);
+      uint32_t m0w = magmax2(v[0].x, v[0].y), m1w = magmax2(v[0].z, v[0].w);
 #pragma unroll
-      for (int j = 1; j < 8; ++j) m = umax2(m, absmax8(v[j]));
+      for (int j = 1; j < 8; ++j) {
+        m0w = magmax2(m0w, magmax2(v[j].x, v[j].y));
+        m1w = magmax2(m1w, magmax2(v[j].z, v[j].w));
+      }
+      uint32_t m = magmax2(m0w, m1w) & kAbsMask;
       m = umax2(m, __shfl_xor_sync(0xffffffffu, m, 8));
       const Divisor d = make_divisor<MODE, FMT>(halves_max(m));
       if (hh == 0) s_row[(k0 / 128) * M + m0 + rr] = d.s;
@@ -142,13 +146,13 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
     // ---- column pass, part 1: the words and the partial maxima
     ColWords cw;
     if (COL) {
-      uint32_t m = 0;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
+      for (int r = 0; r < 32; ++r)
         cw.w[r] = *reinterpret_cast<const uint32_t*>(tb + act_off(cbox, rg * 32 + r, cchunk) + 4 * cword);
-        m = umax2(m, cw.w[r] & kAbsMask);
-      }
-      sm.colmax[cur][rg][wc] = m;
+      uint32_t mw[4] = {cw.w[0], cw.w[1], cw.w[2], cw.w[3]};
+#pragma unroll
+      for (int r = 4; r < 32; ++r) mw[r & 3] = magmax2(mw[r & 3], cw.w[r]);
+      sm.colmax[cur][rg][wc] = magmax2(magmax2(mw[0], mw[1]), magmax2(mw[2], mw[3])) & kAbsMask;
     }
     // Partial maxima complete; every thread is done reading this buffer, so
     // it may take the tile after next.
