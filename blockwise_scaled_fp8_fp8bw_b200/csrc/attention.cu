@@ -399,6 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const float mb = fmaxf(sm.red[b & 1][0][i], sm.red[b & 1][1][i]) * cq;
+      // The two warps of a quarter share one scheduler and meet here every
+      // block; the second folds the previous block's product first and the
+      // first exponentiates first, so one warp's exponentials overlap the
+      // other's fold instead of both waiting on the same unit.
+      if (hf == 1 && b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) {
+        ok = false;
+        break;
+      }
       const float m_new = fmaxf(m, mb);
       const float alpha = ex2(m - m_new);       // 0 on the first block
       m = m_new;
@@ -443,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[b & 1]));
-      if (b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) ok = false;
+      if (hf == 0 && b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) ok = false;
       a_prev = alpha;
       sp_prev = sp;
       if (bars->abort) ok = false;
