@@ -51,6 +51,7 @@ constexpr int kScSlots = 4;          // scale ring
 constexpr uint32_t kTile = 128 * 128;  // one 128x128 E4M3 tile
 constexpr uint32_t kIdesc = idesc_make(0, 0, 128, 128);  // E4M3 x E4M3 -> F32, M = N = 128
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
 // setmaxnreg split: 56 registers for warps 0-3, 224 for the softmax warps;
 // 56*128 + 224*256 = 64512 <= 384 * 168, the launch allocation (checked
 // on the host before the launch).
@@ -136,10 +137,13 @@ __device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_
       const float4 v = sv4[u * 8 + j4];
       const float2 c0 = fmul2(sp2, make_float2(v.x, v.y));
       const float2 c1 = fmul2(sp2, make_float2(v.z, v.w));
-      float2 o0 = c > 0 ? fmul2(make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1])), a2)
-                        : make_float2(0.f, 0.f);
-      float2 o1 = c > 0 ? fmul2(make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3])), a2)
-                        : make_float2(0.f, 0.f);
+      float2 o0 = make_float2(0.f, 0.f), o1 = make_float2(0.f, 0.f);
+      if (c > 0) {
+        o0 = make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1]));
+        o1 = make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3]));
+        o0 = fmul2(o0, a2);
+        o1 = fmul2(o1, a2);
+      }
       o0 = ffma2(make_float2(__uint_as_float(r[4 * j4]), __uint_as_float(r[4 * j4 + 1])), c0, o0);
       o1 = ffma2(make_float2(__uint_as_float(r[4 * j4 + 2]), __uint_as_float(r[4 * j4 + 3])), c1, o1);
       o[4 * j4] = __float_as_uint(o0.x);
@@ -403,15 +407,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // block; the second folds the previous block's product first and the
       // first exponentiates first, so one warp's exponentials overlap the
       // other's fold instead of both waiting on the same unit.
-      if (hf == 1 && b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) {
+      if (hf == 1 && b >= 1 &&
+          !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) {
         ok = false;
         break;
       }
       const float m_new = fmaxf(m, mb);
       const float alpha = ex2(m - m_new);       // 0 on the first block
       m = m_new;
-      // p = 2^(y * cq - m) on packed pairs; four partial pair sums
-      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
+      // P's block scale s_P = amax / 448, amax = 2^(mb - m) the block's
+      // largest p.  The code input p / s_P = 2^(y * cq - mb + log2 448) is
+      // exponentiated directly (it does not depend on m), and the row sum
+      // gains s_P * sum(p / s_P).  If amax underflows, s_P = 0 and the block
+      // adds nothing, as its p do.
+      const float amax = ex2(mb - m_new);
+      const float sp = amax * (1.0f / 448.0f);
+      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(kLog2_448 - mb, kLog2_448 - mb);
       float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
@@ -423,20 +434,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ps2[(j >> 1) & 3] = fadd2(ps2[(j >> 1) & 3], pj);
       }
       const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
-      lh = lh * alpha + (psum.x + psum.y);
-      // P's block scale: amax / 448 with amax = 2^(mb - m) the block's largest
-      // p; codes of p * 448 / amax (within the kernel's fp32 error of p / s)
-      const float amax = ex2(mb - m_new);
-      const float sp = amax > 0.0f ? amax * (1.0f / 448.0f) : 1.0f;
-      const float inv = amax > 0.0f ? __fdividef(448.0f, amax) : 0.0f;
-      const float2 inv2 = make_float2(inv, inv);
+      lh = lh * alpha + sp * (psum.x + psum.y);
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int u = j >> 3, k = 4 * (j & 7);
-        const float2 a0 = fmul2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), inv2);
-        const float2 a1 = fmul2(make_float2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])), inv2);
-        w[j] = cvt_e4m3x2(a0.x, a0.y) | (cvt_e4m3x2(a1.x, a1.y) << 16);
+        w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])) |
+               (cvt_e4m3x2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])) << 16);
       }
       if (!warp_wait(smem_u32(&bars->p_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
         ok = false;
@@ -451,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[b & 1]));
-      if (hf == 0 && b >= 1 && !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) ok = false;
+      if (hf == 0 && b >= 1 &&
+          !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev))
+        ok = false;
       a_prev = alpha;
       sp_prev = sp;
       if (bars->abort) ok = false;
