@@ -13,7 +13,7 @@
 //
 // One CTA computes a 128-query block of one head over its keys (causal or
 // not, inside one packed sequence; GQA: query head h reads KV head
-// h / (Hq / Hkv)).  384 threads:
+// h / (Hq / Hkv)).  128 + 32 * kSoftWarps threads:
 //   warp 0      TMA producer: the Q tile once, then per 128-key block the K
 //               tile [128 keys][128] and the V tile [128 channels][128 keys]
 //               into a 3-stage ring, and the block's 128 key scales and 128
@@ -22,14 +22,14 @@
 //               buffers, then O_(b-1) = P_(b-1) V_(b-1)^T into one of two
 //               more, so the tensor core computes the next S while the
 //               softmax warps work on the current one
-//   warps 4-11  softmax and correction, two warps per TMEM lane quarter
-//               (64 of the 128 columns each; a thread owns one query row):
-//               read S_b, scale by the key and query scales, block maximum
-//               (exchanged between the two halves of the row), running
-//               maximum, p = 2^(z - m), partial row sums, P codes into a
-//               shared tile in the MMA's layout; then fold O_(b-1) into the
-//               fp32 output accumulator, kept in TMEM: O = O * 2^(m_old -
-//               m_new) + s_P * s_V[channel] * O_(b-1).
+//   warps 4..   softmax and correction, kNH warps per TMEM lane quarter
+//               (kCols of the 128 columns each; a thread owns one query
+//               row): read S_b, scale by the key and query scales, block
+//               maximum (exchanged between the kNH parts of the row),
+//               running maximum, p = 2^(z - m), partial row sums, P codes
+//               into a shared tile in the MMA's layout; then fold O_(b-1)
+//               into the fp32 output accumulator, kept in TMEM:
+//               O = O * 2^(m_old - m_new) + s_P * s_V[channel] * O_(b-1).
 // At the end O / l is rounded to bf16 and stored; padding query rows get 0.
 // TMEM: S buffers at columns 0 and 128, the P.V product at 256, the output
 // accumulator at 384.  Every wait is bounded; a timeout latches an error bit
@@ -45,18 +45,34 @@ __device__ uint32_t g_attn_error;
 namespace {
 
 constexpr int kD = 128;              // head dimension (one 1x128 block)
-constexpr int kThreads = 384;
+#ifndef FP8BW_ATTN_WARPS_PER_QUARTER
+#define FP8BW_ATTN_WARPS_PER_QUARTER 2
+#endif
+// Softmax warps per TMEM lane quarter: each owns kCols of a row's 128
+// columns.  All warps of a quarter run on one scheduler (TMEM lane quarter =
+// warp index mod 4).  Four per quarter (640 threads, 112 registers) is
+// correct but slower on B200 (570 against 617 TFLOP/s on the packed 32K
+// batch): every block's maximum then waits for the slowest of four warps.
+constexpr int kNH = FP8BW_ATTN_WARPS_PER_QUARTER;
+static_assert(kNH == 2 || kNH == 4, "2 or 4 softmax warps per lane quarter");
+constexpr int kCols = 128 / kNH;                 // columns per softmax thread
+constexpr int kSoftWarps = 4 * kNH;
+constexpr int kThreads = 128 + 32 * kSoftWarps;  // warps 0-3 + the softmax warps
 constexpr int kStages = 3;           // K/V ring
 constexpr int kScSlots = 4;          // scale ring
 constexpr uint32_t kTile = 128 * 128;  // one 128x128 E4M3 tile
 constexpr uint32_t kIdesc = idesc_make(0, 0, 128, 128);  // E4M3 x E4M3 -> F32, M = N = 128
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
-// setmaxnreg split: 56 registers for warps 0-3, 224 for the softmax warps;
-// 56*128 + 224*256 = 64512 <= 384 * 168, the launch allocation (checked
-// on the host before the launch).
-constexpr int kRegsLow = 56, kRegsHigh = 224, kRegsLaunch = 168;
-static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kRegsLaunch * kThreads, "register split");
+// setmaxnreg split of the launch allocation (kThreads x kRegsLaunch, checked
+// on the host before the launch): kRegsLow for warps 0-3, kRegsHigh for the
+// softmax warps.  2 per quarter: 56*128 + 224*256 = 64512 <= 384*168;
+// 4 per quarter: 32*128 + 112*512 = 61440 <= 640*96.
+constexpr int kRegsLow = kNH == 2 ? 56 : 32;
+constexpr int kRegsHigh = kNH == 2 ? 224 : 112;
+constexpr int kRegsLaunch = kNH == 2 ? 168 : 96;
+static_assert(kRegsLow * 128 + kRegsHigh * 32 * kSoftWarps <= kRegsLaunch * kThreads, "register split");
+static_assert(kRegsLaunch * kThreads <= 65536, "launch allocation");
 
 struct ScSlot {
   float sk[128];   // key scales of the block (one per key)
@@ -70,7 +86,7 @@ struct AttnBars {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t o_full, o_empty;  // the single P.V product buffer
-  uint64_t pair[4];          // the two warps of a TMEM lane quarter meet here
+  uint64_t pair[4];          // the kNH warps of a TMEM lane quarter meet here
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -80,8 +96,8 @@ struct AttnSmem {
   uint8_t kv[kStages][2][kTile];       // [stage][K, V^T]
   uint8_t p[2][kTile];
   ScSlot sc[kScSlots];
-  float red[2][2][128];                // [block parity][half][row]: block maxima
-  float lsum[2][128];                  // [half][row]: row sums at the end
+  float red[2][kNH][128];              // [block parity][column part][row]: block maxima
+  float lsum[kNH][128];                // [column part][row]: row sums at the end
   AttnBars bars;
 };
 
@@ -106,8 +122,35 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns (thread i: row lane base + i).
+__device__ __forceinline__ void tmem_ld16c(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16c(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// tmem_fence_regs for 16 registers.
+__device__ __forceinline__ void fence_regs16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+
 // Folds O_c (block c's P.V product in TMEM) into the output accumulator
-// (TMEM columns 384..511, this thread's row and 64 columns):
+// (TMEM columns 384..511, this thread's row and kCols columns):
 // acc = acc * alpha + s_P * s_V[channel] * O_c (acc = 0 before block 0),
 // then hands the product buffer and the block's scale slot back.  False if
 // a wait ran out.
@@ -118,31 +161,30 @@ __device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_
   const uint32_t tp = tmem + lane_off + 256 + col0, to = tmem + lane_off + 384 + col0;
   const float2 sp2 = make_float2(sp, sp), a2 = make_float2(alpha, alpha);
   const float4* sv4 = reinterpret_cast<const float4*>(&sm.sc[c % kScSlots].sv[col0]);
+  // rounds of 16 columns
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    uint32_t r[32], o[32];
-    tmem_ld32(tp + 32 * u, r);
-    if (c > 0) tmem_ld32(to + 32 * u, o);
+  for (int u = 0; u < kCols / 16; ++u) {
+    uint32_t r[16], o[16];
+    tmem_ld16c(tp + 16 * u, r);
+    if (c > 0) tmem_ld16c(to + 16 * u, o);
     tmem_wait_ld();
-    tmem_fence_regs(r);
-    if (c > 0) tmem_fence_regs(o);
-    if (u == 1) {
+    fence_regs16(r);
+    if (c > 0) fence_regs16(o);
+    if (u == kCols / 16 - 1) {
       // the product is in registers: the next P.V may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->o_empty));
     }
 #pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-      const float4 v = sv4[u * 8 + j4];
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 v = sv4[u * 4 + j4];
       const float2 c0 = fmul2(sp2, make_float2(v.x, v.y));
       const float2 c1 = fmul2(sp2, make_float2(v.z, v.w));
       float2 o0 = make_float2(0.f, 0.f), o1 = make_float2(0.f, 0.f);
       if (c > 0) {
-        o0 = make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1]));
-        o1 = make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3]));
-        o0 = fmul2(o0, a2);
-        o1 = fmul2(o1, a2);
+        o0 = fmul2(make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1])), a2);
+        o1 = fmul2(make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3])), a2);
       }
       o0 = ffma2(make_float2(__uint_as_float(r[4 * j4]), __uint_as_float(r[4 * j4 + 1])), c0, o0);
       o1 = ffma2(make_float2(__uint_as_float(r[4 * j4 + 2]), __uint_as_float(r[4 * j4 + 3])), c1, o1);
@@ -151,7 +193,7 @@ __device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_
       o[4 * j4 + 2] = __float_as_uint(o1.x);
       o[4 * j4 + 3] = __float_as_uint(o1.y);
     }
-    tmem_st32(to + 32 * u, o);
+    tmem_st16c(to + 16 * u, o);
   }
   tmem_wait_st();
   __syncwarp();
@@ -159,9 +201,9 @@ __device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_
   return true;
 }
 
-// The two warps of lane quarter q meet (each after writing its half's value
+// The kNH warps of lane quarter q meet (each after writing its part's value
 // to shared memory); `uses` counts this quarter's earlier meetings.  False if
-// the other warp did not arrive in time.
+// another warp did not arrive in time.
 __device__ __forceinline__ bool pair_meet(AttnBars* bars, int q, int lane, uint32_t uses) {
   __syncwarp();
   if (lane == 0) mbar_arrive(smem_u32(&bars->pair[q]));
@@ -227,17 +269,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kScSlots; ++i) {
       mbar_init(smem_u32(&bars->sc_full[i]), 1);
-      mbar_init(smem_u32(&bars->sc_empty[i]), 8);
+      mbar_init(smem_u32(&bars->sc_empty[i]), kSoftWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->s_empty[i]), 8);
-      mbar_init(smem_u32(&bars->p_full[i]), 8);
+      mbar_init(smem_u32(&bars->s_empty[i]), kSoftWarps);
+      mbar_init(smem_u32(&bars->p_full[i]), kSoftWarps);
       mbar_init(smem_u32(&bars->p_empty[i]), 1);
     }
     mbar_init(smem_u32(&bars->o_full), 1);
-    mbar_init(smem_u32(&bars->o_empty), 8);
-    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), 2);
+    mbar_init(smem_u32(&bars->o_empty), kSoftWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), kNH);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -326,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<kRegsHigh>();
     // --------------------------------------------- softmax and correction --
-    const int q = warp & 3, hf = (warp - 4) >> 2;
+    const int q = warp & 3, hf = (warp - 4) >> 2;   // lane quarter, column part
     const int i = q * 32 + lane, t = q0 + i;
-    const int col0 = hf * 64;                       // this thread's 64 columns
+    const int col0 = hf * kCols;                    // this thread's kCols columns
     const float cq = a.sq[(size_t)h * a.T + t] * (kLog2e * 0.08838834764831845f);  // sq * log2(e) / sqrt(128)
     // keys of this row: [j0, jend); a block needs a mask where it reaches jend
     const int jend = a.causal ? min(jreal, t + 1) : jreal;
@@ -337,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;
     uint32_t meets = 0;
+    constexpr int kU = kCols / 32;                  // 32-column TMEM loads per thread
 
     for (int b = 0; b < nb && ok; ++b) {
       const int kb = kb_first + b;
@@ -346,13 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t r[2][32];
+      uint32_t r[kU][32];
       const uint32_t ta = tmem + lane_off + (b & 1) * 128 + col0;
-      tmem_ld32(ta, r[0]);
-      tmem_ld32(ta + 32, r[1]);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) tmem_ld32(ta + 32 * u, r[u]);
       tmem_wait_ld();
-      tmem_fence_regs(r[0]);
-      tmem_fence_regs(r[1]);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) tmem_fence_regs(r[u]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b & 1]));
@@ -364,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // in place: r becomes y = s_k * (q . k), then p (as fp32 bits)
       float mh;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kU; ++u) {
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const float4 kv4 = sk4[u * 8 + j4];
@@ -378,36 +421,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           r[u][4 * j4 + 3] = __float_as_uint(p1.y);
         }
       }
-      if (lim < 64) {
+      if (lim < kCols) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
+        for (int j = 0; j < kCols; ++j)
           if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
       }
       {
-        // block maximum of the thread's 64 values: a tree of three-input maxima
-        float m1[22], m2[8];
+        // block maximum of the thread's kCols values: three-input maxima over
+        // groups of 8, then over the groups
+        float mg[kCols / 8];
 #pragma unroll
-        for (int t = 0; t < 21; ++t)
-          m1[t] = fmax3(__uint_as_float(r[(3 * t) >> 5][(3 * t) & 31]), __uint_as_float(r[(3 * t + 1) >> 5][(3 * t + 1) & 31]),
-                        __uint_as_float(r[(3 * t + 2) >> 5][(3 * t + 2) & 31]));
-        m1[21] = __uint_as_float(r[1][31]);
+        for (int g = 0; g < kCols / 8; ++g) {
+          const uint32_t* v = &r[(8 * g) >> 5][(8 * g) & 31];
+          mg[g] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                        fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                        fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+        }
+        mh = mg[0];
 #pragma unroll
-        for (int t = 0; t < 7; ++t) m2[t] = fmax3(m1[3 * t], m1[3 * t + 1], m1[3 * t + 2]);
-        m2[7] = m1[21];
-        mh = fmax3(fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]), fmaxf(m2[6], m2[7]));
+        for (int g = 1; g + 1 < kCols / 8; g += 2) mh = fmax3(mh, mg[g], mg[g + 1]);
+        if ((kCols / 8) % 2 == 0) mh = fmaxf(mh, mg[kCols / 8 - 1]);
       }
-      // block maximum of the row: combine the two halves
+      // block maximum of the row: combine the kNH parts
       sm.red[b & 1][hf][i] = mh;
       if (!pair_meet(bars, q, lane, meets++)) {
         ok = false;
         break;
       }
-      const float mb = fmaxf(sm.red[b & 1][0][i], sm.red[b & 1][1][i]) * cq;
-      // The two warps of a quarter share one scheduler and meet here every
-      // block; the second folds the previous block's product first and the
-      // first exponentiates first, so one warp's exponentials overlap the
-      // other's fold instead of both waiting on the same unit.
-      if (hf == 1 && b >= 1 &&
+      float mrow = sm.red[b & 1][0][i];
+#pragma unroll
+      for (int k = 1; k < kNH; ++k) mrow = fmaxf(mrow, sm.red[b & 1][k][i]);
+      const float mb = mrow * cq;
+      // The warps of a quarter share one scheduler and meet here every
+      // block; the odd parts fold the previous block's product first and the
+      // even parts exponentiate first, so exponentials overlap folds instead
+      // of all of them waiting on the same unit.
+      const bool fold_first = (hf & 1) != 0;
+      if (fold_first && b >= 1 &&
           !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev)) {
         ok = false;
         break;
@@ -425,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(kLog2_448 - mb, kLog2_448 - mb);
       float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
+      for (int j = 0; j < kCols; j += 2) {
         const int u = j >> 5, k = j & 31;
         const float2 z = ffma2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), cq2, nm2);
         const float2 pj = make_float2(ex2(z.x), ex2(z.y));
@@ -435,9 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
       lh = lh * alpha + sp * (psum.x + psum.y);
-      uint32_t w[16];
+      uint32_t w[kCols / 4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < kCols / 4; ++j) {
         const int u = j >> 3, k = 4 * (j & 7);
         w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])) |
                (cvt_e4m3x2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])) << 16);
@@ -449,13 +499,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // row i of the P tile: 16-byte chunk c at c ^ (i & 7) (128-byte swizzle)
       uint8_t* prow = sm.p[b & 1] + i * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(prow + (((hf * 4 + c) ^ (i & 7)) << 4)) =
+      for (int c = 0; c < kCols / 16; ++c)
+        *reinterpret_cast<uint4*>(prow + (((hf * (kCols / 16) + c) ^ (i & 7)) << 4)) =
             make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[b & 1]));
-      if (hf == 0 && b >= 1 &&
+      if (!fold_first && b >= 1 &&
           !fold_block(sm, bars, tmem, lane_off, col0, lane, b - 1, a_prev, sp_prev))
         ok = false;
       a_prev = alpha;
@@ -464,15 +514,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && !fold_block(sm, bars, tmem, lane_off, col0, lane, nb - 1, a_prev, sp_prev)) ok = false;
     if (!ok) raise_attn_timeout(bars);
-    // row sum of both halves, then O / l in bf16 (padding rows: 0)
+    // row sum of the kNH parts, then O / l in bf16 (padding rows: 0)
     sm.lsum[hf][i] = lh;
     if (!pair_meet(bars, q, lane, meets++)) ok = false;
-    const float l = sm.lsum[0][i] + sm.lsum[1][i];
+    float l = sm.lsum[0][i];
+#pragma unroll
+    for (int k = 1; k < kNH; ++k) l += sm.lsum[k][i];
     const bool real = t < jreal && ok;
     const float il = real ? __fdiv_rn(1.0f, l) : 0.0f;
     uint16_t* orow = orow_base + (size_t)t * ostride + col0;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kU; ++u) {
       uint32_t o[32];
       tmem_ld32(tmem + lane_off + 384 + col0 + 32 * u, o);
       tmem_wait_ld();
