@@ -88,7 +88,7 @@ def lib():
         L.orc_check_tol.argtypes = [vp, vp, vp, i64, dbl, vp]
         L.orc_check_tol.restype = i64
         L.orc_attention_fwd_rows.argtypes = [i64, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp,
-                                             vp, vp, i64, vp, vp, vp, vp, vp]
+                                             vp, vp, i64, vp, vp, vp, vp, vp, i32]
         L.orc_set_threads.argtypes = [i32]
         L.orc_max_threads.restype = i32
         _lib = L
@@ -320,12 +320,14 @@ def check_tol_f32(y, yref, yabs, rel=REL_TOL):
 HEAD_DIM = 128
 
 
-def attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, seg_off, seg_len, causal, rows_t, rows_h):
+def attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, seg_off, seg_len, causal, rows_t, rows_h, mode=0):
     """FP8 attention forward reference ("NVIDIA NeMo RL erreicht 48% ...",
     "Leistungsgewinne in der Praxis": FP8 KV cache and attention) for the
     (token, head) rows given.  q [T, Hq*128] codes, sq [Hq, T]; k [T, Hkv*128],
     sk [Hkv, T]; vT [Hkv*128, T] codes of V's column-wise copy, sv
     [T/128, Hkv*128]; seg_off [nseg+1] (multiples of 128), seg_len [nseg].
+    mode 0: P's block scale by the FP32 rule; mode 1: power-of-2 scales (P
+    taken against an integer power-of-two reference maximum).
     Returns (O [n,128], oabs [n,128], oflip [n,128]) in fp64."""
     q, k, vT = _u8(q), _u8(k), _u8(vT)
     sq, sk, sv = _f32(sq), _f32(sk), _f32(sv)
@@ -340,7 +342,7 @@ def attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, seg_off, seg_len, causal, 
     of = np.empty_like(out)
     lib().orc_attention_fwd_rows(T, int(Hq), int(Hkv), ln.size, _p(off), _p(ln), int(bool(causal)),
                                  _p(q), _p(sq), _p(k), _p(sk), _p(vT), _p(sv), n, _p(rt), _p(rh),
-                                 _p(out), _p(oa), _p(of))
+                                 _p(out), _p(oa), _p(of), int(mode))
     return out, oa, of
 
 

@@ -567,6 +567,26 @@ int64_t orc_check_tol(const uint16_t* y, const double* yref,
 //    because p / amax is what a streaming kernel can reproduce (it meets the
 //    keys relative to a running maximum, which scales a block by a constant);
 //  * O_d = sum_j p^_j v^_{j,d} / l, p^_j = decode(code_j) * s_b.
+// One E4M3 step if the code of tq (tq >= 0) is ambiguous, i.e. tq lies
+// within relative distance eta of the rounding midpoint next to its code;
+// else 0.
+static double midpoint_step(const double* dec, double tq, uint8_t code, double eta) {
+  if (!(tq < 448.0)) return 0.0;
+  const double v = dec[code];
+  const double lo_g = v <= tq ? v : (code > 0 ? dec[code - 1] : 0.0);
+  const double hi_g = v <= tq ? (code < 0x7E ? dec[code + 1] : v) : v;
+  const double mid = 0.5 * (lo_g + hi_g);
+  return (hi_g > lo_g && std::fabs(tq - mid) <= eta * tq) ? hi_g - lo_g : 0.0;
+}
+
+// The power-of-2 scale rule on an fp64 amax > 0 (as block_scale: the
+// smallest e with amax <= qmax 2^e, found by search, clamped to [-127, 127]).
+static int pow2_exponent(double amax, double qmax) {
+  int e = -127;
+  while (e < 127 && amax > std::ldexp(qmax, e)) ++e;
+  return e;
+}
+
 // Sequences: segment g covers tokens [off[g], off[g+1]) (multiples of 128),
 // of which the first len[g] are real tokens; a query token's keys are the
 // real tokens of its segment, and with `causal` only those j <= t.  Query
@@ -582,12 +602,22 @@ int64_t orc_check_tol(const uint16_t* y, const double* yref,
 // logits (2^-21 relative), the exponential (2^-21) and the running maximum
 // (the largest logit error of the row).  Either rounding is then correct.
 // Padding query rows (t beyond its segment's real tokens) give O = 0.
+//
+// mode = MODE_FP32: P's block scale is s_b = amax / 448 (the FP32 rule), and
+// p_j = e^(z_j - zmax) (the reference maximum cancels out of the codes).
+// mode = MODE_POW2 (the recipe's optional power-of-2 scales): s_b is the
+// power-of-2 rule on the block's amax, and p_j = 2^(z_j log2 e - M) with
+// the integer reference M = ceil(zmax log2 e).  Any integer reference gives
+// the same codes, so a kernel may use its running maximum rounded up to an
+// integer.  Where the kernel's fp32 amax can fall on the other side of a
+// power-of-two boundary, the code under the other scale is also correct;
+// oflip then carries the larger of the two outcomes' differences.
 void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
                             const int32_t* off, const int32_t* len, int32_t causal,
                             const uint8_t* q, const float* sq, const uint8_t* k,
                             const float* sk, const uint8_t* vT, const float* sv,
                             int64_t nrows, const int64_t* row_t, const int32_t* row_h,
-                            double* out, double* oabs, double* oflip) {
+                            double* out, double* oabs, double* oflip, int32_t mode) {
   const int64_t D = 128;
   const double* dec = decode_table(FMT_E4M3);
   const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(D));
@@ -625,9 +655,15 @@ void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
       if (z[j - j0] > zmax) zmax = z[j - j0];
       if (dz[j - j0] > dzmax) dzmax = dz[j - j0];
     }
+    // p_j = e^(z_j - zmax) (FP32 mode); in POW2 mode p_j = 2^(z_j log2 e - M)
+    // with the integer reference M = ceil(zmax log2 e): scaling every p by a
+    // power of two scales its power-of-2 block scale by the same power, so
+    // any integer reference gives the same codes.
+    const double kLog2e = 1.0 / std::log(2.0);
+    const double ref = mode == MODE_POW2 ? std::ceil(zmax * kLog2e) : 0.0;
     double l = 0.0;
     for (int64_t j = 0; j < nk; ++j) {
-      z[j] = std::exp(z[j] - zmax);                  // z now holds p
+      z[j] = mode == MODE_POW2 ? std::exp2(z[j] * kLog2e - ref) : std::exp(z[j] - zmax);   // z now holds p
       l += z[j];
     }
     // P . V block by block (128-key blocks at absolute multiples of 128)
@@ -636,27 +672,40 @@ void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
       double amax = 0.0, dzb = 0.0;
       for (int64_t j = lo; j < hi; ++j)
         if (z[j - j0] > amax) { amax = z[j - j0]; dzb = dz[j - j0]; }
-      const double sb = amax > 0.0 ? amax / 448.0 : 1.0;   // an all-zero block has s = 1
+      // the block scale by the mode's rule (an all-zero block has s = 1);
+      // in POW2 mode a kernel's fp32 amax may land on the other side of a
+      // power-of-two boundary (relative error eta_s), giving the other scale
+      double sb = 1.0, sb_alt = 0.0;
+      if (amax > 0.0) {
+        if (mode == MODE_POW2) {
+          const int e = pow2_exponent(amax, 448.0);
+          sb = std::ldexp(1.0, e);
+          const double eta_s = dzb + 2.0 * dzmax + std::ldexp(1.0, -19);
+          if (e > -127 && amax <= 448.0 * std::ldexp(1.0, e - 1) * (1.0 + eta_s)) sb_alt = std::ldexp(1.0, e - 1);
+          if (e < 127 && amax >= 448.0 * sb * (1.0 - eta_s)) sb_alt = std::ldexp(1.0, e + 1);
+        } else {
+          sb = amax / 448.0;
+        }
+      }
       const float* svb = sv + (b0 / 128) * (static_cast<int64_t>(Hkv) * D) + static_cast<int64_t>(g) * D;
       for (int64_t j = lo; j < hi; ++j) {
-        const double tq = z[j - j0] / sb;
+        const double pj = z[j - j0];
+        const double eta = dz[j - j0] + dzb + 2.0 * dzmax + std::ldexp(1.0, -19);
+        const double tq = pj / sb;
         const uint8_t code = e4m3_encode(static_cast<float>(tq));
         const double phat = dec[code] * sb;
-        // ambiguity: the nearest rounding midpoint of the E4M3 grid
-        const double eta = dz[j - j0] + dzb + 2.0 * dzmax + std::ldexp(1.0, -19);
-        double step = 0.0;
-        if (tq < 448.0) {
-          const double v = dec[code];
-          const double lo_g = v <= tq ? v : (code > 0 ? dec[code - 1] : 0.0);
-          const double hi_g = v <= tq ? (code < 0x7E ? dec[code + 1] : v) : v;
-          const double mid = 0.5 * (lo_g + hi_g);
-          if (hi_g > lo_g && std::fabs(tq - mid) <= eta * tq) step = hi_g - lo_g;
+        double amb = midpoint_step(dec, tq, code, eta) * sb;   // either rounding is correct
+        if (sb_alt > 0.0) {
+          const double tq2 = pj / sb_alt;
+          const uint8_t code2 = e4m3_encode(static_cast<float>(tq2));
+          const double d2 = std::fabs(dec[code2] * sb_alt - phat) + midpoint_step(dec, tq2, code2, eta) * sb_alt;
+          if (d2 > amb) amb = d2;
         }
         for (int64_t d = 0; d < D; ++d) {
           const double vv = dec[vT[(static_cast<int64_t>(g) * D + d) * T + j]] * svb[d];
           o[d] += phat * vv;
           oa[d] += std::fabs(phat * vv);
-          of[d] += step * sb * std::fabs(vv);
+          of[d] += amb * std::fabs(vv);
         }
       }
     }

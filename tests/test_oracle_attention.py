@@ -16,26 +16,26 @@ import torch
 D = 128
 
 
-def quant_rows(x, orc):
+def quant_rows(x, orc, mode=0):
     """1x128 row blocks (per token and head) with the oracle's quantizer."""
-    q, s, _, _ = orc.quant_act_1x128(x.view(torch.int16).numpy().view(np.uint16), 0, colwise=False)
+    q, s, _, _ = orc.quant_act_1x128(x.view(torch.int16).numpy().view(np.uint16), mode, colwise=False)
     return q, s
 
 
-def quant_v(x, orc):
+def quant_v(x, orc, mode=0):
     """V's column-wise copy: codes [H*128, T], scales [T/128, H*128]."""
-    _, _, qc, sc = orc.quant_act_1x128(x.view(torch.int16).numpy().view(np.uint16), 0)
+    _, _, qc, sc = orc.quant_act_1x128(x.view(torch.int16).numpy().view(np.uint16), mode)
     return qc, sc
 
 
-def make_case(orc, T, Hq, Hkv, seed, qscale=1.0):
+def make_case(orc, T, Hq, Hkv, seed, qscale=1.0, mode=0):
     g = torch.Generator().manual_seed(seed)
     Q = (torch.randn((T, Hq * D), generator=g) * qscale).to(torch.bfloat16)
     K = torch.randn((T, Hkv * D), generator=g).to(torch.bfloat16)
     V = torch.randn((T, Hkv * D), generator=g).to(torch.bfloat16)
-    q, sq = quant_rows(Q, orc)
-    k, sk = quant_rows(K, orc)
-    vT, sv = quant_v(V, orc)
+    q, sq = quant_rows(Q, orc, mode)
+    k, sk = quant_rows(K, orc, mode)
+    vT, sv = quant_v(V, orc, mode)
     return q, sq, k, sk, vT, sv
 
 
@@ -43,8 +43,17 @@ def e4m3_decode_torch(codes):
     return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
 
 
-def brute_force(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, t, h):
-    """Independent restatement: torch's E4M3 decode and cast, numpy softmax."""
+def pow2_scale(amax):
+    """Power-of-2 rule by frexp: amax / 448 = m 2^x with m in [0.5, 1); the
+    smallest power of two at or above it is 2^(x-1) when m == 0.5, else 2^x."""
+    m, x = math.frexp(amax / 448.0)
+    return math.ldexp(1.0, x - 1 if m == 0.5 else x)
+
+
+def brute_force(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, t, h, mode=0):
+    """Independent restatement: torch's E4M3 decode and cast, numpy softmax.
+    mode 1: p against the integer power-of-two reference ceil(max z log2 e)
+    and power-of-2 block scales."""
     T = q.shape[0]
     g = h // (Hq // Hkv)
     seg = max(i for i in range(len(ln)) if off[i] <= t)
@@ -55,31 +64,36 @@ def brute_force(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, t, h):
     qv = e4m3_decode_torch(q[t, h * D:(h + 1) * D]) * sq[h, t]
     kv = e4m3_decode_torch(k[j0:j1, g * D:(g + 1) * D]) * sk[g, j0:j1][:, None]
     z = kv @ qv / math.sqrt(D)
-    p = np.exp(z - z.max())
+    if mode == 1:
+        y = z / math.log(2.0)
+        p = np.exp2(y - math.ceil(y.max()))
+    else:
+        p = np.exp(z - z.max())
     l = p.sum()
     vv = e4m3_decode_torch(vT[g * D:(g + 1) * D, j0:j1]).T * sv[np.arange(j0, j1) // 128, g * D:(g + 1) * D]
     o = np.zeros(D)
     for b0 in range((j0 // 128) * 128, j1, 128):
         lo, hi = max(b0, j0), min(b0 + 128, j1)
         pb = p[lo - j0:hi - j0]
-        s = pb.max() / 448.0
+        s = pow2_scale(pb.max()) if mode == 1 else pb.max() / 448.0
         codes = torch.from_numpy((pb / s).astype(np.float32)).to(torch.float8_e4m3fn)
         phat = codes.to(torch.float64).numpy() * s
         o += phat @ vv[lo - j0:hi - j0]
     return o / l
 
 
+@pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("causal", [True, False])
-def test_brute_force_tiny(orc, causal):
+def test_brute_force_tiny(orc, causal, mode):
     Hq, Hkv, T = 4, 2, 512
-    q, sq, k, sk, vT, sv = make_case(orc, T, Hq, Hkv, 3)
+    q, sq, k, sk, vT, sv = make_case(orc, T, Hq, Hkv, 3, mode=mode)
     off, ln = [0, 256, 512], [200, 256]          # a padded segment and a full one
     rows = [(t, h) for t in (0, 1, 77, 128, 199, 200, 255, 256, 300, 511) for h in range(Hq)]
     rt = [r[0] for r in rows]
     rh = [r[1] for r in rows]
-    O, oa, of = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, rt, rh)
+    O, oa, of = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, rt, rh, mode)
     for i, (t, h) in enumerate(rows):
-        ref = brute_force(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, t, h)
+        ref = brute_force(q, sq, k, sk, vT, sv, Hq, Hkv, off, ln, causal, t, h, mode)
         np.testing.assert_allclose(O[i], ref, rtol=0, atol=1e-12 * (1 + oa[i].max()))
     # padding query rows are zero
     pad = [i for i, (t, _) in enumerate(rows) if 200 <= t < 256]
@@ -195,3 +209,88 @@ def test_flip_allowance_marks_midpoints(orc):
     sk[0, 1] = np.float32(sk[0, 0] * (1 + math.log(420.0 / 448.0) / zq))
     _, _, of1 = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, 1, 1, [0, T], [T], False, [0], [0])
     assert np.all(of1 == 0)
+
+
+def test_single_key_pow2_closed_form(orc):
+    """Power-of-2 mode, one key: p = 2^(y - ceil(y)) with y = z log2 e, so
+    p lies in (1/2, 1]; its block scale is 2^-8 for p > 448 2^-9 = 0.875 and
+    2^-9 otherwise, and O = v^ * E4M3(p / s) * s / p."""
+    for seed in range(12, 20):
+        q, sq, k, sk, vT, sv = make_case(orc, 128, 1, 1, seed, mode=1)
+        O, _, _ = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, 1, 1, [0, 128], [128], True, [0], [0], 1)
+        dec = np.array([orc.e4m3_decode(c) for c in range(256)])
+        z = float((dec[q[0]] * sq[0, 0]) @ (dec[k[0]] * sk[0, 0])) / math.sqrt(D)
+        y = z / math.log(2.0)
+        p = 2.0 ** (y - math.ceil(y))
+        s = 2.0 ** -8 if p > 0.875 else 2.0 ** -9
+        code = torch.tensor([p / s], dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).item()
+        vhat = dec[vT[:, 0]] * sv[0, :]
+        np.testing.assert_allclose(O[0], vhat * (code * s / p), rtol=1e-13, atol=0)
+
+
+def _pow2_row(orc, seed, targets):
+    """One causal row (t = len(targets) - 1) of a power-of-2 case whose key
+    logits are placed, through the key scales, so that key i has
+    p_i = targets[i] (p against the integer reference of the largest).  The
+    keys repeat the query's codes, so every product of the dot product is
+    positive and the oracle's logit error bound (and with it the midpoint
+    allowance) stays near 1e-4 relative."""
+    T = 128
+    q, sq, k, sk, vT, sv = make_case(orc, T, 1, 1, seed, mode=1)
+    dec = np.array([orc.e4m3_decode(c) for c in range(256)])
+    t = len(targets) - 1
+    k[:t + 1] = q[t]      # every product of the dot product positive: tight logit error bounds
+    qk = float((dec[q[t]] * sq[0, t]) @ dec[k[0]]) / math.sqrt(D) / math.log(2.0)   # y per unit key scale
+    top = 5.0 + math.log2(max(targets))          # ceil(top) = 5: reference 2^5
+    for i, pt in enumerate(targets):
+        sk[0, i] = np.float32((5.0 + math.log2(pt)) / qk)
+    O, oa, of = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, 1, 1, [0, T], [T], True, [t], [0], 1)
+    y = np.array([qk * float(sk[0, i]) for i in range(t + 1)])
+    p = 2.0 ** (y - math.ceil(y.max()))
+    vhat = dec[vT[:, :t + 1]].T * sv[0][None, :]
+    assert math.ceil(top) == 5
+    return O[0], of[0], p, vhat
+
+
+def test_pow2_boundary_single_key(orc):
+    """Power-of-2 mode, one key with p = 448 2^-9 = 0.875 (to fp32 accuracy):
+    amax / 448 sits on the boundary between the scales 2^-9 and 2^-8, and a
+    kernel's fp32 p may pick either; both codes (448 under 2^-9, 224 under
+    2^-8) decode to 0.875, so the allowance is 0 and O = v^ 0.875 / p."""
+    O, of, p, vhat = _pow2_row(orc, 21, [0.875])
+    assert abs(p[0] / 0.875 - 1) < 1e-6
+    assert np.all(of == 0)
+    np.testing.assert_allclose(O, vhat[0] * 0.875 / p[0], rtol=1e-12, atol=0)
+
+
+def test_pow2_boundary_subnormal_allowance(orc):
+    """Power-of-2 mode, two keys: the block maximum p_0 = 0.875 sits on a
+    scale boundary and p_1 = 4.6 2^-18 is tiny.  Under 2^-9, p_1 / s = 4.6
+    2^-9 is an E4M3 subnormal and rounds to 5 2^-9; under 2^-8 it is 2.3 2^-9
+    and rounds to 2 2^-9.  The dequantized values differ by 2^-18, and the
+    allowance of output channel d is that difference times |v^_1[d]| / l."""
+    O, of, p, vhat = _pow2_row(orc, 23, [0.875, 4.6 * 2.0 ** -18])
+    assert abs(p[0] / 0.875 - 1) < 1e-6 and abs(p[1] / (4.6 * 2.0 ** -18) - 1) < 1e-5
+    np.testing.assert_allclose(of, 2.0 ** -18 * np.abs(vhat[1]) / p.sum(), rtol=1e-9, atol=0)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gqa_and_causality_both_modes(orc, mode):
+    """GQA equals replicated KV heads, and causal rows ignore later keys, in
+    either scale mode."""
+    Hq, Hkv, T = 4, 2, 256
+    q, sq, k, sk, vT, sv = make_case(orc, T, Hq, Hkv, 22, mode=mode)
+    rep = [0, 0, 1, 1]
+    k4 = np.concatenate([k[:, g * D:(g + 1) * D] for g in rep], axis=1)
+    vT4 = np.concatenate([vT[g * D:(g + 1) * D] for g in rep], axis=0)
+    sv4 = np.concatenate([sv[:, g * D:(g + 1) * D] for g in rep], axis=1)
+    rt, rh = [3, 100, 255, 3], [0, 1, 2, 3]
+    a = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, [0, T], [T], True, rt, rh, mode)
+    b = orc.attention_fwd_rows(q, sq, k4, sk[rep], vT4, sv4, Hq, Hq, [0, T], [T], True, rt, rh, mode)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    k2, vT2 = k.copy(), vT.copy()
+    k2[101:] = 0x38
+    vT2[:, 101:] = 0x38
+    c = orc.attention_fwd_rows(q, sq, k2, sk, vT2, sv, Hq, Hkv, [0, T], [T], True, [3, 100], [0, 1], mode)
+    assert np.array_equal(c[0], a[0][:2])
