@@ -383,7 +383,7 @@ def moe_calls(fb, mode, layer):
     }
 
 
-def attn_call(fb, seed=0):
+def attn_call(fb, seed=0, mode=0):
     """FP8 attention forward over the packed long-sequence batch (32768
     tokens, 4 sequences), Llama-3.1-8B-like heads (32 query heads, 8 KV heads
     of 128), causal; Q, K, V quantized by the library's activation quantizer.
@@ -399,14 +399,14 @@ def attn_call(fb, seed=0):
     e = lambda *sh, dt=u8: torch.empty(sh, dtype=dt, device=dev)  # noqa: E731
     q, sq, k, sk = e(T, Hq * D), e(Hq, T, dt=f32), e(T, Hkv * D), e(Hkv, T, dt=f32)
     vr, svr, vT, sv = e(T, Hkv * D), e(Hkv, T, dt=f32), e(Hkv * D, T), e(T // 128, Hkv * D, dt=f32)
-    fb.fp8bw_quant_act_1x128(Q, 0, q, sq)
-    fb.fp8bw_quant_act_1x128(K, 0, k, sk)
-    fb.fp8bw_quant_act_1x128(V, 0, vr, svr, vT, sv)
+    fb.fp8bw_quant_act_1x128(Q, mode, q, sq)
+    fb.fp8bw_quant_act_1x128(K, mode, k, sk)
+    fb.fp8bw_quant_act_1x128(V, mode, vr, svr, vT, sv)
     o = e(T, Hq * D, dt=torch.bfloat16)
     offd = torch.tensor(off, dtype=torch.int32, device=dev)
     lnd = torch.tensor(ln, dtype=torch.int32, device=dev)
     flops = 4 * D * Hq * sum(n * (n + 1) // 2 for n in ln)
-    return (lambda: fb.fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, offd, lnd, 1), flops, "TFLOP/s")
+    return (lambda: fb.fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, offd, lnd, 1, mode), flops, "TFLOP/s")
 
 
 def run_case(args):
@@ -421,7 +421,8 @@ def run_case(args):
         time_call(fb, args, name, mode, fn, work, unit)
         return
     if args.case == "attn":
-        fn, work, unit = attn_call(fb)
+        fn, work, unit = attn_call(fb, mode=mode)
+        args.tokens = workloads.PACKED_TOKENS
         time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
         return
     if args.case == "requant_sweep":
@@ -496,11 +497,13 @@ def run_sweep(args):
                 time_call(fb, args, name, mode, fn, work, unit)
             del calls
             torch.cuda.empty_cache()
-        if mname == "fp32":
-            args.case = "attn"
-            fn, work, unit = attn_call(fb)
-            time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
-            torch.cuda.empty_cache()
+        args.case = "attn"
+        fn, work, unit = attn_call(fb, mode=mode)
+        tokens, args.tokens = args.tokens, workloads.PACKED_TOKENS
+        time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
+        args.tokens = tokens
+        del fn
+        torch.cuda.empty_cache()
         for name in ("gate_up", "down"):
             mc = moe_calls(fb, mode, name)
             for c in ("moe_fprop", "moe_dgrad", "moe_wgrad"):

@@ -70,7 +70,7 @@ def _load():
                                              vp, vp, vp, i64, vp]
     L.fp8bw_gemm_quant.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, i32, vp, i64, vp, vp, vp, vp, vp]
     L.fp8bw_attention_fwd.argtypes = [i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp,
-                                      ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp]
+                                      ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm", "fp8bw_attention_fwd",
               "fp8bw_gemm_quant",
               "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
@@ -241,14 +241,16 @@ def fp8bw_gemm_bf16(A, B, D, stream=None):
                                                   _stream(stream)))
 
 
-def fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, seg_off, seg_len, causal=True, stream=None):
+def fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, seg_off, seg_len, causal=True, mode=FP8BW_SCALE_FP32,
+                        stream=None):
     """FP8 attention forward.  q [T, Hq*128] u8, sq [Hq, T]; k [T, Hkv*128] u8,
     sk [Hkv, T]; vT [Hkv*128, T] u8, sv [T/128, Hkv*128]; o [T, Hq*128] bf16;
-    seg_off [nseg+1], seg_len [nseg]: device int32."""
+    seg_off [nseg+1], seg_len [nseg]: device int32; mode: the scales' rule
+    (FP8BW_SCALE_POW2: power-of-two scales, applied by the tensor core)."""
     T = q.shape[0]
     Hq, Hkv = q.shape[1] // 128, k.shape[1] // 128
     _check("fp8bw_attention_fwd", load().fp8bw_attention_fwd(
-        T, Hq, Hkv, seg_len.numel(), _ptr(seg_off), _ptr(seg_len), int(bool(causal)), _ptr(q), _ptr(sq),
+        T, Hq, Hkv, seg_len.numel(), _ptr(seg_off), _ptr(seg_len), int(bool(causal)), int(mode), _ptr(q), _ptr(sq),
         _ptr(k), _ptr(sk), _ptr(vT), _ptr(sv), _ptr(o), _stream(stream)))
 
 

@@ -29,7 +29,7 @@ cudaError_t launch_quant_tensor(const void* x, int64_t M, int64_t K, int64_t ldx
                                 float* scale, float* amax, float* s_grid, int64_t s_grid_len,
                                 int num_sms, cudaStream_t st);
 cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int32_t* d_off,
-                                 const int32_t* d_len, int causal, const uint8_t* q, const float* sq,
+                                 const int32_t* d_len, int causal, int mode, const uint8_t* q, const float* sq,
                                  const uint8_t* k, const float* sk, const uint8_t* vT, const float* sv,
                                  void* o, cudaStream_t st);
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
@@ -369,12 +369,14 @@ FP8BW_API fp8bw_status fp8bw_gemm_quant(fp8bw_gemm_kind kind, int64_t M, int64_t
 
 FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
                                            const int32_t* d_seg_off, const int32_t* d_seg_len,
-                                           int32_t causal, const uint8_t* q, const float* sq,
+                                           int32_t causal, fp8bw_scale_mode mode,
+                                           const uint8_t* q, const float* sq,
                                            const uint8_t* k, const float* sk, const uint8_t* vT,
                                            const float* sv, void* o, fp8bw_stream_t stream) {
   if (!d_seg_off || !d_seg_len || !q || !sq || !k || !sk || !vT || !sv || !o) return FP8BW_ERR_INVALID_ARG;
   if (T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || nseg < 1 || (causal != 0 && causal != 1))
     return FP8BW_ERR_INVALID_ARG;
+  if (mode != FP8BW_SCALE_FP32 && mode != FP8BW_SCALE_POW2) return FP8BW_ERR_INVALID_ARG;
   if (nseg > FP8BW_ATTN_MAX_SEGMENTS || Hq > FP8BW_ATTN_MAX_HEADS) return FP8BW_ERR_TOO_LARGE;
   if (T > kMaxDim || T * Hq * 128 > (int64_t(1) << 40)) return FP8BW_ERR_TOO_LARGE;
   if (!mult128(T)) return FP8BW_ERR_ALIGNMENT;
@@ -385,7 +387,7 @@ FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, i
   fp8bw_status st = current(&sms);
   if (st != FP8BW_OK) return st;
   if (T == 0) return FP8BW_OK;
-  return from_cuda(fp8bw::launch_attention_fwd(T, Hq, Hkv, nseg, d_seg_off, d_seg_len, causal, q, sq, k,
+  return from_cuda(fp8bw::launch_attention_fwd(T, Hq, Hkv, nseg, d_seg_off, d_seg_len, causal, (int)mode, q, sq, k,
                                                sk, vT, sv, o, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -111,7 +111,8 @@ struct AttnArgs {
   uint16_t* o;          // [T][Hq*128] bf16
 };
 
-__device__ __forceinline__ void raise_attn_timeout(AttnBars* b) {
+template <class Bars>
+__device__ __forceinline__ void raise_attn_timeout(Bars* b) {
   atomicOr(&g_attn_error, DEV_ERR_TIMEOUT);
   atomicExch(&b->abort, 1);
 }
@@ -204,10 +205,98 @@ __device__ __forceinline__ bool fold_block(AttnSmem& sm, AttnBars* bars, uint32_
 // The kNH warps of lane quarter q meet (each after writing its part's value
 // to shared memory); `uses` counts this quarter's earlier meetings.  False if
 // another warp did not arrive in time.
-__device__ __forceinline__ bool pair_meet(AttnBars* bars, int q, int lane, uint32_t uses) {
+template <class Bars>
+__device__ __forceinline__ bool pair_meet(Bars* bars, int q, int lane, uint32_t uses) {
   __syncwarp();
   if (lane == 0) mbar_arrive(smem_u32(&bars->pair[q]));
   return warp_wait(smem_u32(&bars->pair[q]), uses & 1);
+}
+
+// TMA producer (one thread): the Q tile once, then per 128-key block the K
+// tile [128 keys][128] and the V tile [128 channels][128 keys] into the
+// kStages ring, and the block's 128 key scales and 128 channel scales (bulk
+// copies) into the kScSlots ring.
+template <class Smem, class Bars>
+__device__ __forceinline__ void attn_producer(Smem& sm, Bars* bars, const CUtensorMap* tmQ,
+                                              const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                              const AttnArgs& a, int h, int g, int q0, int kb_first, int nb) {
+  prefetch_tmap(tmQ);
+  prefetch_tmap(tmK);
+  prefetch_tmap(tmV);
+  mbar_arrive_expect_tx(smem_u32(&bars->q_full), kTile);
+  tma_load_2d(smem_u32(sm.q), tmQ, smem_u32(&bars->q_full), h * kD, q0);
+  for (int b = 0; b < nb; ++b) {
+    const int kb = kb_first + b, s = b % kStages, sl = b % kScSlots;
+    if (!mbar_wait(smem_u32(&bars->kv_empty[s]), ((b / kStages) & 1) ^ 1)) {
+      raise_attn_timeout(bars);
+      break;
+    }
+    mbar_arrive_expect_tx(smem_u32(&bars->kv_full[s]), 2 * kTile);
+    tma_load_2d(smem_u32(sm.kv[s][0]), tmK, smem_u32(&bars->kv_full[s]), g * kD, kb * 128);
+    tma_load_2d(smem_u32(sm.kv[s][1]), tmV, smem_u32(&bars->kv_full[s]), kb * 128, g * kD);
+    if (!mbar_wait(smem_u32(&bars->sc_empty[sl]), ((b / kScSlots) & 1) ^ 1)) {
+      raise_attn_timeout(bars);
+      break;
+    }
+    mbar_arrive_expect_tx(smem_u32(&bars->sc_full[sl]), 1024);
+    bulk_load(smem_u32(sm.sc[sl].sk), a.sk + (size_t)g * a.T + kb * 128, 512, smem_u32(&bars->sc_full[sl]));
+    bulk_load(smem_u32(sm.sc[sl].sv), a.sv + (size_t)kb * a.Hkv * kD + g * kD, 512,
+              smem_u32(&bars->sc_full[sl]));
+    if (bars->abort) break;
+  }
+}
+
+// The CTA's work: query block qb (heavy, late blocks launched first) of
+// head h, its segment and key blocks.  Validates the segment table (every
+// CTA; an invalid one latches FP8BW_ERR_DEVICE_CHECK and nothing is written)
+// and writes zeros for a query block that is all padding; done = true then.
+// Called by every thread (it synchronizes the CTA).
+struct AttnBlock {
+  int qb, h, g, q0, j0, jreal, kb_first, nb;
+  bool done;
+};
+
+template <int NT>
+__device__ __forceinline__ AttnBlock attn_block(const AttnArgs& a, int* s_seg) {
+  AttnBlock w;
+  const int nqb = a.T / 128;
+  w.qb = nqb - 1 - (int)(blockIdx.x / a.Hq);
+  w.h = (int)(blockIdx.x % a.Hq);
+  w.g = w.h / (a.Hq / a.Hkv);
+  w.q0 = w.qb * 128;
+  w.done = false;
+  if (threadIdx.x == 0) *s_seg = -1;
+  __syncthreads();
+  int bad = 0;
+  for (int i = threadIdx.x; i < a.nseg; i += NT) {
+    const int o0 = a.off[i], o1 = a.off[i + 1], ln = a.len[i];
+    if (o1 < o0 || (o0 & 127) || (o1 & 127) || ln < 0 || ln > o1 - o0 || (i == 0 && o0 != 0)) bad = 1;
+    if (o0 <= w.q0 && w.q0 < o1) *s_seg = i;   // at most one segment holds the block
+  }
+  if (threadIdx.x == 0 && a.off[a.nseg] > a.T) bad = 1;
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0) atomicOr(&g_attn_error, DEV_ERR_CHECK);
+    w.done = true;
+    return w;
+  }
+  const int seg = *s_seg;                      // -1: past the last segment
+  w.j0 = seg >= 0 ? a.off[seg] : w.q0;
+  w.jreal = seg >= 0 ? w.j0 + a.len[seg] : w.q0;   // first padding token of the segment
+  if (w.q0 >= w.jreal) {
+    // the whole query block is padding: zeros
+    uint16_t* orow_base = a.o + (size_t)w.h * kD;
+    const size_t ostride = (size_t)a.Hq * kD;
+    for (int idx = threadIdx.x; idx < 128 * 8; idx += NT) {
+      const int r = idx >> 3, c = idx & 7;
+      st_global_v8(orow_base + (size_t)(w.q0 + r) * ostride + c * 16, make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0));
+    }
+    w.done = true;
+    return w;
+  }
+  w.kb_first = w.j0 / 128;
+  const int kb_last = a.causal ? min(w.qb, (w.jreal - 1) / 128) : (w.jreal - 1) / 128;
+  w.nb = kb_last - w.kb_first + 1;
+  return w;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -219,47 +308,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   AttnBars* bars = &sm.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- which block: heavy (late) query blocks first
-  const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)(blockIdx.x / a.Hq);
-  const int h = (int)(blockIdx.x % a.Hq);
-  const int g = h / (a.Hq / a.Hkv);
-  const int q0 = qb * 128;
-
-  // ---- validate the segment table (every CTA; nothing written if invalid)
   __shared__ int s_seg;
-  if (threadIdx.x == 0) s_seg = -1;
-  __syncthreads();
-  {
-    int bad = 0;
-    for (int i = threadIdx.x; i < a.nseg; i += kThreads) {
-      const int o0 = a.off[i], o1 = a.off[i + 1], ln = a.len[i];
-      if (o1 < o0 || (o0 & 127) || (o1 & 127) || ln < 0 || ln > o1 - o0 || (i == 0 && o0 != 0)) bad = 1;
-      if (o0 <= q0 && q0 < o1) s_seg = i;   // at most one segment holds the block
-    }
-    if (threadIdx.x == 0 && a.off[a.nseg] > a.T) bad = 1;
-    if (__syncthreads_or(bad)) {
-      if (threadIdx.x == 0) atomicOr(&g_attn_error, DEV_ERR_CHECK);
-      return;
-    }
-  }
-  const int seg = s_seg;                      // -1: past the last segment
-  const int j0 = seg >= 0 ? a.off[seg] : q0;
-  const int jreal = seg >= 0 ? j0 + a.len[seg] : q0;   // first padding token of the segment
+  const AttnBlock wk = attn_block<kThreads>(a, &s_seg);
+  if (wk.done) return;
+  const int h = wk.h, g = wk.g, q0 = wk.q0, jreal = wk.jreal;
+  const int kb_first = wk.kb_first, nb = wk.nb;
   uint16_t* orow_base = a.o + (size_t)h * kD;
   const size_t ostride = (size_t)a.Hq * kD;
-
-  if (q0 >= jreal) {
-    // the whole query block is padding: zeros
-    for (int idx = threadIdx.x; idx < 128 * 8; idx += kThreads) {
-      const int r = idx >> 3, c = idx & 7;
-      st_global_v8(orow_base + (size_t)(q0 + r) * ostride + c * 16, make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0));
-    }
-    return;
-  }
-  const int kb_first = j0 / 128;
-  const int kb_last = a.causal ? min(qb, (jreal - 1) / 128) : (jreal - 1) / 128;
-  const int nb = kb_last - kb_first + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
@@ -296,32 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(smem_u32(&bars->q_full), kTile);
-      tma_load_2d(smem_u32(sm.q), &tmQ, smem_u32(&bars->q_full), h * kD, q0);
-      for (int b = 0; b < nb; ++b) {
-        const int kb = kb_first + b, s = b % kStages, sl = b % kScSlots;
-        if (!mbar_wait(smem_u32(&bars->kv_empty[s]), ((b / kStages) & 1) ^ 1)) {
-          raise_attn_timeout(bars);
-          break;
-        }
-        mbar_arrive_expect_tx(smem_u32(&bars->kv_full[s]), 2 * kTile);
-        tma_load_2d(smem_u32(sm.kv[s][0]), &tmK, smem_u32(&bars->kv_full[s]), g * kD, kb * 128);
-        tma_load_2d(smem_u32(sm.kv[s][1]), &tmV, smem_u32(&bars->kv_full[s]), kb * 128, g * kD);
-        if (!mbar_wait(smem_u32(&bars->sc_empty[sl]), ((b / kScSlots) & 1) ^ 1)) {
-          raise_attn_timeout(bars);
-          break;
-        }
-        mbar_arrive_expect_tx(smem_u32(&bars->sc_full[sl]), 1024);
-        bulk_load(smem_u32(sm.sc[sl].sk), a.sk + (size_t)g * a.T + kb * 128, 512, smem_u32(&bars->sc_full[sl]));
-        bulk_load(smem_u32(sm.sc[sl].sv), a.sv + (size_t)kb * a.Hkv * kD + g * kD, 512,
-                  smem_u32(&bars->sc_full[sl]));
-        if (bars->abort) break;
-      }
-    }
+    if (lane == 0) attn_producer(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
   } else if (warp == 1) {
     // ----------------------------------------------------- MMA issuer -----
     if (lane == 0) {
@@ -549,10 +579,395 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------
+// Power-of-2 scales ("Warum dies für die KI-Ökonomie wichtig ist": the
+// recipe's optional power-of-2 scale factors).  Every scale is then a UE8M0
+// value, so the tensor core applies them itself
+// (tcgen05.mma.kind::mxf8f6f4.block_scale, one scale per row per 32-element
+// block, here replicated over the four 32-blocks of a 128-wide one): Q's
+// and K's scales inside S = Q K^T, which comes out fully scaled, and P's and
+// V's inside O += P V^T, which accumulates across key blocks in one TMEM
+// accumulator.  There is no per-block fold: the softmax warps rescale O in
+// TMEM only when a row's running maximum moves, and they keep that maximum
+// an integer (log2 units) that moves only when a block's maximum exceeds it
+// by more than kLazy.  P is taken against it, p / s_P = 2^(y c - m - e), e
+// the power-of-2 exponent of the block's amax = 2^(m_b - m); any integer
+// reference gives the same codes.  Roles as in k_attn_fwd, plus warp 2,
+// which turns each block's fp32 scales into UE8M0 tiles in shared memory
+// (row i + 32b of 128 at word [i][b], the byte replicated), and latches
+// FP8BW_ERR_DEVICE_CHECK for a scale that is not a power of two.
+// TMEM: S at 0 and 128, O at 256, scale tiles (4 columns each) from 384.
+constexpr uint32_t kMxO = 256;
+constexpr uint32_t kMxSfq = 384, kMxSfk = 388, kMxSfp = 396, kMxSfv = 404;   // K, P, V: two slots each
+constexpr float kLazy = 8.0f;
+
+struct SfTile {
+  uint32_t w[32][4];
+};
+
+struct AttnBarsMx {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t sc_full[kScSlots], sc_empty[kScSlots];
+  uint64_t sfq_full, sfkv_full[2], sfkv_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t o_full;           // one P.V into O complete
+  uint64_t pair[4];
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct AttnSmemMx {
+  uint8_t q[kTile];                    // 1024-aligned tiles first
+  uint8_t kv[kStages][2][kTile];
+  uint8_t p[2][kTile];
+  SfTile sfq, sfk[2], sfv[2], sfp[2];  // UE8M0 tiles for tcgen05.cp (16-byte rows)
+  ScSlot sc[kScSlots];
+  float red[2][kNH][128];
+  float lsum[kNH][128];
+  AttnBarsMx bars;
+};
+
+// The UE8M0 byte of a positive power-of-two fp32 scale, replicated into the
+// four bytes of a word (2^-127 is the subnormal 0x00400000: code 0).
+__device__ __forceinline__ uint32_t ue8m0_word(float s, bool& bad) {
+  const uint32_t b = __float_as_uint(s);
+  if (((b & 0x7FFFFFu) != 0u && b != 0x00400000u) || (b >> 23) == 0xFFu || (b >> 31) != 0u || b == 0u) bad = true;
+  return ((b >> 23) & 0xFFu) * 0x01010101u;
+}
+
+// One warp: the 128 scales src[0..127] as a UE8M0 tile.
+__device__ __forceinline__ bool sf_tile(const float* src, SfTile* dst, int lane) {
+  bool bad = false;
+  uint4 v;
+  v.x = ue8m0_word(src[lane], bad);
+  v.y = ue8m0_word(src[lane + 32], bad);
+  v.z = ue8m0_word(src[lane + 64], bad);
+  v.w = ue8m0_word(src[lane + 96], bad);
+  *reinterpret_cast<uint4*>(&dst->w[lane][0]) = v;
+  return bad;
+}
+
+// 2^e for an integer e in [-126, 127] (exact).
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// Softmax and correction warps of k_attn_fwd_mx (one query row per thread,
+// kCols of its 128 columns): per key block, S_b (fully scaled by the MMA)
+// from TMEM, mask and block maximum (combined across the row's kNH parts),
+// the integer running maximum, the P codes 2^(y c - m - e) and the row's
+// scale byte e + 127 into shared memory, the rescale of O in TMEM when the
+// row's maximum moved (after the previous P.V is complete), then the signal
+// for the next P.V.  At the end O / l in bf16.
+__device__ __forceinline__ void attn_softmax_mx(AttnSmemMx& sm, AttnBarsMx* bars, uint32_t tmem,
+                                                const AttnArgs& a, int warp, int lane, int h, int q0,
+                                                int jreal, int kb_first, int nb) {
+  const int q = warp & 3, hf = (warp - 4) >> 2;   // lane quarter, column part
+  const int i = q * 32 + lane, t = q0 + i;
+  const int col0 = hf * kCols;
+  constexpr float c = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+  const int jend = a.causal ? min(jreal, t + 1) : jreal;
+  const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+  constexpr int kU = kCols / 32;
+  float m = -INFINITY, lh = 0.0f;
+  bool ok = true;
+  uint32_t meets = 0;
+
+  for (int b = 0; b < nb && ok; ++b) {
+    const int kb = kb_first + b;
+    if (!warp_wait(smem_u32(&bars->s_full[b & 1]), (b >> 1) & 1)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    uint32_t r[kU][32];
+    const uint32_t ta = tmem + lane_off + (b & 1) * 128 + col0;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) tmem_ld32(ta + 32 * u, r[u]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < kU; ++u) tmem_fence_regs(r[u]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b & 1]));
+
+    const int lim = jend - kb * 128 - col0;      // columns >= lim are masked
+    if (lim < kCols) {
+#pragma unroll
+      for (int j = 0; j < kCols; ++j)
+        if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+    }
+    float mh;
+    {
+      float mg[kCols / 8];
+#pragma unroll
+      for (int gi = 0; gi < kCols / 8; ++gi) {
+        const uint32_t* v = &r[(8 * gi) >> 5][(8 * gi) & 31];
+        mg[gi] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                       fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                       fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+      }
+      mh = mg[0];
+#pragma unroll
+      for (int gi = 1; gi + 1 < kCols / 8; gi += 2) mh = fmax3(mh, mg[gi], mg[gi + 1]);
+      if ((kCols / 8) % 2 == 0) mh = fmaxf(mh, mg[kCols / 8 - 1]);
+    }
+    sm.red[b & 1][hf][i] = mh;
+    if (!pair_meet(bars, q, lane, meets++)) {
+      ok = false;
+      break;
+    }
+    float mrow = sm.red[b & 1][0][i];
+#pragma unroll
+    for (int k = 1; k < kNH; ++k) mrow = fmaxf(mrow, sm.red[b & 1][k][i]);
+    const float mb = mrow * c;                   // the block's largest logit, log2 units
+    // integer running maximum, moved only by more than kLazy (then p may
+    // reach 2^kLazy in between, harmless in fp32)
+    const float m_new = mb > m + kLazy ? ceilf(mb) : m;
+    const bool moved = m_new != m;
+    const float dm = m - m_new;                  // an integer, or -inf on the first block
+    const float alpha = moved ? (dm < -126.0f ? 0.0f : exp2i((int)dm)) : 1.0f;
+    m = m_new;
+    // P's power-of-2 block scale 2^e: the smallest e with 2^(mb - m) <= 448 2^e
+    int e = (int)ceilf((mb - m) - kLog2_448);
+    e = max(-127, min(127, e));
+    const float sp = e == -127 ? __uint_as_float(0x00400000u) : exp2i(e);
+    const float2 c2 = make_float2(c, c);
+    const float off = -(m + (float)e);
+    const float2 nm2 = make_float2(off, off);
+    float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int j = 0; j < kCols; j += 2) {
+      const int u = j >> 5, k = j & 31;
+      const float2 z = ffma2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), c2, nm2);
+      const float2 pj = make_float2(ex2(z.x), ex2(z.y));
+      r[u][k] = __float_as_uint(pj.x);
+      r[u][k + 1] = __float_as_uint(pj.y);
+      ps2[(j >> 1) & 3] = fadd2(ps2[(j >> 1) & 3], pj);
+    }
+    const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+    lh = lh * alpha + sp * (psum.x + psum.y);
+    uint32_t w[kCols / 4];
+#pragma unroll
+    for (int j = 0; j < kCols / 4; ++j) {
+      const int u = j >> 3, k = 4 * (j & 7);
+      w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])) |
+             (cvt_e4m3x2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])) << 16);
+    }
+    if (!warp_wait(smem_u32(&bars->p_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
+      ok = false;
+      break;
+    }
+    // row i of the P tile: 16-byte chunk c at c ^ (i & 7) (128-byte swizzle)
+    uint8_t* prow = sm.p[b & 1] + i * 128;
+#pragma unroll
+    for (int cc = 0; cc < kCols / 16; ++cc)
+      *reinterpret_cast<uint4*>(prow + (((hf * (kCols / 16) + cc) ^ (i & 7)) << 4)) =
+          make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+    if (hf == 0) sm.sfp[b & 1].w[i & 31][i >> 5] = (uint32_t)(e + 127) * 0x01010101u;
+    if (b >= 1) {
+      // the previous P.V is complete; rescale O if a row of this warp moved
+      if (!warp_wait(smem_u32(&bars->o_full), (b - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          uint32_t o[32];
+          const uint32_t to = tmem + lane_off + kMxO + col0 + 32 * u;
+          tmem_ld32(to, o);
+          tmem_wait_ld();
+          tmem_fence_regs(o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(to, o);
+        }
+        tmem_wait_st();
+      }
+    }
+    fence_proxy_async_smem();   // the P tile and scale bytes, for the MMA
+    tc_fence_before();          // the rescaled O, for the MMA that accumulates onto it
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[b & 1]));
+    if (bars->abort) ok = false;
+  }
+  if (ok && !warp_wait(smem_u32(&bars->o_full), (nb - 1) & 1)) ok = false;
+  tc_fence_after();
+  if (!ok) raise_attn_timeout(bars);
+  // row sum of the kNH parts, then O / l in bf16 (padding rows: 0)
+  sm.lsum[hf][i] = lh;
+  if (!pair_meet(bars, q, lane, meets++)) ok = false;
+  float l = sm.lsum[0][i];
+#pragma unroll
+  for (int k = 1; k < kNH; ++k) l += sm.lsum[k][i];
+  const bool real = t < jreal && ok;
+  const float il = real ? __fdiv_rn(1.0f, l) : 0.0f;
+  uint16_t* orow = a.o + (size_t)h * kD + (size_t)t * ((size_t)a.Hq * kD) + col0;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    uint32_t o[32];
+    tmem_ld32(tmem + lane_off + kMxO + col0 + 32 * u, o);
+    tmem_wait_ld();
+    tmem_fence_regs(o);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t o8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o8[j] = real ? pack_bf16x2(__uint_as_float(o[16 * cc + 2 * j]) * il,
+                                   __uint_as_float(o[16 * cc + 2 * j + 1]) * il)
+                     : 0u;
+      st_global_v8(orow + 32 * u + 16 * cc, make_uint4(o8[0], o8[1], o8[2], o8[3]),
+                   make_uint4(o8[4], o8[5], o8[6], o8[7]));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd_mx(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmemMx& sm = *reinterpret_cast<AttnSmemMx*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                  ~uintptr_t(1023));
+  AttnBarsMx* bars = &sm.bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_seg;
+  const AttnBlock wk = attn_block<kThreads>(a, &s_seg);
+  if (wk.done) return;
+  const int h = wk.h, g = wk.g, q0 = wk.q0, jreal = wk.jreal;
+  const int kb_first = wk.kb_first, nb = wk.nb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->kv_full[i]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < kScSlots; ++i) {
+      mbar_init(smem_u32(&bars->sc_full[i]), 1);
+      mbar_init(smem_u32(&bars->sc_empty[i]), 1);   // read by the scale converter only
+    }
+    mbar_init(smem_u32(&bars->sfq_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->sfkv_full[i]), 1);
+      mbar_init(smem_u32(&bars->sfkv_empty[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->s_empty[i]), kSoftWarps);
+      mbar_init(smem_u32(&bars->p_full[i]), kSoftWarps);
+      mbar_init(smem_u32(&bars->p_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&bars->o_full), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), kNH);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) attn_producer(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
+  } else if (warp == 1) {
+    // ----------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_mx(128, 128, 0);   // E4M3 x E4M3, UE8M0 scales, byte 0
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0) && mbar_wait(smem_u32(&bars->sfq_full), 0);
+      tc_fence_after();
+      if (ok) tmem_cp_32x128b_x4(tmem + kMxSfq, sdesc_k_noswz_16B(smem_u32(&sm.sfq.w[0][0])));
+      const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q));
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
+          const int s = b % kStages;
+          if (!mbar_wait(smem_u32(&bars->kv_full[s]), (b / kStages) & 1) ||
+              !mbar_wait(smem_u32(&bars->s_empty[b & 1]), ((b >> 1) & 1) ^ 1) ||
+              !mbar_wait(smem_u32(&bars->sfkv_full[b & 1]), (b >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tk = tmem + kMxSfk + 4 * (b & 1);
+          tmem_cp_32x128b_x4(tk, sdesc_k_noswz_16B(smem_u32(&sm.sfk[b & 1].w[0][0])));
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.kv[s][0]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_mx(tmem + (b & 1) * 128, dq + 2 * kk, dk + 2 * kk, idesc, tmem + kMxSfq, tk, kk > 0 ? 1u : 0u);
+          umma_commit(smem_u32(&bars->s_full[b & 1]));
+        }
+        if (b >= 1) {
+          const int c = b - 1, s = c % kStages;
+          if (!mbar_wait(smem_u32(&bars->p_full[c & 1]), (c >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tp = tmem + kMxSfp + 4 * (c & 1), tv = tmem + kMxSfv + 4 * (c & 1);
+          tmem_cp_32x128b_x4(tp, sdesc_k_noswz_16B(smem_u32(&sm.sfp[c & 1].w[0][0])));
+          tmem_cp_32x128b_x4(tv, sdesc_k_noswz_16B(smem_u32(&sm.sfv[c & 1].w[0][0])));
+          const uint64_t dp = sdesc_k_sw128(smem_u32(sm.p[c & 1]));
+          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.kv[s][1]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_mx(tmem + kMxO, dp + 2 * kk, dv + 2 * kk, idesc, tp, tv, (c > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&bars->p_empty[c & 1]));
+          umma_commit(smem_u32(&bars->kv_empty[s]));
+          umma_commit(smem_u32(&bars->sfkv_empty[c & 1]));
+          umma_commit(smem_u32(&bars->o_full));
+        }
+        if (bars->abort) break;
+      }
+      if (!ok) raise_attn_timeout(bars);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ scale converter -----
+    bool bad = sf_tile(a.sq + (size_t)h * a.T + q0, &sm.sfq, lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->sfq_full));
+    for (int b = 0; b < nb; ++b) {
+      const int sl = b % kScSlots;
+      if (!warp_wait(smem_u32(&bars->sc_full[sl]), (b / kScSlots) & 1) ||
+          !warp_wait(smem_u32(&bars->sfkv_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
+        if (lane == 0) raise_attn_timeout(bars);
+        break;
+      }
+      bad |= sf_tile(sm.sc[sl].sk, &sm.sfk[b & 1], lane);
+      bad |= sf_tile(sm.sc[sl].sv, &sm.sfv[b & 1], lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bars->sfkv_full[b & 1]));
+        mbar_arrive(smem_u32(&bars->sc_empty[sl]));
+      }
+      if (bars->abort) break;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_attn_error, DEV_ERR_CHECK);
+  }
+  } else {
+    regs_inc<kRegsHigh>();
+    attn_softmax_mx(sm, bars, tmem, a, warp, lane, h, q0, jreal, kb_first, nb);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int32_t* d_off,
-                                 const int32_t* d_len, int causal, const uint8_t* q, const float* sq,
+                                 const int32_t* d_len, int causal, int mode, const uint8_t* q, const float* sq,
                                  const uint8_t* k, const float* sk, const uint8_t* vT, const float* sv,
                                  void* o, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
@@ -577,17 +992,20 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
   a.sk = sk;
   a.sv = sv;
   a.o = static_cast<uint16_t*>(o);
-  const size_t smem = sizeof(AttnSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool mx = mode == FP8BW_SCALE_POW2;
+  const void* kern = mx ? reinterpret_cast<const void*>(k_attn_fwd_mx) : reinterpret_cast<const void*>(k_attn_fwd);
+  const size_t smem = (mx ? sizeof(AttnSmemMx) : sizeof(AttnSmem)) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes attr;
-  e = cudaFuncGetAttributes(&attr, k_attn_fwd);
+  e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
   // setmaxnreg draws on the launch allocation: refuse to launch if the
   // compiled register count could not cover the split.
   if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
   const unsigned grid = (unsigned)((T / 128) * Hq);
-  k_attn_fwd<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  if (mx) k_attn_fwd_mx<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  else k_attn_fwd<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

@@ -349,6 +349,16 @@ FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int6
  * |o - ref| <= 1e-2 * sum_j |p^_j v^_j| / l + (one E4M3 step of each p_j
  * whose p / s lies within the kernel's fp32 error of a rounding midpoint)
  * + 1 bf16 ulp of the fp64 reference of the same definition.
+ * mode = FP8BW_SCALE_POW2 (the recipe's optional power-of-2 scales,
+ * "Warum dies für die KI-Ökonomie wichtig ist"): sq, sk and sv must be
+ * powers of two, as fp8bw_quant_act_1x128 makes them in that mode; the
+ * tensor core then applies every scale itself (block-scaled MMA), and P's
+ * block scale is the power-of-2 rule on its amax, p taken against an integer
+ * power-of-two reference maximum (any such reference gives the same codes).
+ * The result is within the gate above, widened where the block amax sits
+ * within the kernel's error of a power-of-two boundary (either scale is
+ * correct there).  A scale that is not a power of two latches
+ * FP8BW_ERR_DEVICE_CHECK and leaves o undefined.
  * Requires T a multiple of 128, Hq a multiple of Hkv, Hq <=
  * FP8BW_ATTN_MAX_HEADS, 1 <= nseg <= FP8BW_ATTN_MAX_SEGMENTS, 16-byte
  * aligned codes and scales.  Invalid offsets are rejected on the device:
@@ -358,7 +368,8 @@ FP8BW_API fp8bw_status fp8bw_quant_tensor_delayed(const void* x, int64_t M, int6
 #define FP8BW_ATTN_MAX_HEADS 1024
 FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
                                            const int32_t* d_seg_off, const int32_t* d_seg_len,
-                                           int32_t causal, const uint8_t* q, const float* sq,
+                                           int32_t causal, fp8bw_scale_mode mode,
+                                           const uint8_t* q, const float* sq,
                                            const uint8_t* k, const float* sk, const uint8_t* vT,
                                            const float* sv, void* o, fp8bw_stream_t stream);
 
