@@ -248,7 +248,7 @@ struct TileInfo {
 // [off[g], off[g+1]) form ceil(rows/256) of them (pp[g] = those of the
 // experts before g); in the last one the second CTA's 128 rows may lie past
 // the segment, and that CTA then writes nothing.
-template <int KIND, bool GROUPED, bool PAIR>
+template <int KIND, bool GROUPED, bool PAIR, bool WARP = false>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const int32_t* off,
                                                 const int32_t* pp, int& hint) {
   TileInfo ti;
@@ -278,11 +278,24 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, int t, const 
       return ti;
     }
     // The expert that owns pt: the last g with pp[g] <= pt.  A role visits
-    // its tiles in increasing order, so the search walks forward from the
-    // expert of its previous tile (`hint`): one or two dependent shared
-    // loads per tile instead of a full binary search.
+    // its tiles in increasing order, so the search moves forward from the
+    // expert of its previous tile (`hint`).  A role steps over one tile per
+    // CTA pair, so with short experts it passes many of them per tile: a
+    // whole warp (WARP) tests the next 32 experts at once (pp is
+    // non-decreasing, so the passing lanes are a prefix and their count is
+    // the step); a single thread walks one expert per shared load.
     int g = hint;
-    while (g + 1 < a.G && pp[g + 1] <= pt) ++g;
+    if (WARP) {
+      const int lane = (int)(threadIdx.x & 31);
+      for (;;) {
+        const int cand = g + 1 + lane;
+        const int adv = __popc(__ballot_sync(0xffffffffu, cand < a.G && pp[cand] <= pt));
+        g += adv;
+        if (adv < 32) break;
+      }
+    } else {
+      while (g + 1 < a.G && pp[g + 1] <= pt) ++g;
+    }
     hint = g;
     ti.g = g;
     ti.m0 = off[g] + (pt - pp[g]) * (2 * BM);
@@ -482,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
@@ -557,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sphase = 0;
       const int nKb = a.K / BK, nNb = a.N / 128;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const bool rows_ok = row0 < a.M;
@@ -604,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
       if (ti.skip) continue;
       const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
@@ -1007,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, chunk = 0;
       uint32_t phase = 0;
       for (int t = cta_slot; t < a.tiles; t += cta_step) {
-        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+        const TileInfo ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
         if (ti.skip) continue;
         const int arow = ti.m0 + (PAIR ? (int)rank * BM : 0);
         const int brow = PAIR ? ti.nt * BN + (int)rank * (BN / 2) : ti.nt * BN;
@@ -1119,7 +1132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool have = t < a.tiles;
         TileInfo ti = {};
         if (have) {
-          ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+          ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
           if (ti.skip) continue;
         }
         const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
@@ -1192,7 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* epi0 = epi_base + (warp - 4) * kMxEpiBufs * kEpiPiece;
     uint32_t tphase = 0;
     for (int t = cta_slot; t < a.tiles; t += cta_step) {
-      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR>(a, t, s_off, s_pp, ghint);
+      const TileInfo ti = decode_tile<KIND, GROUPED, PAIR, KIND != FP8BW_WGRAD>(a, t, s_off, s_pp, ghint);
       if (ti.skip) continue;
       const int row0 = ti.m0 + (PAIR ? (int)rank * BM : 0);
       const int col0 = ti.nt * BN + half * 128;
