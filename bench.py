@@ -226,6 +226,28 @@ def bf16_ratio(fb, layers, reps=3):
     return tot_flops / (tot_ms * 1e-3) / 1e12
 
 
+def attn_rates(fb, reps=10):
+    """FP8 attention forward over the packed 32K-token batch in both scale
+    modes (outside the timed step): TFLOP/s of 10 launches after 3 warm-up."""
+    out = {}
+    for name, mode in (("fp32", 0), ("pow2", 1)):
+        fn, work, _ = attn_call(fb, mode=mode)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        out[name] = work / (s.elapsed_time(e) / reps * 1e-3) / 1e12
+        del fn
+        torch.cuda.empty_cache()
+    out["workload"] = "packed 32768 tokens (4 sequences), 32 query / 8 KV heads of 128, causal"
+    return out
+
+
 # ---------------------------------------------------------- CPU oracle ----
 _ORC = {}
 
@@ -686,6 +708,7 @@ def main():
 
     # ---- BF16 comparison GEMMs (outside the timed region)
     bf16 = bf16_ratio(fb, layers) if rank == 0 else None
+    attn = attn_rates(fb) if rank == 0 else None
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -791,7 +814,8 @@ def main():
                       "requant_ms_per_step": req_ms, "requant_gbs": req_bytes / (req_ms * 1e-3) / 1e9,
                       "hbm_peak_gbs": pk["hbm_gbs"],
                       "bf16_gemm_tflops": bf16, "fp8_over_bf16": (gemm_tflops / bf16) if bf16 else None,
-                      "requant_over_step": req_ms / ms_step},
+                      "requant_over_step": req_ms / ms_step,
+                      "attention_tflops": attn},
             "steady_state": steady,
             "pow2_scales": pow2,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
