@@ -173,25 +173,38 @@ def build_layers(dev, M=workloads.LLAMA8B_TOKENS):
 
 
 def run_step(fb, layers, mode, ev=None):
-    """One step; if `ev` is a dict, records (start, end) events per call kind."""
-    def rec(kind, fn):
-        if ev is None:
-            fn()
-            return
-        s = torch.cuda.Event(enable_timing=True)
-        e = torch.cuda.Event(enable_timing=True)
-        s.record()
-        fn()
-        e.record()
-        ev.setdefault(kind, []).append((s, e))
-
-    rec("requant", lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT) for l in layers], mode))
+    """One step.  If `ev` is a dict, CUDA events are recorded at the
+    boundaries between calls of different kinds (one event ends a run of
+    calls and starts the next, so a step carries 18 events for 21 launches);
+    ev[kind] collects (start, end, launches) per run of consecutive calls of
+    that kind."""
+    calls = [("requant", lambda: fb.fp8bw_requant_weights([(l.W, l.qw, l.sw, l.qwT) for l in layers], mode))]
     for l in layers:
-        rec("quant_act", lambda: fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc))
-        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode))
-        rec("quant_act", lambda: fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc))
-        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode))
-        rec("gemm", lambda: fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode))
+        calls += [
+            ("quant_act", lambda l=l: fb.fp8bw_quant_act_1x128(l.X, mode, l.qx, l.sx, l.qxc, l.sxc)),
+            ("gemm", lambda l=l: fb.fp8bw_gemm(fb.FP8BW_FPROP, l.qx, l.sx, l.qw, l.sw, l.Y, mode)),
+            ("quant_act", lambda l=l: fb.fp8bw_quant_act_1x128(l.dY, mode, l.qd, l.sd, l.qdc, l.sdc)),
+            ("gemm", lambda l=l: fb.fp8bw_gemm(fb.FP8BW_DGRAD, l.qd, l.sd, l.qwT, l.sw, l.dX, mode)),
+            ("gemm", lambda l=l: fb.fp8bw_gemm(fb.FP8BW_WGRAD, l.qdc, l.sdc, l.qxc, l.sxc, l.dW, mode)),
+        ]
+    if ev is None:
+        for _, fn in calls:
+            fn()
+        return
+
+    def event():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    start, n = event(), 0
+    for i, (kind, fn) in enumerate(calls):
+        fn()
+        n += 1
+        if i + 1 == len(calls) or calls[i + 1][0] != kind:
+            end = event()
+            ev.setdefault(kind, []).append((start, end, n))
+            start, n = end, 0
 
 
 LAUNCHES_PER_STEP = 1 + 4 * 5   # requant + per layer (2 quant_act + 3 gemm)
@@ -639,13 +652,13 @@ def main():
     value = job_rate(step_flops * args.steps, world, ms_total) / 1e12
 
     def kind_ms(k):
-        return sum(s.elapsed_time(e) for s, e in ev[k])
+        return sum(s.elapsed_time(e) for s, e, _ in ev[k])
 
     gemm_ms = kind_ms("gemm") / (args.steps)
     quant_ms = kind_ms("quant_act") / args.steps
     req_ms = kind_ms("requant") / args.steps
     gemm_tflops = step_flops / (gemm_ms * 1e-3) / 1e12
-    gemm_launch_ms = kind_ms("gemm") / len(ev["gemm"])
+    gemm_launch_ms = kind_ms("gemm") / sum(n for _, _, n in ev["gemm"])
     quant_bytes = sum(l.act_bytes(l.M, l.K) + l.act_bytes(l.M, l.N) for l in layers)
     req_bytes = sum(l.weight_bytes for l in layers)
     pk = peaks()
@@ -676,7 +689,7 @@ def main():
         st = fb.fp8bw_last_device_error()
         if st != 0:
             raise RuntimeError(f"device error (steady state): {fb.status_string(st)}")
-        g2_ms = sum(a.elapsed_time(b) for a, b in ev2["gemm"]) / n_steady
+        g2_ms = sum(a.elapsed_time(b) for a, b, _ in ev2["gemm"]) / n_steady
         g2_tflops = step_flops / (g2_ms * 1e-3) / 1e12
         steady = {"value": job_rate(step_flops * n_steady, world, q_ms) / 1e12, "unit": "TFLOP/s",
                   "ms_per_step": q_ms / n_steady, "steps": n_steady, "timed_s": q_ms / 1e3,

@@ -127,3 +127,49 @@ def test_act_e5m2(fb, orc, mode):
         assert_bytes_equal(f32(s_row).view(np.uint32), os_.view(np.uint32), "s_row")
         assert_bytes_equal(u8(q_col), oqc, "q_col")
         assert_bytes_equal(f32(s_col).view(np.uint32), osc.view(np.uint32), "s_col")
+
+
+def _every_amax_input(seed):
+    """[32768, 128] bf16: row i < 32639 is one 1x128 block whose magnitude
+    maximum is the positive bf16 with bit pattern i + 1 (placed at column
+    i % 128, sign random); the other elements have random magnitudes at or
+    below it and random signs.  Rows past 32639 are zero."""
+    rng = np.random.default_rng(seed)
+    n = 0x7F7F
+    top = np.arange(1, n + 1, dtype=np.uint32)
+    x = np.zeros((32768, 128), np.uint16)
+    mags = (rng.random((n, 128)) * (top[:, None] + 1)).astype(np.uint32)
+    mags = np.minimum(mags, top[:, None])
+    mags[np.arange(n), np.arange(n) % 128] = top
+    signs = rng.integers(0, 2, (n, 128), dtype=np.uint32) << 15
+    x[:n] = (mags | signs).astype(np.uint16)
+    return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16), top
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_act_every_bf16_amax(fb, orc, mode, fmt):
+    """Every positive finite bf16 block amax through the activation
+    quantizer: the row scales equal amax / qmax (one IEEE binary32 division)
+    or the power-of-2 rule, and codes and scales of both copies are
+    bit-exact against the oracle."""
+    x_cpu, top = _every_amax_input(21 + fmt)
+    x = x_cpu.to(DEV)
+    M, K = x.shape
+    q_row, s_row, q_col, s_col = act_buffers(M, K, DEV)
+    fb.fp8bw_quant_act_1x128_fmt(x, mode, fmt, q_row, s_row, q_col, s_col)
+    torch.cuda.synchronize()
+    assert fb.fp8bw_last_device_error() == 0
+    qmax = np.float32(448.0 if fmt == 0 else 57344.0)
+    amax = (top << 16).view(np.float32)
+    got = f32(s_row)[0, : len(top)]
+    if mode == 0:
+        assert np.array_equal(got.view(np.uint32), (amax / qmax).view(np.uint32))
+    else:
+        assert np.array_equal(got, np.array([orc.block_scale_fmt(float(a), 1, fmt) for a in amax],
+                                            np.float32))
+    oq, os_, oqc, osc = orc.quant_act_1x128(bits(x_cpu), mode, fmt=fmt)
+    assert_bytes_equal(u8(q_row), oq, "q_row")
+    assert_bytes_equal(f32(s_row).view(np.uint32), os_.view(np.uint32), "s_row")
+    assert_bytes_equal(u8(q_col), oqc, "q_col")
+    assert_bytes_equal(f32(s_col).view(np.uint32), osc.view(np.uint32), "s_col")
