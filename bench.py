@@ -89,56 +89,109 @@ def gemm_traffic():
 
 
 # ------------------------------------------------------------ clocks ------
-class ClockSampler:
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+def pci_bus_id(dev_index: int) -> str:
+    """PCI bus id of a CUDA device (CUDA_VISIBLE_DEVICES-proof handle for NVML
+    and nvidia-smi, whose indices are not CUDA's)."""
+    p = torch.cuda.get_device_properties(dev_index)
+    return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
 
-    def __init__(self, index: int):
-        self.index = index
+
+class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled in a background
+    thread every 10 ms through NVML (read-only queries), or every 100 ms by
+    nvidia-smi where NVML is unavailable.  Only the samples taken between
+    begin() and end() (the timed region, on the host clock) are summarised."""
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev_index = dev_index
+        self.bus = pci_bus_id(dev_index)
+        self.samples = []          # (host time, sm MHz, set of active reasons)
+        self.max_mhz = None
+        self.window = [None, None]
+        self.kind = None
+        self._stop = threading.Event()
+        self.thread = None
         self.proc = None
-        self.lines = []
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(self.bus)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            bits = dict(zip(self.NAMES, (pynvml.nvmlClocksEventReasonHwSlowdown,
+                                         pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                                         pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                                         pynvml.nvmlClocksEventReasonSwPowerCap)))
+
+            def poll():
+                while not self._stop.is_set():
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.perf_counter(), float(mhz),
+                                         {n for n, b in bits.items() if r & b}))
+                    self._stop.wait(0.01)
+                pynvml.nvmlShutdown()
+
+            self.kind = "nvml, 10 ms"
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # no NVML: nvidia-smi by bus id
+            pass
+        try:
+            q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+                ["nvidia-smi", "-i", self.bus, f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+            def read():
+                for line in self.proc.stdout:
+                    f = [x.strip() for x in line.split(",")]
+                    try:
+                        mhz, self.max_mhz = float(f[0]), float(f[1])
+                    except (ValueError, IndexError):
+                        continue
+                    act = {n for n, v in zip(self.NAMES, f[2:6]) if v.lower() == "active"}
+                    self.samples.append((time.perf_counter(), mhz, act))
+
+            self.kind = "nvidia-smi, 100 ms"
+            self.thread = threading.Thread(target=read, daemon=True)
             self.thread.start()
         except OSError:
-            self.proc = None
+            self.kind = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def begin(self):
+        self.window[0] = time.perf_counter()
+
+    def end(self):
+        self.window[1] = time.perf_counter()
 
     def stop(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 7:
-                continue
+        if self.kind is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no NVML or nvidia-smi"]}
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.thread.join(timeout=2)
+        t0, t1 = self.window
+        inside = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not inside and self.samples:  # region shorter than the interval: the last sample before its end
+            before = [x for x in self.samples if t1 is None or x[0] <= t1]
+            inside = before[-1:] or self.samples[:1]
+        reasons = set()
+        for x in inside:
+            reasons |= x[2]
+        mhz = [x[1] for x in inside]
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz), "sampler": self.kind}
 
 
 # ----------------------------------------------------------- workload -----
@@ -627,7 +680,7 @@ def main():
     assert fb.fp8bw_last_device_error() == 0
 
     # ---- timed region: K steps, per-call events, clocks sampled meanwhile
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     ev = {}
@@ -635,11 +688,13 @@ def main():
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    clocks.begin()
     t0.record()
     for _ in range(args.steps):
         run_step(fb, layers, mode, ev)
     t1.record()
     torch.cuda.synchronize()
+    clocks.end()
     barrier()
     ck = clocks.stop()
     ms_total = t0.elapsed_time(t1)
@@ -662,7 +717,10 @@ def main():
     quant_bytes = sum(l.act_bytes(l.M, l.K) + l.act_bytes(l.M, l.N) for l in layers)
     req_bytes = sum(l.weight_bytes for l in layers)
     pk = peaks()
-    timed_long = ms_total > 1000.0
+    # Half a second in, the step already runs at the power-capped clock
+    # (median 1635 MHz over a 0.7 s region against 1965 max), so a region of
+    # that length is rated against the sustained figure.
+    timed_long = ms_total > 500.0
     fp8_peak = 2.0 * (pk["bf16_sustained"] if timed_long else pk["bf16_burst"])
 
     # ---- steady state: the same step timed for at least 1.5 s, so that the
@@ -671,18 +729,20 @@ def main():
     steady = None
     if not args.no_steady:
         n_steady = max(args.steps, int(np.ceil(1500.0 / ms_step)))
-        ck2 = ClockSampler(clocks.index)
+        ck2 = ClockSampler(local)
         ck2.start()
         time.sleep(0.3)
         ev2 = {}
         barrier()
         torch.cuda.synchronize()
         q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ck2.begin()
         q0.record()
         for _ in range(n_steady):
             run_step(fb, layers, mode, ev2)
         q1.record()
         torch.cuda.synchronize()
+        ck2.end()
         barrier()
         ck2s = ck2.stop()
         q_ms = max_over_ranks(q0.elapsed_time(q1), dist, dev)
