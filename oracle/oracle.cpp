@@ -684,7 +684,11 @@ void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
           if (e > -127 && amax <= 448.0 * std::ldexp(1.0, e - 1) * (1.0 + eta_s)) sb_alt = std::ldexp(1.0, e - 1);
           if (e < 127 && amax >= 448.0 * sb * (1.0 - eta_s)) sb_alt = std::ldexp(1.0, e + 1);
         } else {
+          // a block whose largest p is so small that amax / 448 underflows
+          // (p below ~2e-321, far below fp32's range) is treated like an
+          // all-zero block (s = 1): its codes are 0 under any positive scale
           sb = amax / 448.0;
+          if (!(sb > 0.0)) sb = 1.0;
         }
       }
       const float* svb = sv + (b0 / 128) * (static_cast<int64_t>(Hkv) * D) + static_cast<int64_t>(g) * D;

@@ -139,6 +139,33 @@ def test_dominating_key(orc):
     np.testing.assert_allclose(O[0], vhat, rtol=1e-12, atol=0)
 
 
+def test_block_below_the_scale_range(orc):
+    """A 128-key block far below the row's maximum: one key at e^-745 (p the
+    smallest subnormal double), the others at e^-800 (p = 0), so amax / 448
+    underflows to zero.  That block counts as all-zero (scale 1, every code
+    0), as it does in fp32, where all its p are exactly 0; dividing its
+    zero p by the underflowed scale would give 0/0.  Closed form: the other
+    block holds the one key with p = 1 (code 0x7E against s = 1/448, p^ = 1)
+    and keys at e^-745, so O = that key's V^ exactly."""
+    T = 256
+    dec = np.array([orc.e4m3_decode(c) for c in range(256)])
+    one, m_one, two = 0x38, 0xB8, 0x40                  # E4M3 codes of 1, -1, 2
+    assert (dec[one], dec[m_one], dec[two]) == (1.0, -1.0, 2.0)
+    q = np.full((T, D), one, np.uint8)
+    sq = np.full((1, T), 1.0 / 128, np.float32)          # q^ . k^ s_q = k^: z_j = k^_j s_kj / sqrt(128)
+    k = np.full((T, D), m_one, np.uint8)
+    sk = np.full((1, T), np.float32(745.0 * math.sqrt(D)), np.float32)   # z_j ~ -745
+    sk[0, 1:128] = np.float32(800.0 * math.sqrt(D))     # z_j ~ -800: p = 0 in double
+    k[128] = one
+    sk[0, 128] = np.float32(1e-3)                         # z_128 ~ 0: the row's maximum
+    vT = np.full((D, T), one, np.uint8)
+    vT[:, 128] = two
+    sv = np.ones((T // 128, D), np.float32)
+    O, oa, of = orc.attention_fwd_rows(q, sq, k, sk, vT, sv, 1, 1, [0, T], [T], False, [3], [0])
+    assert np.all(np.isfinite(O)) and np.all(np.isfinite(oa)) and np.all(np.isfinite(of))
+    assert np.array_equal(O[0], np.full(D, 2.0))
+
+
 def test_gqa_equals_replicated_heads(orc):
     Hq, Hkv, T = 4, 2, 256
     q, sq, k, sk, vT, sv = make_case(orc, T, Hq, Hkv, 8)
