@@ -33,7 +33,10 @@
 // At the end O / l is rounded to bf16 and stored; padding query rows get 0.
 // TMEM: S buffers at columns 0 and 128, the P.V product at 256, the output
 // accumulator at 384.  Every wait is bounded; a timeout latches an error bit
-// and the CTA leaves.
+// and the CTA leaves.  With power-of-2 scales the tensor core applies every
+// scale (k_attn_fwd_mx), and when Hq / Hkv is even a CTA takes two query
+// heads of one KV group (k_attn_fwd_mx2), so that one head's exponentials
+// overlap the other head's remaining softmax phases.
 
 #include "common.cuh"
 #include "tmap.cuh"
@@ -212,19 +215,23 @@ __device__ __forceinline__ bool pair_meet(Bars* bars, int q, int lane, uint32_t 
   return warp_wait(smem_u32(&bars->pair[q]), uses & 1);
 }
 
-// TMA producer (one thread): the Q tile once, then per 128-key block the K
-// tile [128 keys][128] and the V tile [128 channels][128 keys] into the
-// kStages ring, and the block's 128 key scales and 128 channel scales (bulk
-// copies) into the kScSlots ring.
-template <class Smem, class Bars>
+// TMA producer (one thread): the NQ Q tiles (heads h .. h+NQ-1, stored one
+// after another from sm.q) once, then per 128-key block the K tile [128
+// keys][128] and the V tile [128 channels][128 keys] into the kStages ring,
+// and the block's 128 key scales and 128 channel scales (bulk copies) into
+// the kScSlots ring.
+template <int NQ, class Smem, class Bars>
 __device__ __forceinline__ void attn_producer(Smem& sm, Bars* bars, const CUtensorMap* tmQ,
                                               const CUtensorMap* tmK, const CUtensorMap* tmV,
                                               const AttnArgs& a, int h, int g, int q0, int kb_first, int nb) {
   prefetch_tmap(tmQ);
   prefetch_tmap(tmK);
   prefetch_tmap(tmV);
-  mbar_arrive_expect_tx(smem_u32(&bars->q_full), kTile);
-  tma_load_2d(smem_u32(sm.q), tmQ, smem_u32(&bars->q_full), h * kD, q0);
+  mbar_arrive_expect_tx(smem_u32(&bars->q_full), NQ * kTile);
+  uint8_t* qdst = reinterpret_cast<uint8_t*>(&sm.q);
+#pragma unroll
+  for (int i = 0; i < NQ; ++i)
+    tma_load_2d(smem_u32(qdst + i * kTile), tmQ, smem_u32(&bars->q_full), (h + i) * kD, q0);
   for (int b = 0; b < nb; ++b) {
     const int kb = kb_first + b, s = b % kStages, sl = b % kScSlots;
     if (!mbar_wait(smem_u32(&bars->kv_empty[s]), ((b / kStages) & 1) ^ 1)) {
@@ -247,21 +254,22 @@ __device__ __forceinline__ void attn_producer(Smem& sm, Bars* bars, const CUtens
 }
 
 // The CTA's work: query block qb (heavy, late blocks launched first) of
-// head h, its segment and key blocks.  Validates the segment table (every
-// CTA; an invalid one latches FP8BW_ERR_DEVICE_CHECK and nothing is written)
-// and writes zeros for a query block that is all padding; done = true then.
-// Called by every thread (it synchronizes the CTA).
+// heads h .. h+HPC-1 (HPC query heads of one KV group), its segment and key
+// blocks.  Validates the segment table (every CTA; an invalid one latches
+// FP8BW_ERR_DEVICE_CHECK and nothing is written) and writes zeros for a
+// query block that is all padding; done = true then.  Called by every
+// thread (it synchronizes the CTA).
 struct AttnBlock {
   int qb, h, g, q0, j0, jreal, kb_first, nb;
   bool done;
 };
 
-template <int NT>
+template <int NT, int HPC = 1>
 __device__ __forceinline__ AttnBlock attn_block(const AttnArgs& a, int* s_seg) {
   AttnBlock w;
-  const int nqb = a.T / 128;
-  w.qb = nqb - 1 - (int)(blockIdx.x / a.Hq);
-  w.h = (int)(blockIdx.x % a.Hq);
+  const int nqb = a.T / 128, hgroups = a.Hq / HPC;
+  w.qb = nqb - 1 - (int)(blockIdx.x / hgroups);
+  w.h = (int)(blockIdx.x % hgroups) * HPC;
   w.g = w.h / (a.Hq / a.Hkv);
   w.q0 = w.qb * 128;
   w.done = false;
@@ -286,9 +294,10 @@ __device__ __forceinline__ AttnBlock attn_block(const AttnArgs& a, int* s_seg) {
     // the whole query block is padding: zeros
     uint16_t* orow_base = a.o + (size_t)w.h * kD;
     const size_t ostride = (size_t)a.Hq * kD;
-    for (int idx = threadIdx.x; idx < 128 * 8; idx += NT) {
-      const int r = idx >> 3, c = idx & 7;
-      st_global_v8(orow_base + (size_t)(w.q0 + r) * ostride + c * 16, make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0));
+    for (int idx = threadIdx.x; idx < HPC * 128 * 8; idx += NT) {
+      const int hh = idx / (128 * 8), r = (idx >> 3) & 127, c = idx & 7;
+      st_global_v8(orow_base + (size_t)(w.q0 + r) * ostride + hh * kD + c * 16, make_uint4(0, 0, 0, 0),
+                   make_uint4(0, 0, 0, 0));
     }
     w.done = true;
     return w;
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
-    if (lane == 0) attn_producer(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
+    if (lane == 0) attn_producer<1>(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
   } else if (warp == 1) {
     // ----------------------------------------------------- MMA issuer -----
     if (lane == 0) {
@@ -876,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
-    if (lane == 0) attn_producer(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
+    if (lane == 0) attn_producer<1>(sm, bars, &tmQ, &tmK, &tmV, a, h, g, q0, kb_first, nb);
   } else if (warp == 1) {
     // ----------------------------------------------------- MMA issuer -----
     if (lane == 0) {
@@ -964,6 +973,359 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------
+// Power-of-2 scales, two query heads per CTA.  With one query tile, the two
+// softmax warps of a TMEM lane quarter run the same phases at the same time
+// (they meet on every block's maximum), so the MUFU idles while they load S,
+// reduce, store P and rescale.  Here a CTA takes one 128-query block of two
+// query heads h, h+1 of the same KV group (they read the same K and V tiles
+// and share the causal mask), and each head has its own four softmax warps,
+// one per lane quarter, a thread owning a whole row (128 columns, no
+// meeting).  The two heads' warps share the schedulers, so one head's
+// exponentials overlap the other's remaining phases.  Per key block the MMA
+// warp computes S_A, S_B (one S buffer in TMEM, taken in turn: S_B is
+// issued once head A has read S_A), then O_A += P_A V^T and O_B += P_B V^T
+// for the previous block.  Numerics as in k_attn_fwd_mx (every scale
+// applied by the block-scaled MMA, integer running maximum, P codes against
+// it).  TMEM: S at 0, O_A at 128, O_B at 256, scale tiles (4 columns each)
+// from 384: Q (per head), K and V (two slots), P (per head, two slots).
+// Launched when Hq / Hkv is even.
+constexpr uint32_t kM2S = 0, kM2O = 128;              // O of head tl at kM2O + 128 tl
+constexpr uint32_t kM2Sfq = 384, kM2Sfk = 392, kM2Sfv = 400, kM2Sfp = 408;
+
+struct AttnBarsMx2 {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t sc_full[kScSlots], sc_empty[kScSlots];
+  uint64_t sfq_full, sfkv_full[2], sfkv_empty[2];
+  uint64_t s_full[2];              // [head]: its S is in the buffer
+  uint64_t s_empty;                // the buffer's last S has been read (four warps)
+  uint64_t p_full[2][2], p_empty[2][2];   // [head][slot]
+  uint64_t o_full[2];              // [head]: a P.V into its O is complete
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct AttnSmemMx2 {
+  uint8_t q[2][kTile];                 // 1024-aligned tiles first
+  uint8_t kv[kStages][2][kTile];
+  uint8_t p[2][2][kTile];              // [head][slot]
+  SfTile sfq[2], sfk[2], sfv[2], sfp[2][2];
+  ScSlot sc[kScSlots];
+  AttnBarsMx2 bars;
+};
+static_assert(sizeof(AttnSmemMx2) + 1024 <= 232448, "shared memory budget (two heads)");
+static_assert(kM2Sfp + 16 <= 512, "TMEM columns (two heads)");
+
+// Softmax and correction warps of k_attn_fwd_mx2: warps 4-7 own head h0,
+// warps 8-11 head h0 + 1; one query row per thread, all 128 columns.  Per
+// key block as attn_softmax_mx, without the exchange of partial maxima.
+__device__ __forceinline__ void attn_softmax_mx2(AttnSmemMx2& sm, AttnBarsMx2* bars, uint32_t tmem,
+                                                 const AttnArgs& a, int warp, int lane, int h0, int q0,
+                                                 int jreal, int kb_first, int nb) {
+  const int q = warp & 3, tl = (warp - 4) >> 2;   // lane quarter, head of the pair
+  const int i = q * 32 + lane, t = q0 + i;
+  constexpr float c = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+  const int jend = a.causal ? min(jreal, t + 1) : jreal;
+  const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+  const uint32_t to = tmem + lane_off + kM2O + 128 * tl;
+  float m = -INFINITY, lh = 0.0f;
+  bool ok = true;
+
+  for (int b = 0; b < nb && ok; ++b) {
+    const int kb = kb_first + b;
+    if (!warp_wait(smem_u32(&bars->s_full[tl]), b & 1)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    uint32_t r[4][32];
+    tmem_ld64(tmem + lane_off + kM2S, r[0], r[1]);
+    tmem_ld64(tmem + lane_off + kM2S + 64, r[2], r[3]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) tmem_fence_regs(r[u]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
+
+    const int lim = jend - kb * 128;             // columns >= lim are masked
+    if (lim < 128) {
+#pragma unroll
+      for (int j = 0; j < 128; ++j)
+        if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+    }
+    float mh;
+    {
+      float mg[16];
+#pragma unroll
+      for (int gi = 0; gi < 16; ++gi) {
+        const uint32_t* v = &r[gi >> 2][(8 * gi) & 31];
+        mg[gi] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                       fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                       fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+      }
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi) mg[gi] = fmaxf(mg[gi], mg[gi + 8]);
+      mh = fmax3(fmax3(mg[0], mg[1], mg[2]), fmax3(mg[3], mg[4], mg[5]), fmaxf(mg[6], mg[7]));
+    }
+    const float mb = mh * c;                     // the block's largest logit, log2 units
+    const float m_new = mb > m + kLazy ? ceilf(mb) : m;
+    const bool moved = m_new != m;
+    const float dm = m - m_new;                  // an integer, or -inf on the first block
+    const float alpha = moved ? (dm < -126.0f ? 0.0f : exp2i((int)dm)) : 1.0f;
+    m = m_new;
+    // P's power-of-2 block scale 2^e: the smallest e with 2^(mb - m) <= 448 2^e
+    int e = (int)ceilf((mb - m) - kLog2_448);
+    e = max(-127, min(127, e));
+    const float sp = e == -127 ? __uint_as_float(0x00400000u) : exp2i(e);
+    const float2 c2 = make_float2(c, c);
+    const float off = -(m + (float)e);
+    const float2 nm2 = make_float2(off, off);
+    float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int j = 0; j < 128; j += 2) {
+      const int u = j >> 5, k = j & 31;
+      const float2 z = ffma2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), c2, nm2);
+      const float2 pj = make_float2(ex2(z.x), ex2(z.y));
+      r[u][k] = __float_as_uint(pj.x);
+      r[u][k + 1] = __float_as_uint(pj.y);
+      ps2[(j >> 1) & 3] = fadd2(ps2[(j >> 1) & 3], pj);
+    }
+    const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+    lh = lh * alpha + sp * (psum.x + psum.y);
+    uint32_t w[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int u = j >> 3, k = 4 * (j & 7);
+      w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])) |
+             (cvt_e4m3x2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])) << 16);
+    }
+    if (!warp_wait(smem_u32(&bars->p_empty[tl][b & 1]), ((b >> 1) & 1) ^ 1)) {
+      ok = false;
+      break;
+    }
+    // row i of the P tile: 16-byte chunk cc at cc ^ (i & 7) (128-byte swizzle)
+    uint8_t* prow = sm.p[tl][b & 1] + i * 128;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+      *reinterpret_cast<uint4*>(prow + ((cc ^ (i & 7)) << 4)) =
+          make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+    sm.sfp[tl][b & 1].w[i & 31][i >> 5] = (uint32_t)(e + 127) * 0x01010101u;
+    if (b >= 1) {
+      // the previous P.V of this head is complete; rescale O if a row moved
+      if (!warp_wait(smem_u32(&bars->o_full[tl]), (b - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t o[32];
+          tmem_ld32(to + 32 * u, o);
+          tmem_wait_ld();
+          tmem_fence_regs(o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(to + 32 * u, o);
+        }
+        tmem_wait_st();
+      }
+    }
+    fence_proxy_async_smem();   // the P tile and scale bytes, for the MMA
+    tc_fence_before();          // the rescaled O, for the MMA that accumulates onto it
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[tl][b & 1]));
+    if (bars->abort) ok = false;
+  }
+  if (ok && !warp_wait(smem_u32(&bars->o_full[tl]), (nb - 1) & 1)) ok = false;
+  tc_fence_after();
+  if (!ok) raise_attn_timeout(bars);
+  const bool real = t < jreal && ok;
+  const float il = real ? __fdiv_rn(1.0f, lh) : 0.0f;
+  uint16_t* orow = a.o + (size_t)(h0 + tl) * kD + (size_t)t * ((size_t)a.Hq * kD);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t o[32];
+    tmem_ld32(to + 32 * u, o);
+    tmem_wait_ld();
+    tmem_fence_regs(o);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t o8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o8[j] = real ? pack_bf16x2(__uint_as_float(o[16 * cc + 2 * j]) * il,
+                                   __uint_as_float(o[16 * cc + 2 * j + 1]) * il)
+                     : 0u;
+      st_global_v8(orow + 32 * u + 16 * cc, make_uint4(o8[0], o8[1], o8[2], o8[3]),
+                   make_uint4(o8[4], o8[5], o8[6], o8[7]));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd_mx2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  static_assert(kSoftWarps == 8, "four softmax warps per head of the pair");
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmemMx2& sm = *reinterpret_cast<AttnSmemMx2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                    ~uintptr_t(1023));
+  AttnBarsMx2* bars = &sm.bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_seg;
+  const AttnBlock wk = attn_block<kThreads, 2>(a, &s_seg);
+  if (wk.done) return;
+  const int h0 = wk.h, g = wk.g, q0 = wk.q0, jreal = wk.jreal;
+  const int kb_first = wk.kb_first, nb = wk.nb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->kv_full[i]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < kScSlots; ++i) {
+      mbar_init(smem_u32(&bars->sc_full[i]), 1);
+      mbar_init(smem_u32(&bars->sc_empty[i]), 1);   // read by the scale converter only
+    }
+    mbar_init(smem_u32(&bars->sfq_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->sfkv_full[i]), 1);
+      mbar_init(smem_u32(&bars->sfkv_empty[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->o_full[i]), 1);
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(smem_u32(&bars->p_full[i][j]), 4);
+        mbar_init(smem_u32(&bars->p_empty[i][j]), 1);
+      }
+    }
+    mbar_init(smem_u32(&bars->s_empty), 4);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) attn_producer<2>(sm, bars, &tmQ, &tmK, &tmV, a, h0, g, q0, kb_first, nb);
+  } else if (warp == 1) {
+    // ----------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_mx(128, 128, 0);   // E4M3 x E4M3, UE8M0 scales, byte 0
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0) && mbar_wait(smem_u32(&bars->sfq_full), 0);
+      tc_fence_after();
+      if (ok) {
+        tmem_cp_32x128b_x4(tmem + kM2Sfq, sdesc_k_noswz_16B(smem_u32(&sm.sfq[0].w[0][0])));
+        tmem_cp_32x128b_x4(tmem + kM2Sfq + 4, sdesc_k_noswz_16B(smem_u32(&sm.sfq[1].w[0][0])));
+      }
+      const uint64_t dq0 = sdesc_k_sw128(smem_u32(sm.q[0])), dq1 = sdesc_k_sw128(smem_u32(sm.q[1]));
+      uint32_t suse = 0;   // S computations so far (the buffer alternates between the heads)
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
+          const int s = b % kStages;
+          if (!mbar_wait(smem_u32(&bars->kv_full[s]), (b / kStages) & 1) ||
+              !mbar_wait(smem_u32(&bars->sfkv_full[b & 1]), (b >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tk = tmem + kM2Sfk + 4 * (b & 1);
+          tmem_cp_32x128b_x4(tk, sdesc_k_noswz_16B(smem_u32(&sm.sfk[b & 1].w[0][0])));
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.kv[s][0]));
+          for (int tl = 0; tl < 2 && ok; ++tl) {
+            // the previous S (the other head's, or this one's last block) has been read
+            if (!mbar_wait(smem_u32(&bars->s_empty), (suse & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_mx(tmem + kM2S, (tl ? dq1 : dq0) + 2 * kk, dk + 2 * kk, idesc, tmem + kM2Sfq + 4 * tl, tk,
+                      kk > 0 ? 1u : 0u);
+            umma_commit(smem_u32(&bars->s_full[tl]));
+            ++suse;
+          }
+          if (!ok) break;
+        }
+        if (b >= 1) {
+          const int c = b - 1, s = c % kStages;
+          const uint32_t tv = tmem + kM2Sfv + 4 * (c & 1);
+          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.kv[s][1]));
+          for (int tl = 0; tl < 2 && ok; ++tl) {
+            if (!mbar_wait(smem_u32(&bars->p_full[tl][c & 1]), (c >> 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t tp = tmem + kM2Sfp + 8 * tl + 4 * (c & 1);
+            tmem_cp_32x128b_x4(tp, sdesc_k_noswz_16B(smem_u32(&sm.sfp[tl][c & 1].w[0][0])));
+            if (tl == 0) tmem_cp_32x128b_x4(tv, sdesc_k_noswz_16B(smem_u32(&sm.sfv[c & 1].w[0][0])));
+            const uint64_t dp = sdesc_k_sw128(smem_u32(sm.p[tl][c & 1]));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_mx(tmem + kM2O + 128 * tl, dp + 2 * kk, dv + 2 * kk, idesc, tp, tv,
+                      (c > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(smem_u32(&bars->p_empty[tl][c & 1]));
+            umma_commit(smem_u32(&bars->o_full[tl]));
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&bars->kv_empty[s]));
+          umma_commit(smem_u32(&bars->sfkv_empty[c & 1]));
+        }
+        if (bars->abort) break;
+      }
+      if (!ok) raise_attn_timeout(bars);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ scale converter -----
+    bool bad = sf_tile(a.sq + (size_t)h0 * a.T + q0, &sm.sfq[0], lane);
+    bad |= sf_tile(a.sq + (size_t)(h0 + 1) * a.T + q0, &sm.sfq[1], lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->sfq_full));
+    for (int b = 0; b < nb; ++b) {
+      const int sl = b % kScSlots;
+      if (!warp_wait(smem_u32(&bars->sc_full[sl]), (b / kScSlots) & 1) ||
+          !warp_wait(smem_u32(&bars->sfkv_empty[b & 1]), ((b >> 1) & 1) ^ 1)) {
+        if (lane == 0) raise_attn_timeout(bars);
+        break;
+      }
+      bad |= sf_tile(sm.sc[sl].sk, &sm.sfk[b & 1], lane);
+      bad |= sf_tile(sm.sc[sl].sv, &sm.sfv[b & 1], lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bars->sfkv_full[b & 1]));
+        mbar_arrive(smem_u32(&bars->sc_empty[sl]));
+      }
+      if (bars->abort) break;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_attn_error, DEV_ERR_CHECK);
+  }
+  } else {
+    regs_inc<kRegsHigh>();
+    attn_softmax_mx2(sm, bars, tmem, a, warp, lane, h0, q0, jreal, kb_first, nb);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int32_t* d_off,
@@ -993,8 +1355,11 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
   a.sv = sv;
   a.o = static_cast<uint16_t*>(o);
   const bool mx = mode == FP8BW_SCALE_POW2;
-  const void* kern = mx ? reinterpret_cast<const void*>(k_attn_fwd_mx) : reinterpret_cast<const void*>(k_attn_fwd);
-  const size_t smem = (mx ? sizeof(AttnSmemMx) : sizeof(AttnSmem)) + 1024;
+  const bool pair = mx && (Hq / Hkv) % 2 == 0;   // two query heads of one KV group per CTA
+  const void* kern = pair ? reinterpret_cast<const void*>(k_attn_fwd_mx2)
+                   : mx   ? reinterpret_cast<const void*>(k_attn_fwd_mx)
+                          : reinterpret_cast<const void*>(k_attn_fwd);
+  const size_t smem = (pair ? sizeof(AttnSmemMx2) : mx ? sizeof(AttnSmemMx) : sizeof(AttnSmem)) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes attr;
@@ -1003,8 +1368,9 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
   // setmaxnreg draws on the launch allocation: refuse to launch if the
   // compiled register count could not cover the split.
   if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-  const unsigned grid = (unsigned)((T / 128) * Hq);
-  if (mx) k_attn_fwd_mx<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  const unsigned grid = (unsigned)((T / 128) * (pair ? Hq / 2 : Hq));
+  if (pair) k_attn_fwd_mx2<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  else if (mx) k_attn_fwd_mx<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   else k_attn_fwd<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }

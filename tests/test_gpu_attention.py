@@ -72,22 +72,24 @@ def test_attention_tiny_all_rows(fb, orc, causal, mode):
     assert torch.all(o[200:256] == 0)
 
 
+@pytest.mark.parametrize("heads", [(2, 2), (4, 2)])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_attention_ragged_segments(fb, orc, mode):
+def test_attention_ragged_segments(fb, orc, mode, heads):
     """Odd lengths, an empty segment, a one-token sequence and tokens past
-    the last segment (zeros); Hq = Hkv (no grouping); scales spread over
+    the last segment (zeros); Hq = Hkv (no grouping) and two query heads per
+    KV head (in power-of-2 mode the two-head kernel); scales spread over
     orders of magnitude (some rows scaled by 2^-20, some by 2^12)."""
     g = torch.Generator(device="cpu").manual_seed(2)
-    T, H = 1024, 2
-    Q = torch.randn((T, H * D), generator=g)
+    T, (Hq, Hkv) = 1024, heads
+    Q = torch.randn((T, Hq * D), generator=g)
     Q[::7] *= 2.0 ** -20
     Q[3::11] *= 2.0 ** 12
-    K = torch.randn((T, H * D), generator=g)
+    K = torch.randn((T, Hkv * D), generator=g)
     K[5::13] *= 2.0 ** -10
-    V = torch.randn((T, H * D), generator=g)
+    V = torch.randn((T, Hkv * D), generator=g)
     Q, K, V = (x.to(torch.bfloat16).to(DEV) for x in (Q, K, V))
     off, ln = [0, 384, 384, 512, 640, 896], [301, 0, 1, 128, 255]
-    rows = [(t, h) for t in list(range(0, 400)) + list(range(500, 1024, 3)) for h in range(H)]
+    rows = [(t, h) for t in list(range(0, 400)) + list(range(500, 1024, 3)) for h in range(Hq)]
     o = run_and_check(fb, orc, Q, K, V, off, ln, 1, rows, mode)
     assert torch.all(o[896:] == 0) and torch.all(o[301:384] == 0) and torch.all(o[385:512] == 0)
 
@@ -132,15 +134,18 @@ def test_attention_bad_offsets(fb, orc):
     assert fb.fp8bw_last_device_error() == 0
 
 
-def test_attention_pow2_rejects_other_scales(fb, orc):
+@pytest.mark.parametrize("hq", [1, 2])
+def test_attention_pow2_rejects_other_scales(fb, orc, hq):
     """Power-of-2 mode with scales from the FP32 rule (not powers of two):
     the kernel latches FP8BW_ERR_DEVICE_CHECK (o is undefined); the same
-    operands in FP32 mode are fine."""
-    T, H = 256, 1
+    operands in FP32 mode are fine.  One KV head with one query head, and
+    with two (the two-head kernel)."""
+    T = 256
     g = torch.Generator(device="cpu").manual_seed(5)
-    Q = torch.randn((T, H * D), generator=g).to(torch.bfloat16).to(DEV)
-    ops = quantize_qkv(fb, Q, Q, Q, 0)
-    o = torch.empty((T, H * D), dtype=torch.bfloat16, device=DEV)
+    Q = torch.randn((T, hq * D), generator=g).to(torch.bfloat16).to(DEV)
+    KV = Q[:, :D].contiguous()
+    ops = quantize_qkv(fb, Q, KV, KV, 0)
+    o = torch.empty((T, hq * D), dtype=torch.bfloat16, device=DEV)
     off = torch.tensor([0, T], dtype=torch.int32, device=DEV)
     ln = torch.tensor([T], dtype=torch.int32, device=DEV)
     fb.fp8bw_attention_fwd(*ops, o, off, ln, 1, 1)
