@@ -34,9 +34,9 @@
 // TMEM: S buffers at columns 0 and 128, the P.V product at 256, the output
 // accumulator at 384.  Every wait is bounded; a timeout latches an error bit
 // and the CTA leaves.  With power-of-2 scales the tensor core applies every
-// scale (k_attn_fwd_mx), and when Hq / Hkv is even a CTA takes two query
-// heads of one KV group (k_attn_fwd_mx2), so that one head's exponentials
-// overlap the other head's remaining softmax phases.
+// scale (k_attn_fwd_mx).  When Hq / Hkv is even a CTA takes two query heads
+// of one KV group instead (k_attn_fwd2, k_attn_fwd_mx2), so that one head's
+// exponentials overlap the other head's remaining softmax phases.
 
 #include "common.cuh"
 #include "tmap.cuh"
@@ -576,6 +576,351 @@ __global__ void __launch_bounds__(kThreads, 1)
           o8[j] = real ? pack_bf16x2(__uint_as_float(o[16 * c + 2 * j]) * il, __uint_as_float(o[16 * c + 2 * j + 1]) * il)
                        : 0u;
         st_global_v8(orow + 32 * u + 16 * c, make_uint4(o8[0], o8[1], o8[2], o8[3]),
+                     make_uint4(o8[4], o8[5], o8[6], o8[7]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------
+// FP32 scales, two query heads per CTA (the arrangement of k_attn_fwd_mx2
+// for k_attn_fwd's numerics).  A CTA takes one 128-query block of query
+// heads h, h+1 of one KV group; each head has four softmax warps (one per
+// lane quarter, a thread owning a whole row), so one head's exponentials
+// overlap the other's key scaling, P codes and folds.  TMEM: one S buffer
+// at 0 and one P.V product buffer at 128, each taken by the two heads in
+// turn; the output accumulators at 256 (head A) and 384 (head B).  Per key
+// block the MMA warp computes S_A, S_B, then P_A V^T and P_B V^T of the
+// previous block (P_B V^T once head A has read its product).  Launched
+// when Hq / Hkv is even.
+constexpr uint32_t kF2S = 0, kF2P = 128, kF2O = 256;   // O of head tl at kF2O + 128 tl
+
+struct AttnBars2 {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t sc_full[kScSlots], sc_empty[kScSlots];
+  uint64_t s_full[2];              // [head]: its S is in the buffer
+  uint64_t s_empty;                // the buffer's last S has been read (four warps)
+  uint64_t p_full[2][2], p_empty[2][2];   // [head][slot]
+  uint64_t o_full[2];              // [head]: its P.V product is in the product buffer
+  uint64_t o_empty;                // the product buffer's last product has been read
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct AttnSmem2 {
+  uint8_t q[2][kTile];                 // 1024-aligned tiles first
+  uint8_t kv[kStages][2][kTile];
+  uint8_t p[2][2][kTile];              // [head][slot]
+  ScSlot sc[kScSlots];
+  AttnBars2 bars;
+};
+static_assert(sizeof(AttnSmem2) + 1024 <= 232448, "shared memory budget (two heads, FP32 scales)");
+
+// Folds block c's P.V product of head tl into its accumulator (this
+// thread's row, all 128 columns): acc = acc * alpha + s_P * s_V[channel] *
+// O_c (acc = 0 before block 0).  The product is read whole first, so the
+// buffer goes back to the MMA before the arithmetic; then the block's scale
+// slot is released.  False if a wait ran out.
+__device__ __forceinline__ bool fold_block2(AttnSmem2& sm, AttnBars2* bars, uint32_t tmem, uint32_t lane_off,
+                                           int tl, int lane, int c, float alpha, float sp) {
+  if (!warp_wait(smem_u32(&bars->o_full[tl]), c & 1)) return false;
+  tc_fence_after();
+  const uint32_t tp = tmem + lane_off + kF2P, to = tmem + lane_off + kF2O + 128 * tl;
+  uint32_t pr[4][32];
+  tmem_ld64(tp, pr[0], pr[1]);
+  tmem_ld64(tp + 64, pr[2], pr[3]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int u = 0; u < 4; ++u) tmem_fence_regs(pr[u]);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars->o_empty));
+  const float2 sp2 = make_float2(sp, sp), a2 = make_float2(alpha, alpha);
+  const float4* sv4 = reinterpret_cast<const float4*>(sm.sc[c % kScSlots].sv);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t o[32];
+    if (c > 0) {
+      tmem_ld32(to + 32 * u, o);
+      tmem_wait_ld();
+      tmem_fence_regs(o);
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+      const float4 v = sv4[u * 8 + j4];
+      const float2 c0 = fmul2(sp2, make_float2(v.x, v.y));
+      const float2 c1 = fmul2(sp2, make_float2(v.z, v.w));
+      float2 o0 = make_float2(0.f, 0.f), o1 = make_float2(0.f, 0.f);
+      if (c > 0) {
+        o0 = fmul2(make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1])), a2);
+        o1 = fmul2(make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3])), a2);
+      }
+      o0 = ffma2(make_float2(__uint_as_float(pr[u][4 * j4]), __uint_as_float(pr[u][4 * j4 + 1])), c0, o0);
+      o1 = ffma2(make_float2(__uint_as_float(pr[u][4 * j4 + 2]), __uint_as_float(pr[u][4 * j4 + 3])), c1, o1);
+      o[4 * j4] = __float_as_uint(o0.x);
+      o[4 * j4 + 1] = __float_as_uint(o0.y);
+      o[4 * j4 + 2] = __float_as_uint(o1.x);
+      o[4 * j4 + 3] = __float_as_uint(o1.y);
+    }
+    tmem_st32(to + 32 * u, o);
+  }
+  tmem_wait_st();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars->sc_empty[c % kScSlots]));
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  static_assert(kSoftWarps == 8, "four softmax warps per head of the pair");
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmem2& sm = *reinterpret_cast<AttnSmem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+  AttnBars2* bars = &sm.bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_seg;
+  const AttnBlock wk = attn_block<kThreads, 2>(a, &s_seg);
+  if (wk.done) return;
+  const int h0 = wk.h, g = wk.g, q0 = wk.q0, jreal = wk.jreal;
+  const int kb_first = wk.kb_first, nb = wk.nb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->kv_full[i]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < kScSlots; ++i) {
+      mbar_init(smem_u32(&bars->sc_full[i]), 1);
+      mbar_init(smem_u32(&bars->sc_empty[i]), kSoftWarps);   // both heads' warps
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->o_full[i]), 1);
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(smem_u32(&bars->p_full[i][j]), 4);
+        mbar_init(smem_u32(&bars->p_empty[i][j]), 1);
+      }
+    }
+    mbar_init(smem_u32(&bars->s_empty), 4);
+    mbar_init(smem_u32(&bars->o_empty), 4);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) attn_producer<2>(sm, bars, &tmQ, &tmK, &tmV, a, h0, g, q0, kb_first, nb);
+  } else if (warp == 1) {
+    // ----------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0);
+      tc_fence_after();
+      const uint64_t dq0 = sdesc_k_sw128(smem_u32(sm.q[0])), dq1 = sdesc_k_sw128(smem_u32(sm.q[1]));
+      uint32_t suse = 0, ouse = 0;   // S and product computations so far (each buffer alternates)
+      for (int b = 0; ok && b <= nb; ++b) {
+        if (b < nb) {
+          const int s = b % kStages;
+          if (!mbar_wait(smem_u32(&bars->kv_full[s]), (b / kStages) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.kv[s][0]));
+          for (int tl = 0; tl < 2 && ok; ++tl) {
+            if (!mbar_wait(smem_u32(&bars->s_empty), (suse & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4(tmem + kF2S, (tl ? dq1 : dq0) + 2 * kk, dk + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+            umma_commit(smem_u32(&bars->s_full[tl]));
+            ++suse;
+          }
+          if (!ok) break;
+        }
+        if (b >= 1) {
+          const int c = b - 1, s = c % kStages;
+          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.kv[s][1]));
+          for (int tl = 0; tl < 2 && ok; ++tl) {
+            if (!mbar_wait(smem_u32(&bars->p_full[tl][c & 1]), (c >> 1) & 1) ||
+                !mbar_wait(smem_u32(&bars->o_empty), (ouse & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dp = sdesc_k_sw128(smem_u32(sm.p[tl][c & 1]));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8f6f4(tmem + kF2P, dp + 2 * kk, dv + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+            umma_commit(smem_u32(&bars->p_empty[tl][c & 1]));
+            umma_commit(smem_u32(&bars->o_full[tl]));
+            ++ouse;
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&bars->kv_empty[s]));
+        }
+        if (bars->abort) break;
+      }
+      if (!ok) raise_attn_timeout(bars);
+    }
+  }
+  } else {
+    regs_inc<kRegsHigh>();
+    // --------------------------------------------- softmax and correction --
+    const int q = warp & 3, tl = (warp - 4) >> 2;   // lane quarter, head of the pair
+    const int h = h0 + tl;
+    const int i = q * 32 + lane, t = q0 + i;
+    const float cq = a.sq[(size_t)h * a.T + t] * (kLog2e * 0.08838834764831845f);  // sq * log2(e) / sqrt(128)
+    const int jend = a.causal ? min(jreal, t + 1) : jreal;
+    float m = -INFINITY, lh = 0.0f;
+    float a_prev = 0.0f, sp_prev = 0.0f;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+
+    for (int b = 0; b < nb && ok; ++b) {
+      const int kb = kb_first + b;
+      if (!warp_wait(smem_u32(&bars->sc_full[b % kScSlots]), (b / kScSlots) & 1) ||
+          !warp_wait(smem_u32(&bars->s_full[tl]), b & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[4][32];
+      tmem_ld64(tmem + lane_off + kF2S, r[0], r[1]);
+      tmem_ld64(tmem + lane_off + kF2S + 64, r[2], r[3]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 4; ++u) tmem_fence_regs(r[u]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
+
+      // y = (q . k) * s_k per key; the query scale and 1/sqrt(d) log2(e)
+      // (cq > 0) are applied after the maximum
+      const int lim = jend - kb * 128;             // columns >= lim are masked
+      const float4* sk4 = reinterpret_cast<const float4*>(sm.sc[b % kScSlots].sk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 kv4 = sk4[u * 8 + j4];
+          const float2 p0 = fmul2(make_float2(__uint_as_float(r[u][4 * j4]), __uint_as_float(r[u][4 * j4 + 1])),
+                                  make_float2(kv4.x, kv4.y));
+          const float2 p1 = fmul2(make_float2(__uint_as_float(r[u][4 * j4 + 2]), __uint_as_float(r[u][4 * j4 + 3])),
+                                  make_float2(kv4.z, kv4.w));
+          r[u][4 * j4] = __float_as_uint(p0.x);
+          r[u][4 * j4 + 1] = __float_as_uint(p0.y);
+          r[u][4 * j4 + 2] = __float_as_uint(p1.x);
+          r[u][4 * j4 + 3] = __float_as_uint(p1.y);
+        }
+      }
+      if (lim < 128) {
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (j >= lim) r[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+      }
+      float mrow;
+      {
+        float mg[16];
+#pragma unroll
+        for (int gi = 0; gi < 16; ++gi) {
+          const uint32_t* v = &r[gi >> 2][(8 * gi) & 31];
+          mg[gi] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                         fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                         fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+        }
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi) mg[gi] = fmaxf(mg[gi], mg[gi + 8]);
+        mrow = fmax3(fmax3(mg[0], mg[1], mg[2]), fmax3(mg[3], mg[4], mg[5]), fmaxf(mg[6], mg[7]));
+      }
+      const float mb = mrow * cq;
+      const float m_new = fmaxf(m, mb);
+      const float alpha = ex2(m - m_new);       // 0 on the first block
+      m = m_new;
+      // P's block scale s_P = amax / 448, amax = 2^(mb - m) the block's
+      // largest p; the code input p / s_P = 2^(y * cq - mb + log2 448)
+      const float amax = ex2(mb - m_new);
+      const float sp = amax * (1.0f / 448.0f);
+      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(kLog2_448 - mb, kLog2_448 - mb);
+      float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int j = 0; j < 128; j += 2) {
+        const int u = j >> 5, k = j & 31;
+        const float2 z = ffma2(make_float2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])), cq2, nm2);
+        const float2 pj = make_float2(ex2(z.x), ex2(z.y));
+        r[u][k] = __float_as_uint(pj.x);
+        r[u][k + 1] = __float_as_uint(pj.y);
+        ps2[(j >> 1) & 3] = fadd2(ps2[(j >> 1) & 3], pj);
+      }
+      const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+      lh = lh * alpha + sp * (psum.x + psum.y);
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int u = j >> 3, k = 4 * (j & 7);
+        w[j] = cvt_e4m3x2(__uint_as_float(r[u][k]), __uint_as_float(r[u][k + 1])) |
+               (cvt_e4m3x2(__uint_as_float(r[u][k + 2]), __uint_as_float(r[u][k + 3])) << 16);
+      }
+      if (!warp_wait(smem_u32(&bars->p_empty[tl][b & 1]), ((b >> 1) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      // row i of the P tile: 16-byte chunk cc at cc ^ (i & 7) (128-byte swizzle)
+      uint8_t* prow = sm.p[tl][b & 1] + i * 128;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (i & 7)) << 4)) =
+            make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[tl][b & 1]));
+      if (b >= 1 && !fold_block2(sm, bars, tmem, lane_off, tl, lane, b - 1, a_prev, sp_prev)) ok = false;
+      a_prev = alpha;
+      sp_prev = sp;
+      if (bars->abort) ok = false;
+    }
+    if (ok && !fold_block2(sm, bars, tmem, lane_off, tl, lane, nb - 1, a_prev, sp_prev)) ok = false;
+    if (!ok) raise_attn_timeout(bars);
+    const bool real = t < jreal && ok;
+    const float il = real ? __fdiv_rn(1.0f, lh) : 0.0f;
+    uint16_t* orow = a.o + (size_t)h * kD + (size_t)t * ((size_t)a.Hq * kD);
+    const uint32_t to = tmem + lane_off + kF2O + 128 * tl;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t o[32];
+      tmem_ld32(to + 32 * u, o);
+      tmem_wait_ld();
+      tmem_fence_regs(o);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t o8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          o8[j] = real ? pack_bf16x2(__uint_as_float(o[16 * cc + 2 * j]) * il,
+                                     __uint_as_float(o[16 * cc + 2 * j + 1]) * il)
+                       : 0u;
+        st_global_v8(orow + 32 * u + 16 * cc, make_uint4(o8[0], o8[1], o8[2], o8[3]),
                      make_uint4(o8[4], o8[5], o8[6], o8[7]));
       }
     }
@@ -1355,11 +1700,13 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
   a.sv = sv;
   a.o = static_cast<uint16_t*>(o);
   const bool mx = mode == FP8BW_SCALE_POW2;
-  const bool pair = mx && (Hq / Hkv) % 2 == 0;   // two query heads of one KV group per CTA
-  const void* kern = pair ? reinterpret_cast<const void*>(k_attn_fwd_mx2)
-                   : mx   ? reinterpret_cast<const void*>(k_attn_fwd_mx)
-                          : reinterpret_cast<const void*>(k_attn_fwd);
-  const size_t smem = (pair ? sizeof(AttnSmemMx2) : mx ? sizeof(AttnSmemMx) : sizeof(AttnSmem)) + 1024;
+  const bool pair = (Hq / Hkv) % 2 == 0;   // two query heads of one KV group per CTA
+  const void* kern = mx ? (pair ? reinterpret_cast<const void*>(k_attn_fwd_mx2)
+                                : reinterpret_cast<const void*>(k_attn_fwd_mx))
+                        : (pair ? reinterpret_cast<const void*>(k_attn_fwd2)
+                                : reinterpret_cast<const void*>(k_attn_fwd));
+  const size_t smem = (mx ? (pair ? sizeof(AttnSmemMx2) : sizeof(AttnSmemMx))
+                          : (pair ? sizeof(AttnSmem2) : sizeof(AttnSmem))) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes attr;
@@ -1369,8 +1716,9 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
   // compiled register count could not cover the split.
   if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
   const unsigned grid = (unsigned)((T / 128) * (pair ? Hq / 2 : Hq));
-  if (pair) k_attn_fwd_mx2<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  if (mx && pair) k_attn_fwd_mx2<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   else if (mx) k_attn_fwd_mx<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  else if (pair) k_attn_fwd2<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   else k_attn_fwd<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
