@@ -89,6 +89,7 @@ def lib():
         L.orc_check_tol.restype = i64
         L.orc_attention_fwd_rows.argtypes = [i64, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp,
                                              vp, vp, i64, vp, vp, vp, vp, vp, i32]
+        L.orc_attention_decode.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.orc_set_threads.argtypes = [i32]
         L.orc_max_threads.restype = i32
         _lib = L
@@ -344,6 +345,26 @@ def attention_fwd_rows(q, sq, k, sk, vT, sv, Hq, Hkv, seg_off, seg_len, causal, 
                                  _p(q), _p(sq), _p(k), _p(sk), _p(vT), _p(sv), n, _p(rt), _p(rh),
                                  _p(out), _p(oa), _p(of), int(mode))
     return out, oa, of
+
+
+def attention_decode(q_bits, k, sk, v, sv, Hq, Hkv, lens, Lmax):
+    """FP8 KV-cache decode attention reference ("NVIDIA NeMo RL erreicht 48%
+    ...", "Leistungsgewinne in der Praxis": FP8 KV cache and attention in
+    generation): one bf16 query token per sequence, q_bits uint16 [B,
+    Hq*128]; the cache k, v [B*Lmax, Hkv*128] E4M3 codes with scales sk, sv
+    [Hkv, B*Lmax] (one per token and KV head); lens [B].  Returns (O, oabs,
+    oerr), each [B, Hq, 128] fp64 (oerr: the fp32 logit-error allowance)."""
+    q = _u16(q_bits)
+    k, v = _u8(k), _u8(v)
+    sk, sv = _f32(sk), _f32(sv)
+    B = q.shape[0]
+    ln = np.ascontiguousarray(lens, np.int32)
+    out = np.empty((B, int(Hq), HEAD_DIM), np.float64)
+    oa = np.empty_like(out)
+    oe = np.empty_like(out)
+    lib().orc_attention_decode(int(B), int(Hq), int(Hkv), int(Lmax), _p(ln), _p(q), _p(k), _p(sk),
+                               _p(v), _p(sv), _p(out), _p(oa), _p(oe))
+    return out, oa, oe
 
 
 def check_tol_attn(y_bits, oref, oabs, oflip, rel=REL_TOL):

@@ -722,4 +722,80 @@ void orc_attention_fwd_rows(int64_t T, int32_t Hq, int32_t Hkv, int32_t nseg,
   }
 }
 
+// FP8 KV-cache decode attention ["NVIDIA NeMo RL erreicht 48% ...",
+// "Leistungsgewinne in der Praxis": FP8 KV cache and attention in
+// generation].  One new query token per sequence attends to its cached keys.
+// The cache is the row-wise 1x128 quantization of the token matrix
+// [B*Lmax][Hkv*128]: one E4M3 code row and one fp32 scale per (token, KV
+// head), for K and for V alike; sequence b holds tokens b*Lmax .. b*Lmax +
+// len[b] - 1.  Scales are laid out [Hkv][B*Lmax].  The query is bf16
+// [B][Hq*128]; query head h reads KV head h / (Hq / Hkv).
+//   z_j = (q . k^_j) / sqrt(128),  k^_j = decode(k_j) * s_k,j
+//   O = sum_j e^(z_j - max z) v^_j / sum_j e^(z_j - max z)
+// in fp64, for every (b, h): out[(b*Hq + h)*128 + d].  A sequence with
+// len = 0 gives zeros.  oabs = sum_j p_j |v^_j| / l; oerr = 4 dzmax * oabs,
+// dzmax bounding the logit error of an fp32 kernel (the fp32 sum of the 128
+// exact products q_d * code, at most 2^-16 of their absolute sum, and the
+// two fp32 scalings, 2^-21 of |z|): each p and the sum l then carry at most
+// 2 dzmax relative error.
+void orc_attention_decode(int32_t B, int32_t Hq, int32_t Hkv, int64_t Lmax, const int32_t* len,
+                          const uint16_t* q, const uint8_t* k, const float* sk, const uint8_t* v,
+                          const float* sv, double* out, double* oabs, double* oerr) {
+  const int64_t D = 128;
+  const double* dec = decode_table(FMT_E4M3);
+  const double inv_sqrt_d = 1.0 / std::sqrt(static_cast<double>(D));
+  const int32_t group = Hq / Hkv;
+  const int64_t ld = static_cast<int64_t>(Hkv) * D;    // bytes per cache token row
+  const int64_t T = static_cast<int64_t>(B) * Lmax;    // tokens in the cache
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < static_cast<int64_t>(B) * Hq; ++r) {
+    const int64_t b = r / Hq;
+    const int32_t h = static_cast<int32_t>(r % Hq), g = h / group;
+    double* o = out + r * D;
+    double* oa = oabs + r * D;
+    double* oe = oerr + r * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = oa[d] = oe[d] = 0.0;
+    const int64_t L = len[b];
+    if (L <= 0) continue;
+    double qd[128];
+    for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_float(q[b * Hq * D + h * D + d]);
+    double* z = static_cast<double*>(std::malloc(sizeof(double) * L));
+    double zmax = -INFINITY, dzmax = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+      const int64_t row = b * Lmax + j;
+      double acc = 0.0, aabs = 0.0;
+      for (int64_t d = 0; d < D; ++d) {
+        const double prod = qd[d] * dec[k[row * ld + g * D + d]];
+        acc += prod;
+        aabs += std::fabs(prod);
+      }
+      const double c = static_cast<double>(sk[static_cast<int64_t>(g) * T + row]) * inv_sqrt_d;
+      z[j] = acc * c;
+      const double dz = std::fabs(c) * aabs * std::ldexp(1.0, -16) + std::fabs(z[j]) * std::ldexp(1.0, -21);
+      if (z[j] > zmax) zmax = z[j];
+      if (dz > dzmax) dzmax = dz;
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+      z[j] = std::exp(z[j] - zmax);   // z now holds p
+      l += z[j];
+    }
+    for (int64_t j = 0; j < L; ++j) {
+      const int64_t row = b * Lmax + j;
+      const double svj = sv[static_cast<int64_t>(g) * T + row];
+      for (int64_t d = 0; d < D; ++d) {
+        const double vv = dec[v[row * ld + g * D + d]] * svj;
+        o[d] += z[j] * vv;
+        oa[d] += z[j] * std::fabs(vv);
+      }
+    }
+    for (int64_t d = 0; d < D; ++d) {
+      o[d] /= l;
+      oa[d] /= l;
+      oe[d] = 4.0 * dzmax * oa[d];
+    }
+    std::free(z);
+  }
+}
+
 }  // extern "C"
