@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--case", default=None,
                    help="time one call only (for profiling): fprop|dgrad|wgrad|quant_x|quant_dy|attn|"
                         "requant|bf16_fprop|wgrad_acc|quant_delayed_dy|quant_delayed_x on --layer at "
-                        "--tokens, requant_sweep (32 layers), or "
+                        "--tokens, requant_sweep (32 layers), decode (FP8 KV-cache decode attention), or "
                         "moe_fprop|moe_dgrad|moe_wgrad "
                         "on the MoE expert layer --layer gate_up|down")
     p.add_argument("--sweep", action="store_true",
@@ -314,6 +314,28 @@ def attn_rates(fb, reps=10):
     return out
 
 
+def decode_rate(fb, hbm_gbs, reps=20):
+    """FP8 KV-cache decode attention (outside the timed step): GB/s of the
+    bytes one call reads and writes, 20 launches after 3 warm-up, against
+    the copy bandwidth."""
+    fn, work, _ = decode_call(fb)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / reps
+    del fn
+    torch.cuda.empty_cache()
+    gbs = work / (ms * 1e-3) / 1e9
+    return {"gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "ms": ms,
+            "workload": "64 rollouts, 16K-token FP8 KV cache (lengths 762-16048), 32 query / 8 KV heads of 128"}
+
+
 # ---------------------------------------------------------- CPU oracle ----
 _ORC = {}
 
@@ -497,6 +519,33 @@ def attn_call(fb, seed=0, mode=0):
     return (lambda: fb.fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, offd, lnd, 1, mode), flops, "TFLOP/s")
 
 
+def decode_call(fb, seed=0, mode=0):
+    """FP8 KV-cache decode attention: one new token for each of 64 rollouts
+    over a 16K-token cache (the seeded length mix of workloads.decode_lengths),
+    Llama-3.1-8B-like heads (32 query, 8 KV of 128); the cache quantized
+    row-wise by the library's activation quantizer.  Work = the bytes the
+    call must read or write: every cached token's K and V codes and scales
+    (sum_b len_b * Hkv * 2 * (128 + 4)), the bf16 queries and outputs."""
+    dev = torch.device("cuda", 0)
+    lens, Lmax = workloads.decode_lengths(seed)
+    B, Hq, Hkv, D = len(lens), 32, 8, 128
+    T = B * Lmax
+    u8, f32 = torch.uint8, torch.float32
+    e = lambda *sh, dt=u8: torch.empty(sh, dtype=dt, device=dev)  # noqa: E731
+    Q = workloads.normal_bf16((B, Hq * D), 1.0, 61, dev)
+    k, sk, v, sv = e(T, Hkv * D), e(Hkv, T, dt=f32), e(T, Hkv * D), e(Hkv, T, dt=f32)
+    X = workloads.normal_bf16((T, Hkv * D), 1.0, 62, dev)
+    fb.fp8bw_quant_act_1x128(X, mode, k, sk)
+    X = workloads.normal_bf16((T, Hkv * D), 1.0, 63, dev)
+    fb.fp8bw_quant_act_1x128(X, mode, v, sv)
+    del X
+    torch.cuda.empty_cache()
+    o = e(B, Hq * D, dt=torch.bfloat16)
+    lnd = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nbytes = sum(lens) * Hkv * 2 * (D + 4) + 2 * B * Hq * D * 2
+    return (lambda: fb.fp8bw_attention_decode(Q, k, sk, v, sv, o, lnd, Lmax), nbytes, "GB/s")
+
+
 def run_case(args):
     """Times a single call of one layer (used for ncu captures and sweeps)."""
     import blockwise_scaled_fp8_fp8bw_b200 as fb
@@ -512,6 +561,11 @@ def run_case(args):
         fn, work, unit = attn_call(fb, mode=mode)
         args.tokens = workloads.PACKED_TOKENS
         time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
+        return
+    if args.case == "decode":
+        fn, work, unit = decode_call(fb, mode=mode)
+        args.tokens = workloads.DECODE_BATCH
+        time_call(fb, args, "llama8b-decode-64x16k", mode, fn, work, unit)
         return
     if args.case == "requant_sweep":
         # the per-step requant of 32 layers x 4 weights (about 7B parameters)
@@ -589,6 +643,13 @@ def run_sweep(args):
         fn, work, unit = attn_call(fb, mode=mode)
         tokens, args.tokens = args.tokens, workloads.PACKED_TOKENS
         time_call(fb, args, "llama8b-packed-32k", mode, fn, work, unit)
+        args.tokens = tokens
+        del fn
+        torch.cuda.empty_cache()
+        args.case = "decode"
+        fn, work, unit = decode_call(fb, mode=mode)
+        tokens, args.tokens = args.tokens, workloads.DECODE_BATCH
+        time_call(fb, args, "llama8b-decode-64x16k", mode, fn, work, unit)
         args.tokens = tokens
         del fn
         torch.cuda.empty_cache()
@@ -782,6 +843,7 @@ def main():
     # ---- BF16 comparison GEMMs (outside the timed region)
     bf16 = bf16_ratio(fb, layers) if rank == 0 else None
     attn = attn_rates(fb) if rank == 0 else None
+    dec = decode_rate(fb, peaks()["hbm_gbs"]) if rank == 0 else None
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -888,7 +950,7 @@ def main():
                       "hbm_peak_gbs": pk["hbm_gbs"],
                       "bf16_gemm_tflops": bf16, "fp8_over_bf16": (gemm_tflops / bf16) if bf16 else None,
                       "requant_over_step": req_ms / ms_step,
-                      "attention_tflops": attn},
+                      "attention_tflops": attn, "attention_decode": dec},
             "steady_state": steady,
             "pow2_scales": pow2,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,

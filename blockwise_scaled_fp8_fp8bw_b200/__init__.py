@@ -71,7 +71,10 @@ def _load():
     L.fp8bw_gemm_quant.argtypes = [i32, i64, i64, i64, vp, vp, vp, vp, i32, vp, i64, vp, vp, vp, vp, vp]
     L.fp8bw_attention_fwd.argtypes = [i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp,
                                       ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8bw_attention_decode.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, i64, vp, vp, vp, vp,
+                                         vp, vp, vp, vp]
     for f in ("fp8bw_init", "fp8bw_last_device_error", "fp8bw_testing_stall_next_gemm", "fp8bw_attention_fwd",
+              "fp8bw_attention_decode",
               "fp8bw_gemm_quant",
               "fp8bw_quant_act_1x128", "fp8bw_quant_act_1x128_fmt", "fp8bw_gemm_fmt",
               "fp8bw_quant_weight_128x128", "fp8bw_requant_weights", "fp8bw_gemm",
@@ -252,6 +255,18 @@ def fp8bw_attention_fwd(q, sq, k, sk, vT, sv, o, seg_off, seg_len, causal=True, 
     _check("fp8bw_attention_fwd", load().fp8bw_attention_fwd(
         T, Hq, Hkv, seg_len.numel(), _ptr(seg_off), _ptr(seg_len), int(bool(causal)), int(mode), _ptr(q), _ptr(sq),
         _ptr(k), _ptr(sk), _ptr(vT), _ptr(sv), _ptr(o), _stream(stream)))
+
+
+def fp8bw_attention_decode(q, k, sk, v, sv, o, lens, Lmax, stream=None):
+    """FP8 KV-cache decode attention.  q [B, Hq*128] bf16 (one new token per
+    sequence); k, v [B*Lmax, Hkv*128] u8 cache codes, sk, sv [Hkv, B*Lmax]
+    fp32 (one scale per token and KV head); lens [B] device int32; o [B,
+    Hq*128] bf16."""
+    B = q.shape[0]
+    Hq, Hkv = q.shape[1] // 128, k.shape[1] // 128
+    _check("fp8bw_attention_decode", load().fp8bw_attention_decode(
+        B, Hq, Hkv, int(Lmax), _ptr(lens), _ptr(q), _ptr(k), _ptr(sk), _ptr(v), _ptr(sv), _ptr(o),
+        _stream(stream)))
 
 
 def fp8bw_gemm_quant(kind, A, sA, B, sB, q_row, s_row, q_col=None, s_col=None, D=None,

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libfp8bw.so")
-SOURCES = ["quant.cu", "quant_tensor.cu", "gemm.cu", "attention.cu", "api.cu"]
+SOURCES = ["quant.cu", "quant_tensor.cu", "gemm.cu", "attention.cu", "decode.cu", "api.cu"]
 HEADERS = ["common.cuh", "tmap.cuh", "blockquant.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -35,6 +35,10 @@ cudaError_t launch_attention_fwd(int64_t T, int Hq, int Hkv, int nseg, const int
 cudaError_t gemm_read_clear_error(uint32_t* out, cudaStream_t st);
 cudaError_t quant_read_clear_error(uint32_t* out, cudaStream_t st);
 cudaError_t attn_read_clear_error(uint32_t* out, cudaStream_t st);
+cudaError_t launch_attention_decode(int B, int Hq, int Hkv, int64_t Lmax, const int32_t* d_len,
+                                    const void* q, const uint8_t* k, const float* sk, const uint8_t* v,
+                                    const float* sv, void* o, cudaStream_t st);
+cudaError_t dec_read_clear_error(uint32_t* out, cudaStream_t st);
 extern int gemm_stall_chunk;
 }  // namespace fp8bw
 
@@ -115,12 +119,13 @@ FP8BW_API fp8bw_status fp8bw_testing_stall_next_gemm(int32_t chunk) {
 }
 
 FP8BW_API fp8bw_status fp8bw_last_device_error(fp8bw_stream_t stream) {
-  uint32_t v = 0, vq = 0, va = 0;
+  uint32_t v = 0, vq = 0, va = 0, vd = 0;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (fp8bw::gemm_read_clear_error(&v, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
   if (fp8bw::quant_read_clear_error(&vq, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
   if (fp8bw::attn_read_clear_error(&va, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
-  v |= vq | va;
+  if (fp8bw::dec_read_clear_error(&vd, cs) != cudaSuccess) return FP8BW_ERR_CUDA;
+  v |= vq | va | vd;
   if (v & 1u) return FP8BW_ERR_TIMEOUT;
   if (v & 2u) return FP8BW_ERR_DEVICE_CHECK;
   return FP8BW_OK;
@@ -389,6 +394,30 @@ FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, i
   if (T == 0) return FP8BW_OK;
   return from_cuda(fp8bw::launch_attention_fwd(T, Hq, Hkv, nseg, d_seg_off, d_seg_len, causal, (int)mode, q, sq, k,
                                                sk, vT, sv, o, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP8BW_API fp8bw_status fp8bw_attention_decode(int32_t B, int32_t Hq, int32_t Hkv, int64_t Lmax,
+                                              const int32_t* d_len, const void* q,
+                                              const uint8_t* k, const float* sk,
+                                              const uint8_t* v, const float* sv, void* o,
+                                              fp8bw_stream_t stream) {
+  if (!d_len || !q || !k || !sk || !v || !sv || !o) return FP8BW_ERR_INVALID_ARG;
+  if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || Lmax < 0) return FP8BW_ERR_INVALID_ARG;
+  const int32_t G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FP8BW_ERR_INVALID_ARG;
+  if (Hq > FP8BW_ATTN_MAX_HEADS || Lmax > kMaxDim || (int64_t)B * Lmax > kMaxDim ||
+      (int64_t)B * Hkv * 8 > (int64_t(1) << 31) - 1)
+    return FP8BW_ERR_TOO_LARGE;
+  if (!mult128(Lmax)) return FP8BW_ERR_ALIGNMENT;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(q) || !aligned16(sk) || !aligned16(sv) ||
+      !aligned4(d_len) || (reinterpret_cast<uintptr_t>(o) & 1u) != 0)
+    return FP8BW_ERR_ALIGNMENT;
+  int sms = 0;
+  fp8bw_status st = current(&sms);
+  if (st != FP8BW_OK) return st;
+  if (B == 0) return FP8BW_OK;
+  return from_cuda(fp8bw::launch_attention_decode(B, Hq, Hkv, Lmax, d_len, q, k, sk, v, sv, o,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -373,6 +373,36 @@ FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, i
                                            const uint8_t* k, const float* sk, const uint8_t* vT,
                                            const float* sv, void* o, fp8bw_stream_t stream);
 
+/* FP8 KV-cache decode attention ("NVIDIA NeMo RL erreicht 48% ...", section
+ * "Leistungsgewinne in der Praxis": FP8 for the KV cache and the attention
+ * operations of generation).  One new query token per sequence attends to
+ * the keys cached for it.  Head dimension 128.  The cache is the row-wise
+ * 1x128 quantization of its token matrix, as fp8bw_quant_act_1x128 (FP32 or
+ * power-of-2 scales, row-wise only) makes it:
+ *   k  [B*Lmax][Hkv*128] E4M3 codes, sk [Hkv][B*Lmax] fp32 scales (one per
+ *      token and KV head); sequence b owns rows b*Lmax .. b*Lmax + Lmax - 1,
+ *      of which the first len[b] are its cached tokens
+ *   v, sv  the same for V
+ *   q  [B][Hq*128] bf16, the new tokens' queries (not quantized)
+ *   o  [B][Hq*128] bf16 output.
+ * d_len is a DEVICE array [B] with 0 <= len[b] <= Lmax.  Query head h reads
+ * KV head h / (Hq / Hkv).  Per (b, h): z_j = (q . k^_j) / sqrt(128) with
+ * k^_j = E4M3(k_j) * s_k,j, p_j = exp(z_j - max z), o = sum_j p_j v^_j /
+ * sum_j p_j in bf16; len[b] = 0 gives zeros.  The kernel computes in fp32;
+ * the result is within |o - ref| <= 2^-10 * sum_j p_j |v^_j| / l + 4 dz *
+ * sum_j p_j |v^_j| / l + 1 bf16 ulp of the fp64 reference, dz = max_j
+ * (2^-16 |s_k,j| / sqrt(128) * sum_d |q_d E4M3(k_j,d)| + 2^-21 |z_j|) (the
+ * fp32 logit error).  A length outside [0, Lmax] latches
+ * FP8BW_ERR_DEVICE_CHECK and that sequence's output is not written.
+ * Requires Lmax a multiple of 128, Hq a multiple of Hkv with Hq / Hkv in
+ * {1, 2, 4, 8}, 16-byte aligned k, v, q, sk and sv, 4-byte aligned d_len,
+ * 2-byte aligned o.  All buffers are the caller's; nothing is allocated. */
+FP8BW_API fp8bw_status fp8bw_attention_decode(int32_t B, int32_t Hq, int32_t Hkv, int64_t Lmax,
+                                              const int32_t* d_len, const void* q,
+                                              const uint8_t* k, const float* sk,
+                                              const uint8_t* v, const float* sv, void* o,
+                                              fp8bw_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,10 @@ MOE_ZIPF = 1.1
 
 PACKED_TOKENS = 32768
 PACKED_NSEQ = 4
+# generation (decode) batch over an FP8 KV cache: rollouts of Llama-3.1-8B
+# ("NeMo-RL v0.3 mit Megatron-Core ...": 16K-token contexts)
+DECODE_BATCH = 64
+DECODE_LMAX = 16384
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -218,6 +222,14 @@ def packed_activations(K: int, seed: int = 0, device="cpu", total: int = PACKED_
     x = student_t_bf16((total, K), 3, scale, seed * 97 + K, device)
     x[~mask] = 0
     return x
+
+
+def decode_lengths(seed: int = 0, batch: int = DECODE_BATCH, lmax: int = DECODE_LMAX):
+    """(cache lengths [batch], Lmax) of a generation step: each rollout's
+    cached tokens (prompt plus tokens generated so far), uniform in
+    [256, lmax]."""
+    g = _gen(seed + 4242, "cpu")
+    return torch.randint(256, lmax + 1, (batch,), generator=g).tolist(), lmax
 
 
 def padded_shape(n: int, mult: int = 128) -> int:
