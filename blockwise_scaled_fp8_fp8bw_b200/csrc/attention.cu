@@ -312,8 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_align1024(smem_raw));
   AttnBars* bars = &sm.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -682,8 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   static_assert(kSoftWarps == 8, "four softmax warps per head of the pair");
   extern __shared__ uint8_t smem_raw[];
-  AttnSmem2& sm = *reinterpret_cast<AttnSmem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+  AttnSmem2& sm = *reinterpret_cast<AttnSmem2*>(smem_align1024(smem_raw));
   AttnBars2* bars = &sm.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int s_seg;
@@ -1183,8 +1181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd_mx(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  AttnSmemMx& sm = *reinterpret_cast<AttnSmemMx*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                  ~uintptr_t(1023));
+  AttnSmemMx& sm = *reinterpret_cast<AttnSmemMx*>(smem_align1024(smem_raw));
   AttnBarsMx* bars = &sm.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int s_seg;
@@ -1515,8 +1512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   static_assert(kSoftWarps == 8, "four softmax warps per head of the pair");
   extern __shared__ uint8_t smem_raw[];
-  AttnSmemMx2& sm = *reinterpret_cast<AttnSmemMx2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                    ~uintptr_t(1023));
+  AttnSmemMx2& sm = *reinterpret_cast<AttnSmemMx2*>(smem_align1024(smem_raw));
   AttnBarsMx2* bars = &sm.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int s_seg;

@@ -98,6 +98,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned byte of a dynamic shared array, as a pointer
+// into that array.  Adding an offset to the array keeps the shared address
+// space, so loads and stores through the result compile to shared-memory
+// instructions; a pointer rounded through an integer would be generic (each
+// access then a generic load or store, with its higher latency).
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  const uint32_t b = smem_u32(raw);
+  return raw + (((b + 1023u) & ~1023u) - b);
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

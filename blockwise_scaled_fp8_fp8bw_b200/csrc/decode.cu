@@ -120,8 +120,7 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  DecSmem<G>& sm = *reinterpret_cast<DecSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                  ~uintptr_t(1023));
+  DecSmem<G>& sm = *reinterpret_cast<DecSmem<G>*>(smem_align1024(smem_raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int cl = (int)(blockIdx.x / kNS);          // cluster = (sequence, KV head)

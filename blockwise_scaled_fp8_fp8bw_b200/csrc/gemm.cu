@@ -405,8 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // row (32x32b, PW = 2)
   constexpr int PW = QOUT ? 2 : 0;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + C::kStages * C::kStageBytes;  // 1024-aligned
   ScaleSlot* slots = reinterpret_cast<ScaleSlot*>(epi_base + 8 * C::kEpiBytes);
@@ -936,8 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
   using C = MxCfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + C::kStages * C::kStageBytes;
   ScaleSlot* raw = reinterpret_cast<ScaleSlot*>(epi_base + 8 * kMxEpiBufs * kEpiPiece);
@@ -1323,8 +1321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + kBf16Stages * kBf16StageBytes;
   Bf16Bars* bars = reinterpret_cast<Bf16Bars*>(epi_base + 8 * kBf16EpiBufs * kEpiPiece);

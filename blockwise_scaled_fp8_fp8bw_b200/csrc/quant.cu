@@ -84,8 +84,7 @@ __global__ void __launch_bounds__(QT, 3) k_quant_act(const __grid_constant__ CUt
                                                      uint8_t* __restrict__ q_col,
                                                      float* __restrict__ s_col) {
   extern __shared__ uint8_t smem_raw[];
-  ActSmem& sm = *reinterpret_cast<ActSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~uintptr_t(1023));
+  ActSmem& sm = *reinterpret_cast<ActSmem*>(smem_align1024(smem_raw));
   const int tid = threadIdx.x;
   const int rr = (tid & 7) + 8 * (tid >> 4), hh = (tid >> 3) & 1;  // row pass
   const int wc = tid & 63, rg = tid >> 6;                            // column pass
