@@ -626,9 +626,11 @@ static_assert(sizeof(AttnSmem2) + 1024 <= 232448, "shared memory budget (two hea
 // thread's row, all 128 columns): acc = acc * alpha + s_P * s_V[channel] *
 // O_c (acc = 0 before block 0).  The product is read whole first, so the
 // buffer goes back to the MMA before the arithmetic; then the block's scale
-// slot is released.  False if a wait ran out.
+// slot is released.  `rescale` (warp-uniform) is false when every row of
+// the warp has alpha = 1 (its running maximum did not move), and the
+// multiply by alpha is skipped: the same result.  False if a wait ran out.
 __device__ __forceinline__ bool fold_block2(AttnSmem2& sm, AttnBars2* bars, uint32_t tmem, uint32_t lane_off,
-                                           int tl, int lane, int c, float alpha, float sp) {
+                                           int tl, int lane, int c, float alpha, float sp, bool rescale) {
   if (!warp_wait(smem_u32(&bars->o_full[tl]), c & 1)) return false;
   tc_fence_after();
   const uint32_t tp = tmem + lane_off + kF2P, to = tmem + lane_off + kF2O + 128 * tl;
@@ -658,8 +660,12 @@ __device__ __forceinline__ bool fold_block2(AttnSmem2& sm, AttnBars2* bars, uint
       const float2 c1 = fmul2(sp2, make_float2(v.z, v.w));
       float2 o0 = make_float2(0.f, 0.f), o1 = make_float2(0.f, 0.f);
       if (c > 0) {
-        o0 = fmul2(make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1])), a2);
-        o1 = fmul2(make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3])), a2);
+        o0 = make_float2(__uint_as_float(o[4 * j4]), __uint_as_float(o[4 * j4 + 1]));
+        o1 = make_float2(__uint_as_float(o[4 * j4 + 2]), __uint_as_float(o[4 * j4 + 3]));
+        if (rescale) {
+          o0 = fmul2(o0, a2);
+          o1 = fmul2(o1, a2);
+        }
       }
       o0 = ffma2(make_float2(__uint_as_float(pr[u][4 * j4]), __uint_as_float(pr[u][4 * j4 + 1])), c0, o0);
       o1 = ffma2(make_float2(__uint_as_float(pr[u][4 * j4 + 2]), __uint_as_float(pr[u][4 * j4 + 3])), c1, o1);
@@ -793,6 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int jend = a.causal ? min(jreal, t + 1) : jreal;
     float m = -INFINITY, lh = 0.0f;
     float a_prev = 0.0f, sp_prev = 0.0f;
+    bool rs_prev = true;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;
 
@@ -893,12 +900,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[tl][b & 1]));
-      if (b >= 1 && !fold_block2(sm, bars, tmem, lane_off, tl, lane, b - 1, a_prev, sp_prev)) ok = false;
+      if (b >= 1 && !fold_block2(sm, bars, tmem, lane_off, tl, lane, b - 1, a_prev, sp_prev, rs_prev)) ok = false;
       a_prev = alpha;
       sp_prev = sp;
+      rs_prev = __any_sync(0xffffffffu, alpha != 1.0f);
       if (bars->abort) ok = false;
     }
-    if (ok && !fold_block2(sm, bars, tmem, lane_off, tl, lane, nb - 1, a_prev, sp_prev)) ok = false;
+    if (ok && !fold_block2(sm, bars, tmem, lane_off, tl, lane, nb - 1, a_prev, sp_prev, rs_prev)) ok = false;
     if (!ok) raise_attn_timeout(bars);
     const bool real = t < jreal && ok;
     const float il = real ? __fdiv_rn(1.0f, lh) : 0.0f;
