@@ -402,7 +402,7 @@ FP8BW_API fp8bw_status fp8bw_attention_decode(int32_t B, int32_t Hq, int32_t Hkv
                                               const uint8_t* v, const float* sv, void* o,
                                               fp8bw_stream_t stream) {
   if (!d_len || !q || !k || !sk || !v || !sv || !o) return FP8BW_ERR_INVALID_ARG;
-  if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || Lmax < 0) return FP8BW_ERR_INVALID_ARG;
+  if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || Lmax < 1) return FP8BW_ERR_INVALID_ARG;
   const int32_t G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FP8BW_ERR_INVALID_ARG;
   if (Hq > FP8BW_ATTN_MAX_HEADS || Lmax > kMaxDim || (int64_t)B * Lmax > kMaxDim ||

@@ -394,7 +394,7 @@ FP8BW_API fp8bw_status fp8bw_attention_fwd(int64_t T, int32_t Hq, int32_t Hkv, i
  * (2^-16 |s_k,j| / sqrt(128) * sum_d |q_d E4M3(k_j,d)| + 2^-21 |z_j|) (the
  * fp32 logit error).  A length outside [0, Lmax] latches
  * FP8BW_ERR_DEVICE_CHECK and that sequence's output is not written.
- * Requires Lmax a multiple of 128, Hq a multiple of Hkv with Hq / Hkv in
+ * Requires Lmax a positive multiple of 128, Hq a multiple of Hkv with Hq / Hkv in
  * {1, 2, 4, 8}, 16-byte aligned k, v, q, sk and sv, 4-byte aligned d_len,
  * 2-byte aligned o.  All buffers are the caller's; nothing is allocated. */
 FP8BW_API fp8bw_status fp8bw_attention_decode(int32_t B, int32_t Hq, int32_t Hkv, int64_t Lmax,

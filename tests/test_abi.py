@@ -109,6 +109,16 @@ def test_host_validation(lib):
     assert dl(p, 128, 128, 128, 0, 0, p, 16, p16, N, p, p, N, 0, N) == 2
     assert dl(p, 128, 128, 128, 0, 0, p, 16, q32, p16, p, p, N, 0, N) == 2
     assert dl(p, 128, 128, 128, 0, 0, ctypes.c_void_p(0x10002), 16, q32, N, p, p, N, 0, N) == 2
+    # KV-cache decode: null pointers, Hq not a multiple of Hkv, a group size
+    # outside {1, 2, 4, 8}, Lmax 0 or not a multiple of 128, misaligned scales
+    dec = r.fp8bw_attention_decode
+    assert dec(2, 4, 2, 128, N, p, p, p, p, p, p, N) == 1
+    assert dec(2, 6, 4, 128, p, p, p, p, p, p, p, N) == 1
+    assert dec(2, 12, 4, 128, p, p, p, p, p, p, p, N) == 1
+    assert dec(2, 32, 2, 128, p, p, p, p, p, p, p, N) == 1
+    assert dec(2, 4, 2, 0, p, p, p, p, p, p, p, N) == 1
+    assert dec(2, 4, 2, 200, p, p, p, p, p, p, p, N) == 2
+    assert dec(2, 4, 2, 128, p, p, p, ctypes.c_void_p(0x10004), p, p, p, N) == 2
     # testing hook: only chunk >= -1 is accepted; -1 cancels
     assert r.fp8bw_testing_stall_next_gemm(-2) == 1
     assert r.fp8bw_testing_stall_next_gemm(-1) == 0
