@@ -48,7 +48,13 @@ __device__ uint32_t g_dec_error;
 namespace {
 
 constexpr int kD = 128;
-constexpr int kNS = 8;                 // CTAs per (sequence, KV head): one cluster
+// CTAs per (sequence, KV head): one cluster.  Four measured faster than
+// eight (3.11-3.13 against 2.66-2.67 TB/s on the 64 x 16K rollout batch,
+// with the first round of loads issued before the query staging): a CTA's
+// fixed costs (barrier setup, query staging, the first loads' latency, the
+// merges) then spread over twice the keys.  Two ran the same as four, three
+// and six slower.
+constexpr int kNS = 4;
 // Eight consumer warps with one ring slot each (two CTAs per SM, 16
 // consumer warps): measured faster than four warps with two slots (2.11 vs
 // 1.97 TB/s on the 64 x 16K rollout batch) and than eight with two (one CTA
@@ -138,6 +144,20 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
   const int64_t row0 = (int64_t)b * a.Lmax;         // the sequence's first cache row
   const int h0 = g * G;
 
+  const float* skg = a.sk + (size_t)g * a.T + row0;
+  const float* svg = a.sv + (size_t)g * a.T + row0;
+  // tile t of this CTA (keys lo + 32 t ..): K and V boxes and both scale
+  // rows into consumer warp t % kCW's slot
+  auto issue = [&](int t) {
+    const int w = t % kCW, s = (t / kCW) % kSlots, j0 = lo + 32 * t;
+    const uint32_t full = smem_u32(&sm.bars.full[w][s]);
+    mbar_arrive_expect_tx(full, 2 * kTileB + 256);
+    tma_load_2d(smem_u32(sm.kt[w][s]), &tmK, full, g * kD, (int)(row0 + j0));
+    tma_load_2d(smem_u32(sm.vt[w][s]), &tmV, full, g * kD, (int)(row0 + j0));
+    bulk_load(smem_u32(sm.ks[w][s]), skg + j0, 128, full);
+    bulk_load(smem_u32(sm.vs[w][s]), svg + j0, 128, full);
+  };
+  const int first = min(ntile, kCW * kSlots);   // the first round: every slot starts empty
   if (threadIdx.x == 0) {
     for (int w = 0; w < kCW; ++w)
       for (int s = 0; s < kSlots; ++s) {
@@ -145,6 +165,10 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
         mbar_init(smem_u32(&sm.bars.empty[w][s]), 1);
       }
     fence_barrier_init();
+    // the first round's loads go out while the query rows are staged
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    for (int t = 0; t < first; ++t) issue(t);
   }
   for (int i = threadIdx.x; i < G * kD; i += kThreads) {
     const int h = i / kD, d = i % kD;
@@ -156,24 +180,14 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
     if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const float* skg = a.sk + (size_t)g * a.T + row0;
-      const float* svg = a.sv + (size_t)g * a.T + row0;
-      int t = 0;
+      int t = first;
       for (; t < ntile; ++t) {
         const int w = t % kCW, i = t / kCW, s = i % kSlots;
         if (!mbar_wait(smem_u32(&sm.bars.empty[w][s]), ((i / kSlots) & 1) ^ 1)) {
           atomicOr(&g_dec_error, DEV_ERR_TIMEOUT);
           break;
         }
-        const int j0 = lo + 32 * t;
-        const uint32_t full = smem_u32(&sm.bars.full[w][s]);
-        mbar_arrive_expect_tx(full, 2 * kTileB + 256);
-        tma_load_2d(smem_u32(sm.kt[w][s]), &tmK, full, g * kD, (int)(row0 + j0));
-        tma_load_2d(smem_u32(sm.vt[w][s]), &tmV, full, g * kD, (int)(row0 + j0));
-        bulk_load(smem_u32(sm.ks[w][s]), skg + j0, 128, full);
-        bulk_load(smem_u32(sm.vs[w][s]), svg + j0, 128, full);
+        issue(t);
       }
       // every copy issued has landed before the CTA goes on (bounded)
       for (int w = 0; w < kCW; ++w)
