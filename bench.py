@@ -292,24 +292,33 @@ def bf16_ratio(fb, layers, reps=3):
     return tot_flops / (tot_ms * 1e-3) / 1e12
 
 
-def attn_rates(fb, reps=10):
+def attn_rates(fb, dev_index=0, reps=10):
     """FP8 attention forward over the packed 32K-token batch in both scale
-    modes (outside the timed step): TFLOP/s of 10 launches after 3 warm-up."""
-    out = {}
+    modes (outside the timed step): TFLOP/s of 10 launches after 3 warm-up,
+    with the median SM clock sampled meanwhile (in the default run these
+    launches follow seconds of GEMM load, so the clock is the power-capped
+    one)."""
+    out, mhz = {}, {}
     for name, mode in (("fp32", 0), ("pow2", 1)):
         fn, work, _ = attn_call(fb, mode=mode)
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
+        ck = ClockSampler(dev_index)
+        ck.start()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ck.begin()
         s.record()
         for _ in range(reps):
             fn()
         e.record()
         torch.cuda.synchronize()
+        ck.end()
+        mhz[name] = ck.stop()["sm_mhz"]
         out[name] = work / (s.elapsed_time(e) / reps * 1e-3) / 1e12
         del fn
         torch.cuda.empty_cache()
+    out["sm_mhz"] = mhz
     out["workload"] = "packed 32768 tokens (4 sequences), 32 query / 8 KV heads of 128, causal"
     return out
 
@@ -842,7 +851,7 @@ def main():
 
     # ---- BF16 comparison GEMMs (outside the timed region)
     bf16 = bf16_ratio(fb, layers) if rank == 0 else None
-    attn = attn_rates(fb) if rank == 0 else None
+    attn = attn_rates(fb, local) if rank == 0 else None
     dec = decode_rate(fb, peaks()["hbm_gbs"]) if rank == 0 else None
 
     # ---- end to end through the C ABI with host buffers
