@@ -72,12 +72,13 @@ def test_attention_tiny_all_rows(fb, orc, causal, mode):
     assert torch.all(o[200:256] == 0)
 
 
-@pytest.mark.parametrize("heads", [(2, 2), (4, 2)])
+@pytest.mark.parametrize("heads", [(2, 2), (4, 2), (3, 1), (8, 1)])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_attention_ragged_segments(fb, orc, mode, heads):
     """Odd lengths, an empty segment, a one-token sequence and tokens past
-    the last segment (zeros); Hq = Hkv (no grouping) and two query heads per
-    KV head (in power-of-2 mode the two-head kernel); scales spread over
+    the last segment (zeros); Hq = Hkv (no grouping), two query heads per
+    KV head (the two-head kernels), three (an odd group: the one-head
+    kernels) and eight (four head pairs of one KV group); scales spread over
     orders of magnitude (some rows scaled by 2^-20, some by 2^12)."""
     g = torch.Generator(device="cpu").manual_seed(2)
     T, (Hq, Hkv) = 1024, heads
