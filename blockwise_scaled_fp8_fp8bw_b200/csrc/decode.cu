@@ -29,8 +29,8 @@
 //   P.V      lane = channels 4 lane .. 4 lane + 3: per key of the tile, its
 //            p * s_V from shared memory (broadcast) and the row's four codes.
 // The warps' states (m, l, o) are merged in shared memory, the cluster's
-// CTAs' states by CTA 0 through distributed shared memory, which writes
-// O / l in bf16.  A sequence with length 0 gives zeros.  Every mbarrier wait
+// CTAs' states through distributed shared memory, each CTA combining and
+// writing (O / l in bf16) its share of the outputs.  A sequence with length 0 gives zeros.  Every mbarrier wait
 // is bounded (a timeout latches an error bit); the producer waits, bounded,
 // for each of its copies before the CTA leaves; the two cluster barriers
 // are reached by every CTA of the cluster.
@@ -88,7 +88,7 @@ struct DecSmem {
   float pw[kCW][32][G];              // p * s_V of the warp's 32 keys
   float wm[kCW][G], wl[kCW][G];
   float wo[kCW][G][kD];              // the warps' partial outputs
-  float cm[G], cl[G];                // the CTA's state, read by CTA 0 of the cluster
+  float cm[G], cl[G];                // the CTA's state, read by every CTA of the cluster
   float co[G][kD];
   DecBars bars;
 };
@@ -317,11 +317,15 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
       sm.cl[h] = l;
     }
   }
-  // ---- merge the cluster's CTAs (CTA 0), then keep every CTA's shared
-  // memory alive until CTA 0 has read it
+  // ---- merge the cluster's CTAs: CTA r combines and writes the r-th
+  // kNS-th of the G x 128 outputs, reading every CTA's state through
+  // distributed shared memory; then every CTA's shared memory stays alive
+  // until all have read it
   cluster_sync();
-  if (rank == 0 && L >= 0) {
-    for (int i = threadIdx.x; i < G * kD; i += kThreads) {
+  if (L >= 0) {
+    constexpr int kPer = G * kD / kNS;
+    static_assert(G * kD % kNS == 0, "outputs split evenly over the cluster");
+    for (int i = (int)rank * kPer + threadIdx.x; i < ((int)rank + 1) * kPer; i += kThreads) {
       const int h = i / kD, d = i % kD;
       float cmr[kNS];
       float mx = -INFINITY;
