@@ -19,9 +19,10 @@
 // t % kCW.  The
 // consumer warps:
 //   logits   lane = key: its K row from shared memory (eight conflict-free
-//            16-byte loads thanks to the swizzle), decoded pairwise
-//            (E4M3 -> f16x2 -> f32) and dotted with the G query rows held
-//            as [dim][head] (broadcast loads; head pairs on packed fp32
+//            16-byte loads thanks to the swizzle), decoded four codes of a
+//            word at a time (E4M3 -> f16x2 -> f32, the word's 16-bit halves
+//            taken in place) and dotted with the G query rows held as
+//            [dim][head] (broadcast loads; head pairs on packed fp32
 //            lanes), times the key's scale;
 //   softmax  per head, online in log2 units (the query is pre-scaled by
 //            log2(e) / sqrt(128)): tile maximum across the warp, running
@@ -93,11 +94,24 @@ struct DecSmem {
   DecBars bars;
 };
 
-// Two E4M3 codes (low byte first) to floats, exactly (E4M3 -> f16 is exact).
-__device__ __forceinline__ float2 dec2(uint32_t pair) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(pair));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+// Four E4M3 codes (byte i of w is code i) to floats, exactly (E4M3 -> f16
+// is exact, f16 -> f32 too).  The word's 16-bit halves are taken as they
+// sit in the register (no mask or shift).
+__device__ __forceinline__ float4 dec4(uint32_t w) {
+  float4 r;
+  asm("{\n\t.reg .b16 lo, hi, a, b, c, d;\n\t.reg .b32 h01, h23;\n\t"
+      "mov.b32 {lo, hi}, %4;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h01, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h23, hi;\n\t"
+      "mov.b32 {a, b}, h01;\n\t"
+      "mov.b32 {c, d}, h23;\n\t"
+      "cvt.f32.f16 %0, a;\n\t"
+      "cvt.f32.f16 %1, b;\n\t"
+      "cvt.f32.f16 %2, c;\n\t"
+      "cvt.f32.f16 %3, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+      : "r"(w));
+  return r;
 }
 
 __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
@@ -230,8 +244,8 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
         const uint32_t ww[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float2 k01 = dec2(ww[u] & 0xFFFFu), k23 = dec2(ww[u] >> 16);
-          const float kv[4] = {k01.x, k01.y, k23.x, k23.y};
+          const float4 k4 = dec4(ww[u]);
+          const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
           const int d = 16 * c + 4 * u;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -273,7 +287,8 @@ __global__ void __launch_bounds__(kThreads) k_attn_decode(const __grid_constant_
 #pragma unroll 8
       for (int kk = 0; kk < n; ++kk) {
         const uint32_t vw = *reinterpret_cast<const uint32_t*>(vt + kk * 128 + (((lane >> 2) ^ (kk & 7)) << 4));
-        const float2 v01 = dec2(vw & 0xFFFFu), v23 = dec2(vw >> 16);
+        const float4 v4 = dec4(vw);
+        const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float wk = sm.pw[cw][kk][h];
