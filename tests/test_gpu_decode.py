@@ -65,13 +65,15 @@ def test_decode_all_rows(fb, orc, heads, mode):
     run_and_check(fb, orc, Q, *make_cache(fb, K, V, mode), lens, Lmax)
 
 
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1)])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_decode_long_cache_spread_scales(fb, orc, mode):
-    """16K-token caches (Llama-3.1-8B heads: 32 query over 8 KV), keys whose
-    rows are scaled by 2^-10 .. 2^8 and queries by up to 2^4, so logits
-    range over orders of magnitude; every row checked."""
+def test_decode_long_cache_spread_scales(fb, orc, mode, heads):
+    """16K-token caches (Llama-3.1-8B heads: 32 query over 8 KV; and eight
+    query heads over one KV head), keys whose rows are scaled by
+    2^-10 .. 2^8 and queries by up to 2^4, so logits range over orders of
+    magnitude; every row checked."""
     g = torch.Generator(device="cpu").manual_seed(44)
-    Hq, Hkv, Lmax = 32, 8, 16384
+    (Hq, Hkv), Lmax = heads, 16384
     lens = [16384, 9000, 1, 12345]
     B = len(lens)
     Q = torch.randn((B, Hq * D), generator=g) * (2.0 ** torch.randint(0, 5, (B, 1), generator=g))
